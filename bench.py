@@ -1,0 +1,412 @@
+#!/usr/bin/env python
+"""Benchmark of the sequence/head-parallel attention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload NAME]
+
+One step is one pass of the path over one batch of synthetic input (inputs resident in HBM):
+
+  video_dit (default)  B1 S32760 H40 D128, N(0,1)*0.5: Q, K, V as 4 sequence shards (simulated ranks);
+                       seq->head relayout of each, attention of every rank on its 10 heads with the head
+                       chunks [3,7,10,10,10] split at rank boundaries, head->seq relayout of O.
+  ring_causal          B1 S57344 H40 D128 causal: 8 KV-block partial launches + log-sum-exp merge.
+  block_sparse         B1 S32768 H40 D128, per-head tile mask of density U[0.1, 0.9]: tile list + attention.
+
+The metric is attention TFLOPS (4 B H S^2 D x density, halved when causal) over the step time; the
+relayout and merge GB/s are reported beside it under "kernels".  With N > 1 (torchrun, one rank per GPU)
+every rank runs its own batch (weak scaling, no data-path collective); time is the max over ranks.
+
+--impl reference times the fp64 CPU oracle (the only reference this path has) on the host cores, on a
+bounded sample of the same workload, and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention TFLOPS & % of bf16 tensor peak at S=32K–56K; relayout/merge GB/s"
+UNIT = "TFLOPS"
+
+
+# ----------------------------------------------------------------------------------------------------
+# distributed plumbing (NCCL on GPUs, gloo on CPU); used by the tests with gloo
+# ----------------------------------------------------------------------------------------------------
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")),
+            int(os.environ.get("LOCAL_RANK", "0")))
+
+
+def init_dist(backend: str, timeout_s: int = 120):
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return rank, world
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def finish_dist():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+def emit(line: dict, rank: int):
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=10)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[4:8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags) if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------------------------------
+# CPU oracle timing (the cpu_baseline of our arm, and the whole of the reference arm)
+# ----------------------------------------------------------------------------------------------------
+def oracle_sample(wname: str, q, k, v, mask, n_rows: int, heads, seed: int = 0, w=None):
+    """Run the fp64 oracle on n_rows sampled query rows of the given heads; return (seconds, flops,
+    threads, description).  FLOPs are counted like the metric: 4 * D per (row, visible key)."""
+    import numpy as np
+    import oracle
+    from sequence_head_attention_b200 import synth
+    w = w or synth.WORKLOADS[wname]
+    rows = synth.sample_rows(w.S, n_rows, seed=seed)[:n_rows]
+    hs = list(heads)
+    q64 = q[:, :, hs][:, rows].double().numpy()
+    k64 = k[:, :, hs].double().numpy()
+    v64 = v[:, :, hs].double().numpy()
+    m = None if mask is None else mask[hs].numpy()
+    # the oracle evaluates the chosen rows against all keys; Q is passed full-length with only the
+    # sampled rows filled in, so row indices keep their global positions
+    qfull = np.zeros((w.B, w.S, len(hs), w.D))
+    qfull[:, rows] = q64
+    nthreads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.attention(qfull, k64, v64, causal=w.causal, block_mask=m, rows=rows, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    if mask is not None:
+        keys = sum(int(mask[h, r // synth.TILE].sum()) * synth.TILE for h in hs for r in rows)
+    elif w.causal:
+        keys = sum(r + 1 for r in rows) * len(hs)
+    else:
+        keys = w.S * len(rows) * len(hs)
+    flops = 4.0 * w.D * keys * w.B
+    desc = f"{len(rows)} stratified query rows x {len(hs)} heads of {wname} (all keys), fp64"
+    return dt, flops, nthreads, desc
+
+
+def calibrated_oracle_baseline(wname, q, k, v, mask, target_s=15.0):
+    heads = list(range(0, q.shape[2], 5))[:8]
+    dt1, _, _, _ = oracle_sample(wname, q, k, v, mask, 4, heads)
+    n = int(max(4, min(2048, 4 * target_s / max(dt1, 1e-3))))
+    dt, flops, nthreads, desc = oracle_sample(wname, q, k, v, mask, n, heads)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": desc, "seconds": round(dt, 3)}
+
+
+# ----------------------------------------------------------------------------------------------------
+def build_inputs(wname: str, seed: int, seq_len: int = 0):
+    import dataclasses
+    from sequence_head_attention_b200 import synth
+    w = synth.WORKLOADS[wname]
+    if seq_len:
+        w = dataclasses.replace(w, S=seq_len)
+    q, k, v = synth.qkv(w.B, w.S, w.H, w.D, seed=seed, scale=w.scale)
+    mask = synth.block_mask(w.H, w.S, seed=seed) if w.sparse else None
+    return w, q, k, v, mask
+
+
+def config_of(w, wname, world, extra=None):
+    c = {"workload": f"{wname}: B{w.B} S{w.S} H{w.H} D{w.D}" + (" causal" if w.causal else ""),
+         "global_batch": w.B * world, "seq_len": w.S, "heads": w.H, "head_dim": w.D,
+         "parallelism": f"replicas{world}" if world > 1 else "single",
+         "l2": "inputs larger than L2 (Q, K, V >= 335 MB each); no flush"}
+    if wname == "video_dit":
+        c.update({"head_chunks": list(w.head_chunks), "simulated_ranks": w.ranks})
+    if wname == "ring_causal":
+        c.update({"kv_blocks": w.n_kv_blocks})
+    if extra:
+        c.update(extra)
+    return c
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0  # the CPU oracle runs once, on rank 0
+    w, q, k, v, mask = build_inputs(args.workload, seed=0)
+    heads = list(range(0, w.H, 5))[:8]
+    n_rows = args.ref_rows
+    for _ in range(args.warmup):
+        oracle_sample(args.workload, q, k, v, mask, n_rows, heads)
+    times, flops_total = [], 0.0
+    desc, nthreads = "", 1
+    for _ in range(args.steps):
+        dt, flops, nthreads, desc = oracle_sample(args.workload, q, k, v, mask, n_rows, heads)
+        times.append(dt)
+        flops_total += flops
+    total = sum(times)
+    value = flops_total / total / 1e12
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * total / max(1, args.steps), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": config_of(w, args.workload, 1), "impl": "reference",
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                             "sample": desc + " per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    emit(line, 0)
+    return 0
+
+
+def run_ours(args):
+    import torch
+    from sequence_head_attention_b200 import spattn, workloads
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl", timeout_s=180)
+    spattn.lib()  # fail now if the library is missing
+
+    w, q, k, v, mask = build_inputs(args.workload, seed=rank, seq_len=args.seq_len)
+    if args.workload == "video_dit":
+        step = workloads.UlyssesStep(w, q, k, v, device=dev)
+    elif args.workload == "ring_causal":
+        step = workloads.RingStep(w, q, k, v, device=dev)
+    else:
+        step = workloads.SparseStep(w, q, k, v, mask, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    E = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+
+    def timed_step(marks):
+        """One step with events around the phases: returns nothing; marks collects (name, ev0, ev1)."""
+        if args.workload == "video_dit":
+            a = E(); a.record(stream); step.relayout_in(); b = E(); b.record(stream)
+            marks.append(("relayout", a, b))
+            for r in range(step.P):
+                a = E(); a.record(stream)
+                spattn.sp_attn_fwd(step.q_head[r], step.k_head[r], step.v_head[r], step.o_head[r], step.lse[r],
+                                   head_chunks=step.chunks[r])
+                b = E(); b.record(stream)
+                marks.append(("attn", a, b))
+            a = E(); a.record(stream); step.relayout_out(); b = E(); b.record(stream)
+            marks.append(("relayout", a, b))
+        elif args.workload == "ring_causal":
+            a = E(); a.record(stream); step.attention(); b = E(); b.record(stream)
+            marks.append(("attn_all", a, b))
+            a = E(); a.record(stream); step.merge(); b = E(); b.record(stream)
+            marks.append(("merge", a, b))
+        else:
+            a = E(); a.record(stream); step.run(); b = E(); b.record(stream)
+            marks.append(("attn", a, b))
+
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize(dev)
+    if spattn.sp_check_device_error() != spattn.SP_OK:
+        raise SystemExit("device error during warm-up")
+
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    sampler = ClockSampler(gpu_id)
+    sampler.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize(dev)
+    marks = []
+    t_start, t_end = E(), E()
+    t_start.record(stream)
+    for _ in range(args.steps):
+        timed_step(marks)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    if spattn.sp_check_device_error() != spattn.SP_OK:
+        raise SystemExit("device error during the timed steps")
+    ms_local = t_start.elapsed_time(t_end)
+    ms = max_over_ranks(ms_local, device=dev)
+    total_flops = step.flops * args.steps * world
+    value = total_flops / (ms / 1000.0) / 1e12
+
+    peaks = measured_peaks()
+    phase = {}
+    for name, a, b in marks:
+        phase.setdefault(name, []).append(a.elapsed_time(b))
+    kernels = {}
+    if args.workload == "video_dit":
+        attn_ms = statistics.mean(phase["attn"])
+        flops_launch = step.flops / step.P
+        rl_ms = sum(phase["relayout"]) / args.steps  # both relayout phases of one step
+        rl_gbs = step.relayout_bytes / (rl_ms / 1000.0) / 1e9
+        kernels["relayout"] = {"gbs": rl_gbs, "ms_per_step": rl_ms, "bytes_per_step": step.relayout_bytes,
+                               "frac_of_measured_hbm": rl_gbs / peaks["hbm_gbs"]}
+    elif args.workload == "ring_causal":
+        attn_ms = statistics.mean(phase["attn_all"])
+        flops_launch = step.flops
+        m_ms = statistics.mean(phase["merge"])
+        kernels["merge"] = {"gbs": step.merge_bytes / (m_ms / 1000.0) / 1e9, "ms": m_ms,
+                            "bytes": step.merge_bytes,
+                            "frac_of_measured_hbm": step.merge_bytes / (m_ms / 1000.0) / 1e9 / peaks["hbm_gbs"]}
+    else:
+        attn_ms = statistics.mean(phase["attn"])
+        flops_launch = step.flops
+    achieved = flops_launch / (attn_ms / 1000.0) / 1e12
+    kernels["attention"] = {"tflops": achieved, "ms_per_launch": attn_ms}
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                "peak_kind": f"{peaks['source']} bf16 dense, sustained (kernel timed inside a long step)",
+                "frac_of_burst_peak": achieved / peaks["bf16_tflops"]}
+
+    # end to end: host buffers in pinned memory, copies inside the timed region
+    e2e = None
+    if not args.no_e2e:
+        ins, outs = step.inputs(), step.outputs()
+        h_in = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in ins]
+        for h, t in zip(h_in, ins):
+            h.copy_(t)
+        h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+        h2d = sum(t.numel() * t.element_size() for t in ins)
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        n_e2e = max(1, min(args.steps, 10))
+        barrier()
+        torch.cuda.synchronize(dev)
+        a = E(); a.record(stream)
+        for _ in range(n_e2e):
+            for h, t in zip(h_in, ins):
+                t.copy_(h, non_blocking=True)
+            step.run()
+            for h, t in zip(h_out, outs):
+                h.copy_(t, non_blocking=True)
+        b = E(); b.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e_ms = max_over_ranks(a.elapsed_time(b), device=dev)
+        e2e = {"value": step.flops * n_e2e * world / (e_ms / 1000.0) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = calibrated_oracle_baseline(args.workload, q, k, v, mask, target_s=args.cpu_seconds)
+
+    extra = {}
+    if args.workload == "block_sparse":
+        extra = {"mask_density": step.density, "kept_tiles": step.kept_tiles}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": config_of(w, args.workload, world, extra), "roofline": roofline, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": step.launches * args.steps, "clocks": clocks, "kernels": kernels,
+            "impl": "ours"}
+    emit(line, rank)
+    del step
+    finish_dist()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=["video_dit", "ring_causal", "block_sparse", "tiny_dense", "megatron"],
+                    default="video_dit", help="tiny_dense / megatron: reference arm only (parity-size cases)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--ref-rows", type=int, default=16, help="query rows per reference step")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override S (profiling captures on a smaller case; not a benchmark number)")
+    args = ap.parse_args(argv)
+    if args.impl == "reference":
+        return run_reference(args)
+    if args.workload not in ("video_dit", "ring_causal", "block_sparse"):
+        ap.error("--impl ours times the full-size workloads only")
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

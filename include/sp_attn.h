@@ -1,0 +1,197 @@
+/*
+ * sp_attn.h -- C ABI of libspattn.so: sequence/head-parallel exact attention for NVIDIA B200 (sm_100a).
+ *
+ * The operations, and the passages that define them:
+ *   - exact multi-head scaled-dot-product attention, O = softmax(Q K^T / sqrt(D)) V per head:
+ *     "LLM Lab Notes 05: Attention Tensor Parallelism -- Splitting QKV by Head, Megatron Style",
+ *     section 2 (code walkthrough) step 4 "local attention" and "Local projections and local attention";
+ *   - heads processed as independent, possibly uneven, contiguous head chunks whose outputs are
+ *     concatenated in chunk order: "HCMS: Head-Chunked Multi-Stream Pipeline ...", abstract (uneven
+ *     head partitions, numerical equivalence) and "LLM Lab Notes 05", sections 4-5 (rank-ordered
+ *     concatenation, divisibility of heads by ranks);
+ *   - KV processed in blocks whose partial (O, LSE) results are re-merged: "CHARM+: How Cross-Hardware
+ *     Attention Breaks Through Distributed Communication Bottlenecks", Ring-Attention paragraph (each
+ *     round computes local attention on one KV block and accumulates partial results), and "CHARM+:
+ *     Cross-Hardware Attention with Re-Merge Multistream Mechanism", abstract (re-merge);
+ *   - a per-head block-sparse mask of 128 x 128 tiles: "db-SP: Accelerating Sparse Attention for
+ *     Visual Generative Models with Dual-Balanced Sequence Parallelism", abstract;
+ *   - the Ulysses all-to-all layout permutation between P sequence shards and P head shards: "HCMS",
+ *     abstract (all-to-all sequence parallelism) and "db-SP", abstract (parallelism along the head
+ *     dimension, as in Ulysses).  Here the P "ranks" are P buffers in one GPU's memory.
+ *
+ * Conventions for every entry point:
+ *   - Q, K, V, O are BSHD: [B, S, H, D] contiguous, row-major; element (b, s, h, d) is at index
+ *     ((b * S + s) * H + h) * D + d.  Q, K, V and a bf16 O are bfloat16.  D is 64 or 128.
+ *   - LSE is fp32 [B, H, S]: the natural-log log-sum-exp of the scaled scores of a row, -inf for a row
+ *     that sees no key (whose O row is then 0).
+ *   - All pointers named as device pointers are device memory owned by the caller; the library never
+ *     allocates or frees device memory and keeps no pointer after a call returns.  Arrays of pointers
+ *     (head_chunks, o_parts, lse_parts, in_ranks, out_ranks) are host memory, read during the call.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL is the legacy default stream) and
+ *     returns after enqueuing.  Arguments are validated on the host before anything is launched: any
+ *     violation returns SP_ERR_INVALID_ARG (or SP_ERR_UNSUPPORTED) and launches nothing.  A launch
+ *     failure returns SP_ERR_CUDA.  A device-side wait that exceeds its time limit (the kernels never
+ *     spin without bound) records an error word that sp_check_device_error() reports as SP_ERR_TIMEOUT.
+ *   - Device pointers must be 16-byte aligned.
+ */
+#ifndef SP_ATTN_H
+#define SP_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SP_API __attribute__((visibility("default")))
+#else
+#define SP_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SP_OK = 0,
+  SP_ERR_INVALID_ARG = 1,
+  SP_ERR_UNSUPPORTED = 2,
+  SP_ERR_CUDA = 3,
+  SP_ERR_TIMEOUT = 4
+} sp_status;
+
+typedef enum { SP_BF16 = 0, SP_F32 = 1 } sp_dtype;
+
+/* Opaque stream handle: a cudaStream_t. */
+typedef void* sp_stream;
+
+/* Tile edge of the block mask and of the kernels' query/key tiles. */
+#define SP_TILE 128
+/* Largest number of partials sp_merge_partials combines in one call, and of relayout ranks. */
+#define SP_MAX_PARTS 64
+#define SP_MAX_RANKS 64
+
+/*
+ * Bytes of device workspace sp_attn_fwd / sp_attn_fwd_partial need for these sizes.
+ * n_kv_blocks > 1 needs n_kv_blocks fp32 partials (O [B,S,H,D] and LSE [B,H,S] each); has_mask != 0
+ * needs the compacted tile list (H * ceil(S/128) + 1 row offsets and up to H * ceil(S/128)^2 tile
+ * indices, int32).  Returns 0 when neither applies, and 0 for invalid sizes.
+ */
+SP_API size_t sp_attn_fwd_workspace_bytes(int B, int S, int H, int D, int n_kv_blocks, int has_mask);
+
+/*
+ * Exact attention, O = softmax(Q K^T / sqrt(D)) V per head (see the header comment for the passages).
+ *
+ * q, k, v   device, bf16 BSHD [B,S,H,D].
+ * o         device, bf16 BSHD [B,S,H,D], written; must not overlap q, k, v.
+ * lse       device, fp32 [B,H,S], written; may be NULL.
+ * head_chunks  host int[n_head_chunks]: contiguous chunks of heads, in order, each > 0, sum == H.
+ *           NULL means one chunk of H heads.  Chunk c covers heads [h0, h0 + head_chunks[c]) and its
+ *           output lands at the same head offset of o, which is the rank-ordered concatenation of the
+ *           chunks' outputs.  Per-head arithmetic does not depend on the chunking: every chunking gives
+ *           bitwise the same o and lse.
+ * n_kv_blocks  >= 1 and <= ceil(S/128).  1: keys are processed in one pass.  > 1: the key range is cut
+ *           into n_kv_blocks contiguous blocks of ceil(S/n) keys (rounded up to a multiple of 128 when a
+ *           block mask is given), each block's partial (O, LSE) is computed over all queries into the
+ *           workspace, and the partials are re-merged (sp_merge_partials) into o and lse.
+ * causal    0 or 1: key j is visible to query i only if j <= i (square, top-left aligned).
+ * block_mask  device uint8 [H, ceil(S/128), ceil(S/128)] or NULL (dense).  Tile (i, j) of head h is
+ *           computed iff block_mask[h][i][j] != 0; combined with causal by AND.  Shared by all b.
+ * workspace, workspace_bytes  device scratch of at least sp_attn_fwd_workspace_bytes(...) bytes
+ *           (may be NULL when that is 0).  Contents on entry are ignored; overwritten.
+ * Errors: SP_ERR_INVALID_ARG for B < 1, S < 1, H < 1, D not in {64, 128}, bad head chunks, bad
+ * n_kv_blocks, causal not 0/1, a NULL or misaligned required pointer, or a short workspace.
+ */
+SP_API sp_status sp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int S,
+                      int H, int D, const int* head_chunks, int n_head_chunks, int n_kv_blocks,
+                      int causal, const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
+                      sp_stream stream);
+
+/*
+ * One KV block (one Ring-Attention round): every one of the S queries attends only to keys
+ * kv_begin <= j < kv_end (positions global, so causal compares global positions).
+ *
+ * o_part    device, fp32 BSHD [B,S,H,D]: the block's normalised output; rows with no visible key are 0.
+ * lse_part  device, fp32 [B,H,S]: the block's LSE, -inf for rows with no visible key.
+ * 0 <= kv_begin <= kv_end <= S.  With a block mask, kv_begin must be a multiple of 128.
+ * Other arguments as in sp_attn_fwd (no head chunks: all H heads).
+ */
+SP_API sp_status sp_attn_fwd_partial(const void* q, const void* k, const void* v, float* o_part,
+                              float* lse_part, int B, int S, int H, int D, int kv_begin, int kv_end,
+                              int causal, const uint8_t* block_mask, void* workspace,
+                              size_t workspace_bytes, sp_stream stream);
+
+/*
+ * Re-merge of n partials with the log-sum-exp rule ("CHARM+ ... Re-Merge", abstract):
+ *   M = max_b lse_b,  lse = M + ln sum_b exp(lse_b - M),  o = sum_b exp(lse_b - lse) * o_b;
+ * a row whose partials are all -inf gives o = 0, lse = -inf (never NaN).
+ *
+ * o_parts, lse_parts  host arrays of n device pointers: fp32 BSHD [B,S,H,D] and fp32 [B,H,S].
+ * 1 <= n <= SP_MAX_PARTS.
+ * o         device, [B,S,H,D] of o_dtype (SP_BF16 rounds to nearest even, or SP_F32).  With SP_F32 it
+ *           may alias o_parts[0] (in-place merge); otherwise no overlap with the inputs.
+ * lse       device, fp32 [B,H,S], or NULL; may alias lse_parts[0].
+ */
+SP_API sp_status sp_merge_partials(const float* const* o_parts, const float* const* lse_parts, int n, void* o,
+                            float* lse, sp_dtype o_dtype, int B, int S, int H, int D, sp_stream stream);
+
+/*
+ * Ulysses relayout, sequence shards -> head shards, between P buffers of one GPU:
+ *   in_ranks[r]  device [B, S/P, H, D]   (rank r's slice of the sequence, all heads)
+ *   out_ranks[r] device [B, S, H/P, D]   (all positions of heads [r*H/P, (r+1)*H/P))
+ *   out_r[b, s, h', :] = in_{s / (S/P)}[b, s % (S/P), r*H/P + h', :]   (a bit-exact byte copy).
+ * Requires 1 <= P <= SP_MAX_RANKS, S % P == 0, H % P == 0 ("LLM Lab Notes 05", section 5: head count
+ * divisible by the parallel degree), elem_bytes in {1, 2, 4, 8}, (D * elem_bytes) % 16 == 0,
+ * 16-byte aligned buffers and no overlap between any input and any output.
+ */
+SP_API sp_status sp_seq_to_head_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B,
+                                  int S, int H, int D, int elem_bytes, sp_stream stream);
+
+/* The exact inverse: in_ranks[r] [B, S, H/P, D] -> out_ranks[r] [B, S/P, H, D].  Same requirements. */
+SP_API sp_status sp_head_to_seq_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B,
+                                  int S, int H, int D, int elem_bytes, sp_stream stream);
+
+/*
+ * Compacted tile list of a block mask, the form in which the attention kernels skip dropped tiles
+ * ("db-SP", abstract: dense blocks irregularly distributed in a per-head mask).
+ *   block_mask device uint8 [H, T, T], T = ceil(S/128); nonzero = keep.
+ *   row_ptr    device int32 [H*T + 1]: row (h, i) lists col_idx[row_ptr[h*T+i] .. row_ptr[h*T+i+1]).
+ *   col_idx    device int32, capacity H*T*T: kept key-tile indices of each row, increasing.
+ *   counts     device int32 [H*T] scratch.
+ */
+SP_API sp_status sp_build_tile_list(const uint8_t* block_mask, int H, int S, int32_t* row_ptr,
+                             int32_t* col_idx, int32_t* counts, sp_stream stream);
+
+/* Human-readable name of a status code (static storage). */
+SP_API const char* sp_status_string(sp_status s);
+
+/*
+ * Synchronises `stream`, then reads and clears the device error word of the current device:
+ * SP_ERR_TIMEOUT if a kernel's bounded wait expired since the last check, SP_ERR_CUDA if the stream
+ * reports an error, else SP_OK.
+ */
+SP_API sp_status sp_check_device_error(sp_stream stream);
+
+/*
+ * As sp_check_device_error, and also returns the raw error word in *bits (may be NULL): one bit per
+ * kind of wait that expired (Q loaded, Q free, K/V loaded, K/V free, S ready, P ready, P V done, O read
+ * out, drain, debug), for diagnosing which hand-off gave up.
+ */
+SP_API sp_status sp_check_device_error_bits(sp_stream stream, unsigned int* bits);
+
+/* Time limit of every device-side wait, in nanoseconds (default 2e9).  Applies to later launches. */
+SP_API void sp_set_wait_timeout_ns(unsigned long long ns);
+
+/*
+ * Exercises the bounded-wait path: launches one warp that waits on a barrier nothing will complete,
+ * with the given limit; the wait gives up, records SP_ERR_TIMEOUT in the device error word and the
+ * kernel returns normally.  The next sp_check_device_error() returns SP_ERR_TIMEOUT.
+ */
+SP_API sp_status sp_debug_wait_timeout(unsigned long long timeout_ns, sp_stream stream);
+
+/* Library version string. */
+SP_API const char* sp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SP_ATTN_H */

@@ -1,0 +1,366 @@
+// api.cu -- the C entry points of libspattn.so: host-side validation, workspace layout, tensor maps and
+// launches.  Declarations and the contract of each call are in include/sp_attn.h.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "sp_internal.h"
+#include "sp_ptx.cuh"
+
+namespace spattn {
+
+// The device error word: bounded waits that expire OR a code into it (see sp_check_device_error).
+__device__ unsigned int g_sp_error = 0;
+
+namespace {
+
+std::mutex g_mu;
+int g_num_sms[kMaxDevices] = {};
+unsigned int* g_err_addr[kMaxDevices] = {};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+unsigned long long g_timeout_ns = 2000000000ull;
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+struct WsLayout {
+  size_t parts_o = 0, parts_lse = 0, row_ptr = 0, col_idx = 0, counts = 0, total = 0;
+};
+
+// Workspace: [n_kv_blocks fp32 O partials][n_kv_blocks fp32 LSE partials][row_ptr][col_idx][counts]
+WsLayout ws_layout(int B, int S, int H, int D, int n_kv_blocks, int has_mask) {
+  WsLayout w;
+  size_t off = 0;
+  if (n_kv_blocks > 1) {
+    w.parts_o = off;
+    off += align_up((size_t)n_kv_blocks * B * S * H * D * sizeof(float), 256);
+    w.parts_lse = off;
+    off += align_up((size_t)n_kv_blocks * B * H * S * sizeof(float), 256);
+  }
+  if (has_mask) {
+    const size_t T = (S + SP_TILE - 1) / SP_TILE;
+    w.row_ptr = off;
+    off += align_up((H * T + 1) * sizeof(int32_t), 256);
+    w.col_idx = off;
+    off += align_up(H * T * T * sizeof(int32_t), 256);
+    w.counts = off;
+    off += align_up(H * T * sizeof(int32_t), 256);
+  }
+  w.total = off;
+  return w;
+}
+
+bool sizes_ok(int B, int S, int H, int D) {
+  if (B < 1 || S < 1 || H < 1) return false;
+  if (D != 64 && D != 128) return false;
+  // keep every element index inside 63 bits and every tile index inside int
+  const double elems = (double)B * S * H * D;
+  return elems < 9.0e15 && S <= (1 << 30) && (double)B * H * ((S + 255) / 256) < 2.0e9;
+}
+
+cudaStream_t as_stream(sp_stream s) { return reinterpret_cast<cudaStream_t>(s); }
+
+sp_status fill_attn_params(AttnParams& p, int B, int S, int H, int D, int kv_begin, int kv_end,
+                           int causal, const int* chunk_h0, int n_chunks) {
+  p = AttnParams{};
+  p.B = B;
+  p.S = S;
+  p.H = H;
+  p.D = D;
+  const int n_qtiles = (S + SP_TILE - 1) / SP_TILE;
+  p.n_qpairs = (n_qtiles + 1) / 2;
+  p.kv_begin = kv_begin;
+  p.kv_lim = kv_end < S ? kv_end : S;
+  p.n_kv_tiles = p.kv_lim > kv_begin ? (p.kv_lim - kv_begin + SP_TILE - 1) / SP_TILE : 0;
+  p.causal = causal;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.mask_T = n_qtiles;
+  p.timeout_ns = g_timeout_ns;
+  p.err = device_error_word();
+  if (!p.err) return SP_ERR_CUDA;
+  p.n_chunks = n_chunks;
+  long long items = 0;
+  for (int c = 0; c < n_chunks; ++c) {
+    p.chunk_h0[c] = chunk_h0[c];
+    p.chunk_item0[c] = (int)items;
+    items += (long long)B * (chunk_h0[c + 1] - chunk_h0[c]) * p.n_qpairs;
+  }
+  p.chunk_h0[n_chunks] = chunk_h0[n_chunks];
+  p.chunk_item0[n_chunks] = (int)items;
+  if (items > 0x7fffffffLL) return SP_ERR_INVALID_ARG;
+  p.n_items = (int)items;
+  return SP_OK;
+}
+
+}  // namespace
+
+int num_sms(int device) {
+  if (device < 0 || device >= kMaxDevices) return 1;
+  if (g_num_sms[device] == 0) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || v < 1) v = 1;
+    g_num_sms[device] = v;
+  }
+  return g_num_sms[device];
+}
+
+unsigned long long wait_timeout_ns() { return g_timeout_ns; }
+
+unsigned int* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_addr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_sp_error) != cudaSuccess) return nullptr;
+    g_err_addr[dev] = static_cast<unsigned int*>(ptr);
+  }
+  return g_err_addr[dev];
+}
+
+bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+          q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  // Dimensions innermost first: d, h, s, b.  Box: 64 head-dim elements (128 bytes, the swizzle span)
+  // of one head, 128 positions, one batch.  Rows past S read as zero.
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace spattn
+
+using namespace spattn;
+
+extern "C" {
+
+size_t sp_attn_fwd_workspace_bytes(int B, int S, int H, int D, int n_kv_blocks, int has_mask) {
+  if (!sizes_ok(B, S, H, D) || n_kv_blocks < 1) return 0;
+  return ws_layout(B, S, H, D, n_kv_blocks, has_mask).total;
+}
+
+const char* sp_status_string(sp_status s) {
+  switch (s) {
+    case SP_OK: return "SP_OK";
+    case SP_ERR_INVALID_ARG: return "SP_ERR_INVALID_ARG";
+    case SP_ERR_UNSUPPORTED: return "SP_ERR_UNSUPPORTED";
+    case SP_ERR_CUDA: return "SP_ERR_CUDA";
+    case SP_ERR_TIMEOUT: return "SP_ERR_TIMEOUT";
+  }
+  return "SP_ERR_UNKNOWN";
+}
+
+const char* sp_version(void) { return "spattn 0.1 (sm_100a)"; }
+
+void sp_set_wait_timeout_ns(unsigned long long ns) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_timeout_ns = ns < 1000ull ? 1000ull : ns;
+}
+
+sp_status sp_check_device_error_bits(sp_stream stream, unsigned int* bits) {
+  if (bits) *bits = 0;
+  if (cudaStreamSynchronize(as_stream(stream)) != cudaSuccess) return SP_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_sp_error, sizeof(v)) != cudaSuccess) return SP_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_sp_error, &zero, sizeof(zero)) != cudaSuccess) return SP_ERR_CUDA;
+  if (bits) *bits = v;
+  return (v & ERR_ANY_TIMEOUT) ? SP_ERR_TIMEOUT : SP_OK;
+}
+
+sp_status sp_check_device_error(sp_stream stream) { return sp_check_device_error_bits(stream, nullptr); }
+
+sp_status sp_debug_wait_timeout(unsigned long long timeout_ns, sp_stream stream) {
+  if (timeout_ns < 1000ull || timeout_ns > 10000000000ull) return SP_ERR_INVALID_ARG;
+  return launch_debug_wait(timeout_ns, as_stream(stream));
+}
+
+sp_status sp_build_tile_list(const uint8_t* block_mask, int H, int S, int32_t* row_ptr, int32_t* col_idx,
+                             int32_t* counts, sp_stream stream) {
+  if (!block_mask || !row_ptr || !col_idx || !counts || H < 1 || S < 1) return SP_ERR_INVALID_ARG;
+  const long long T = (S + SP_TILE - 1) / SP_TILE;
+  if ((long long)H * T * T > 0x7fffffffLL) return SP_ERR_INVALID_ARG;
+  return launch_tile_list(block_mask, H, (int)T, row_ptr, col_idx, counts, as_stream(stream));
+}
+
+sp_status sp_attn_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                              int B, int S, int H, int D, int kv_begin, int kv_end, int causal,
+                              const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
+                              sp_stream stream) {
+  if (!sizes_ok(B, S, H, D)) return SP_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o_part || !lse_part) return SP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part) || !aligned16(lse_part))
+    return SP_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SP_ERR_INVALID_ARG;
+  if (kv_begin < 0 || kv_end < kv_begin || kv_end > S) return SP_ERR_INVALID_ARG;
+  if (block_mask && kv_begin % SP_TILE != 0) return SP_ERR_INVALID_ARG;
+  const WsLayout wl = ws_layout(B, S, H, D, 1, block_mask != nullptr);
+  if (wl.total > 0 && (!workspace || workspace_bytes < wl.total || !aligned16(workspace)))
+    return SP_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  AttnParams p;
+  int h0[2] = {0, H};
+  sp_status s = fill_attn_params(p, B, S, H, D, kv_begin, kv_end, causal, h0, 1);
+  if (s != SP_OK) return s;
+  p.o = o_part;
+  p.o_f32 = 1;
+  p.lse = lse_part;
+  if (block_mask) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* row_ptr = reinterpret_cast<int32_t*>(ws + wl.row_ptr);
+    int32_t* col_idx = reinterpret_cast<int32_t*>(ws + wl.col_idx);
+    s = launch_tile_list(block_mask, H, p.mask_T, row_ptr, col_idx, reinterpret_cast<int32_t*>(ws + wl.counts), st);
+    if (s != SP_OK) return s;
+    p.row_ptr = row_ptr;
+    p.col_idx = col_idx;
+  }
+  return launch_attn(p, q, k, v, st);
+}
+
+sp_status sp_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int S, int H,
+                      int D, const int* head_chunks, int n_head_chunks, int n_kv_blocks, int causal,
+                      const uint8_t* block_mask, void* workspace, size_t workspace_bytes, sp_stream stream) {
+  if (!sizes_ok(B, S, H, D)) return SP_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o) return SP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return SP_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SP_ERR_INVALID_ARG;
+  const int n_tiles = (S + SP_TILE - 1) / SP_TILE;
+  if (n_kv_blocks < 1 || n_kv_blocks > n_tiles || n_kv_blocks > SP_MAX_PARTS) return SP_ERR_INVALID_ARG;
+  // head chunks: contiguous, in order, each > 0, summing to H
+  int h0[kMaxChunks + 1];
+  int n_chunks = 1;
+  h0[0] = 0;
+  h0[1] = H;
+  if (head_chunks) {
+    if (n_head_chunks < 1 || n_head_chunks > kMaxChunks) return SP_ERR_INVALID_ARG;
+    long long acc = 0;
+    for (int c = 0; c < n_head_chunks; ++c) {
+      if (head_chunks[c] < 1) return SP_ERR_INVALID_ARG;
+      h0[c] = (int)acc;
+      acc += head_chunks[c];
+      if (acc > H) return SP_ERR_INVALID_ARG;
+    }
+    if (acc != H) return SP_ERR_INVALID_ARG;
+    h0[n_head_chunks] = H;
+    n_chunks = n_head_chunks;
+  } else if (n_head_chunks != 0 && n_head_chunks != 1) {
+    return SP_ERR_INVALID_ARG;
+  }
+  const WsLayout wl = ws_layout(B, S, H, D, n_kv_blocks, block_mask != nullptr);
+  if (wl.total > 0 && (!workspace || workspace_bytes < wl.total || !aligned16(workspace)))
+    return SP_ERR_INVALID_ARG;
+  cudaStream_t st = as_stream(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  AttnParams p;
+  sp_status s = fill_attn_params(p, B, S, H, D, 0, S, causal, h0, n_chunks);
+  if (s != SP_OK) return s;
+  if (block_mask) {
+    int32_t* row_ptr = reinterpret_cast<int32_t*>(ws + wl.row_ptr);
+    int32_t* col_idx = reinterpret_cast<int32_t*>(ws + wl.col_idx);
+    s = launch_tile_list(block_mask, H, p.mask_T, row_ptr, col_idx, reinterpret_cast<int32_t*>(ws + wl.counts), st);
+    if (s != SP_OK) return s;
+    p.row_ptr = row_ptr;
+    p.col_idx = col_idx;
+  }
+  if (n_kv_blocks == 1) {
+    p.o = o;
+    p.o_f32 = 0;
+    p.lse = lse;
+    return launch_attn(p, q, k, v, st);
+  }
+  // KV blocks: ceil(S / n) keys each (a multiple of 128 with a mask), partials into the workspace, then
+  // the log-sum-exp re-merge.
+  long long blk = (S + n_kv_blocks - 1) / n_kv_blocks;
+  if (block_mask) blk = (blk + SP_TILE - 1) / SP_TILE * SP_TILE;
+  float* parts_o = reinterpret_cast<float*>(ws + wl.parts_o);
+  float* parts_l = reinterpret_cast<float*>(ws + wl.parts_lse);
+  const size_t o_elems = (size_t)B * S * H * D, l_elems = (size_t)B * H * S;
+  const float* op[SP_MAX_PARTS];
+  const float* lp[SP_MAX_PARTS];
+  for (int i = 0; i < n_kv_blocks; ++i) {
+    const long long a = i * blk, e = (i + 1) * blk < S ? (i + 1) * blk : S;
+    AttnParams pi = p;
+    pi.kv_begin = (int)(a < S ? a : S);
+    pi.kv_lim = (int)(e > pi.kv_begin ? e : pi.kv_begin);
+    pi.n_kv_tiles = (pi.kv_lim - pi.kv_begin + SP_TILE - 1) / SP_TILE;
+    pi.o = parts_o + i * o_elems;
+    pi.o_f32 = 1;
+    pi.lse = parts_l + i * l_elems;
+    s = launch_attn(pi, q, k, v, st);
+    if (s != SP_OK) return s;
+    op[i] = parts_o + i * o_elems;
+    lp[i] = parts_l + i * l_elems;
+  }
+  return launch_merge(op, lp, n_kv_blocks, o, lse, 0, B, S, H, D, st);
+}
+
+sp_status sp_merge_partials(const float* const* o_parts, const float* const* lse_parts, int n, void* o,
+                            float* lse, sp_dtype o_dtype, int B, int S, int H, int D, sp_stream stream) {
+  if (!sizes_ok(B, S, H, D)) return SP_ERR_INVALID_ARG;
+  if (!o_parts || !lse_parts || !o || n < 1 || n > SP_MAX_PARTS) return SP_ERR_INVALID_ARG;
+  if (o_dtype != SP_BF16 && o_dtype != SP_F32) return SP_ERR_INVALID_ARG;
+  if (!aligned16(o) || (lse && !aligned16(lse))) return SP_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i) {
+    if (!o_parts[i] || !lse_parts[i] || !aligned16(o_parts[i]) || !aligned16(lse_parts[i]))
+      return SP_ERR_INVALID_ARG;
+    if (i > 0 && (o_parts[i] == o || (lse && lse_parts[i] == lse))) return SP_ERR_INVALID_ARG;
+  }
+  if (o_dtype == SP_BF16 && (const void*)o_parts[0] == o) return SP_ERR_INVALID_ARG;
+  return launch_merge(o_parts, lse_parts, n, o, lse, o_dtype == SP_F32, B, S, H, D, as_stream(stream));
+}
+
+static sp_status relayout_common(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,
+                                 int H, int D, int elem_bytes, bool seq_to_head, sp_stream stream) {
+  if (!in_ranks || !out_ranks || P < 1 || P > SP_MAX_RANKS || B < 1 || S < 1 || H < 1 || D < 1)
+    return SP_ERR_INVALID_ARG;
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8) return SP_ERR_INVALID_ARG;
+  if (S % P != 0 || H % P != 0 || ((long long)D * elem_bytes) % 16 != 0) return SP_ERR_INVALID_ARG;
+  if ((double)B * S * H * D * elem_bytes > 9.0e15) return SP_ERR_INVALID_ARG;
+  const long long in_bytes = seq_to_head ? (long long)B * (S / P) * H * D * elem_bytes
+                                         : (long long)B * S * (H / P) * D * elem_bytes;
+  const long long out_bytes = seq_to_head ? (long long)B * S * (H / P) * D * elem_bytes
+                                          : (long long)B * (S / P) * H * D * elem_bytes;
+  for (int r = 0; r < P; ++r) {
+    if (!in_ranks[r] || !out_ranks[r] || !aligned16(in_ranks[r]) || !aligned16(out_ranks[r]))
+      return SP_ERR_INVALID_ARG;
+  }
+  // no input buffer may overlap any output buffer
+  for (int r = 0; r < P; ++r)
+    for (int g = 0; g < P; ++g) {
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(in_ranks[r]), a1 = a0 + in_bytes;
+      const uintptr_t b0 = reinterpret_cast<uintptr_t>(out_ranks[g]), b1 = b0 + out_bytes;
+      if (a0 < b1 && b0 < a1) return SP_ERR_INVALID_ARG;
+    }
+  return launch_relayout(in_ranks, out_ranks, P, B, S, H, D, elem_bytes, seq_to_head, as_stream(stream));
+}
+
+sp_status sp_seq_to_head_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,
+                                  int H, int D, int elem_bytes, sp_stream stream) {
+  return relayout_common(in_ranks, out_ranks, P, B, S, H, D, elem_bytes, true, stream);
+}
+
+sp_status sp_head_to_seq_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,
+                                  int H, int D, int elem_bytes, sp_stream stream) {
+  return relayout_common(in_ranks, out_ranks, P, B, S, H, D, elem_bytes, false, stream);
+}
+
+}  // extern "C"

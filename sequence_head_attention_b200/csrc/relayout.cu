@@ -1,0 +1,93 @@
+// relayout.cu -- the Ulysses all-to-all layout permutation between P rank buffers of one GPU.
+//
+// "HCMS: Head-Chunked Multi-Stream Pipeline ...", abstract (all-to-all based sequence parallelism) and
+// "db-SP ...", abstract (parallelism along the head dimension, as in Ulysses).  Before attention, rank r
+// holds positions [r S/P, (r+1) S/P) of every head; after it, rank r holds every position of heads
+// [r H/P, (r+1) H/P):
+//   seq -> head:  out_r[b, s, h', :] = in_{s / (S/P)}[b, s % (S/P), r H/P + h', :]
+//   head -> seq:  out_r[b, s', h, :] = in_{h / (H/P)}[b, r S/P + s', h % (H/P), :]
+// Both directions move contiguous runs of (H/P) * D elements: one warp copies one run with 16-byte
+// vector loads and stores (streaming cache hints), so both sides are fully coalesced.  Bit-exact.
+#include <cstdint>
+
+#include "sp_internal.h"
+
+namespace spattn {
+namespace {
+
+struct RankPtrs {
+  const uint8_t* in[SP_MAX_RANKS];
+  uint8_t* out[SP_MAX_RANKS];
+};
+
+template <bool kSeqToHead>
+__global__ void __launch_bounds__(256) relayout_kernel(const __grid_constant__ RankPtrs rp, int P, int B,
+                                                       int S, int H, long long run_bytes) {
+  const int Sl = S / P;
+  const long long n_runs = (long long)P * B * S;
+  const int lane = threadIdx.x & 31;
+  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
+  const int nvec = (int)(run_bytes / 16);
+  for (long long run = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5; run < n_runs; run += warps) {
+    const uint8_t* src;
+    uint8_t* dst;
+    if (kSeqToHead) {
+      // run = (r, b, s): destination out_r[b, s, :, :], contiguous in s
+      const int s = (int)(run % S);
+      const long long rb = run / S;
+      const int b = (int)(rb % B);
+      const int r = (int)(rb / B);
+      src = rp.in[s / Sl] + (((long long)b * Sl + (s % Sl)) * P + r) * run_bytes;  // heads r*H/P.. of row
+      dst = rp.out[r] + ((long long)b * S + s) * run_bytes;
+    } else {
+      // run = (r, b, s', g): destination out_r[b, s', g*H/P : (g+1)*H/P, :], contiguous in g
+      const int g = (int)(run % P);
+      const long long rest = run / P;
+      const int sl = (int)(rest % Sl);
+      const long long rb = rest / Sl;
+      const int b = (int)(rb % B);
+      const int r = (int)(rb / B);
+      src = rp.in[g] + ((long long)b * S + (long long)r * Sl + sl) * run_bytes;
+      dst = rp.out[r] + (((long long)b * Sl + sl) * P + g) * run_bytes;
+    }
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    int v = lane;
+    for (; v + 96 < nvec; v += 128) {
+      const uint4 x0 = __ldcs(s4 + v), x1 = __ldcs(s4 + v + 32), x2 = __ldcs(s4 + v + 64), x3 = __ldcs(s4 + v + 96);
+      __stcs(d4 + v, x0);
+      __stcs(d4 + v + 32, x1);
+      __stcs(d4 + v + 64, x2);
+      __stcs(d4 + v + 96, x3);
+    }
+    for (; v < nvec; v += 32) __stcs(d4 + v, __ldcs(s4 + v));
+  }
+}
+
+}  // namespace
+
+sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,
+                          int H, int D, int elem_bytes, bool seq_to_head, cudaStream_t stream) {
+  RankPtrs rp = {};
+  for (int r = 0; r < P; ++r) {
+    rp.in[r] = static_cast<const uint8_t*>(in_ranks[r]);
+    rp.out[r] = static_cast<uint8_t*>(out_ranks[r]);
+  }
+  // A run is the H/P heads of one (rank, b, s): H/P * D elements.  In the seq-sharded layout a row of
+  // H heads holds P consecutive runs, which is what the kernel's "* P + r" indexing uses.
+  const long long run_bytes = (long long)(H / P) * D * elem_bytes;
+  const long long n_runs = (long long)P * B * S;
+  if (n_runs == 0) return SP_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SP_ERR_CUDA;
+  long long blocks = (n_runs + 7) / 8;
+  const long long cap = (long long)num_sms(dev) * 8;
+  if (blocks > cap) blocks = cap;
+  if (seq_to_head)
+    relayout_kernel<true><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes);
+  else
+    relayout_kernel<false><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes);
+  return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+}
+
+}  // namespace spattn

@@ -1,0 +1,57 @@
+// sp_internal.h -- declarations shared by the library's translation units (not part of the C ABI).
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/sp_attn.h"
+
+namespace spattn {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxChunks = 128;
+
+// Parameters of one attention launch (all H heads, all S queries, keys in [kv_begin, kv_lim)).
+struct AttnParams {
+  int B, S, H, D;
+  int n_qpairs;     // ceil(ceil(S/128) / 2): work items per (b, h)
+  int n_items;      // B * H * n_qpairs
+  int kv_begin;     // first key position
+  int kv_lim;       // one past the last key position (<= S)
+  int n_kv_tiles;   // ceil((kv_lim - kv_begin) / 128)
+  int causal;
+  float scale_log2; // log2(e) / sqrt(D)
+  void* o;          // bf16 or fp32 BSHD
+  int o_f32;
+  float* lse;       // [B, H, S] or nullptr
+  const int* row_ptr;  // block-sparse tile list (nullptr: dense)
+  const int* col_idx;
+  int mask_T;          // ceil(S/128)
+  int n_chunks;
+  int chunk_h0[kMaxChunks + 1];     // first head of each chunk, chunk_h0[n_chunks] = H
+  int chunk_item0[kMaxChunks + 1];  // first work item of each chunk
+  unsigned long long timeout_ns;
+  unsigned int* err;  // device error word of this device
+};
+
+// Device properties and driver entry points (cached per device).
+int num_sms(int device);
+bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, int D);
+unsigned long long wait_timeout_ns();
+unsigned int* device_error_word();  // address of the current device's error word, or nullptr
+
+// Launchers (host validation is done by the C entry points before these are called).
+int attn_smem_bytes(int D);
+sp_status launch_attn(const AttnParams& p, const void* q, const void* k, const void* v,
+                      cudaStream_t stream);
+sp_status launch_merge(const float* const* o_parts, const float* const* lse_parts, int n, void* o,
+                       float* lse, int o_f32, int B, int S, int H, int D, cudaStream_t stream);
+sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,
+                          int H, int D, int elem_bytes, bool seq_to_head, cudaStream_t stream);
+sp_status launch_tile_list(const uint8_t* mask, int H, int T, int32_t* row_ptr, int32_t* col_idx,
+                           int32_t* counts, cudaStream_t stream);
+sp_status launch_debug_wait(unsigned long long timeout_ns, cudaStream_t stream);
+
+}  // namespace spattn

@@ -1,0 +1,114 @@
+// tile_list.cu -- compacted per-(head, query tile) list of the key tiles a block mask keeps.
+//
+// "db-SP: Accelerating Sparse Attention ...", abstract: block-wise sparse attention whose dense blocks
+// are irregularly placed and whose density varies across heads.  The attention kernel walks these lists
+// so that dropped tiles are never loaded or multiplied.  Output is CSR: row (h, i) lists, in increasing
+// order, every j with mask[h][i][j] != 0 -- fully determined, so it is compared bit for bit.
+//
+// Three small launches: count per row (one warp per row, ballots over 32 bytes at a time), an exclusive
+// scan of the counts (one block), and the fill (one warp per row, ballot + popcount for each lane's slot).
+#include <cstdint>
+
+#include "sp_internal.h"
+#include "sp_ptx.cuh"
+
+namespace spattn {
+namespace {
+
+__global__ void __launch_bounds__(256) tile_count_kernel(const uint8_t* mask, int rows, int T, int32_t* counts) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint8_t* m = mask + (size_t)row * T;
+  int c = 0;
+  for (int j0 = 0; j0 < T; j0 += 32) {
+    const int j = j0 + lane;
+    const unsigned bal = __ballot_sync(0xffffffffu, j < T && m[j] != 0);
+    c += __popc(bal);
+  }
+  if (lane == 0) counts[row] = c;
+}
+
+// Exclusive scan of counts[0..n) into row_ptr[0..n]; one block of 1024 threads.
+__global__ void __launch_bounds__(1024) tile_scan_kernel(const int32_t* counts, int n, int32_t* row_ptr) {
+  __shared__ int32_t warp_tot[32];
+  const int tid = threadIdx.x;
+  const int per = (n + 1023) / 1024;
+  const int lo = min(n, tid * per), hi = min(n, lo + per);
+  int local = 0;
+  for (int i = lo; i < hi; ++i) local += counts[i];
+  // inclusive scan of `local` over the block
+  const int lane = tid & 31, warp = tid >> 5;
+  int x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    warp_tot[lane] = t;
+  }
+  __syncthreads();
+  int run = x - local + (warp > 0 ? warp_tot[warp - 1] : 0);  // exclusive prefix of this thread's segment
+  for (int i = lo; i < hi; ++i) {
+    row_ptr[i] = run;
+    run += counts[i];
+  }
+  if (tid == 1023) row_ptr[n] = run;
+}
+
+__global__ void __launch_bounds__(256) tile_fill_kernel(const uint8_t* mask, int rows, int T, const int32_t* row_ptr,
+                                                        int32_t* col_idx) {
+  const int row = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (row >= rows) return;
+  const uint8_t* m = mask + (size_t)row * T;
+  int base = row_ptr[row];
+  for (int j0 = 0; j0 < T; j0 += 32) {
+    const int j = j0 + lane;
+    const bool keep = j < T && m[j] != 0;
+    const unsigned bal = __ballot_sync(0xffffffffu, keep);
+    if (keep) col_idx[base + __popc(bal & ((1u << lane) - 1u))] = j;
+    base += __popc(bal);
+  }
+}
+
+__global__ void debug_wait_kernel(unsigned long long timeout_ns, unsigned int* err) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+    // Nothing ever arrives on this barrier: the bounded wait must give up and record the error.
+    mbar_wait(smem_u32(&bar), 0, timeout_ns, ERR_TIMEOUT_DEBUG, nullptr, err);
+  }
+}
+
+}  // namespace
+
+sp_status launch_tile_list(const uint8_t* mask, int H, int T, int32_t* row_ptr, int32_t* col_idx,
+                           int32_t* counts, cudaStream_t stream) {
+  const int rows = H * T;
+  if (rows == 0) return SP_OK;
+  const int blocks = (rows + 7) / 8;
+  tile_count_kernel<<<blocks, 256, 0, stream>>>(mask, rows, T, counts);
+  tile_scan_kernel<<<1, 1024, 0, stream>>>(counts, rows, row_ptr);
+  tile_fill_kernel<<<blocks, 256, 0, stream>>>(mask, rows, T, row_ptr, col_idx);
+  return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+}
+
+sp_status launch_debug_wait(unsigned long long timeout_ns, cudaStream_t stream) {
+  unsigned int* err = device_error_word();
+  if (!err) return SP_ERR_CUDA;
+  debug_wait_kernel<<<1, 32, 0, stream>>>(timeout_ns, err);
+  return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+}
+
+}  // namespace spattn

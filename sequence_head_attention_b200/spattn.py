@@ -1,0 +1,250 @@
+"""ctypes binding of libspattn.so, one Python function per C entry point, same names.
+
+Argument marshalling only: torch tensors supply device pointers and the stream; every step of the
+computation runs in the library's CUDA kernels.  There is no fallback path: if the shared library is
+missing or fails to load, every call raises.  The C contract (layouts, ownership, errors) is documented
+in include/sp_attn.h.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libspattn.so")
+HEADER = os.path.join(_HERE, "..", "include", "sp_attn.h")
+
+SP_OK, SP_ERR_INVALID_ARG, SP_ERR_UNSUPPORTED, SP_ERR_CUDA, SP_ERR_TIMEOUT = 0, 1, 2, 3, 4
+SP_BF16, SP_F32 = 0, 1
+SP_TILE = 128
+SP_MAX_PARTS = 64
+SP_MAX_RANKS = 64
+
+_lock = threading.Lock()
+_lib = None
+
+
+class SpError(RuntimeError):
+    """A libspattn call returned a status other than SP_OK."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {sp_status_string(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded library (loaded on first use; raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(LIB_PATH):
+                raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                                   "`python -m sequence_head_attention_b200.build`")
+            L = ctypes.CDLL(LIB_PATH)
+            P, I, Z, U64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_ulonglong
+            sig = {
+                "sp_attn_fwd_workspace_bytes": (Z, [I, I, I, I, I, I]),
+                "sp_attn_fwd": (I, [P, P, P, P, P, I, I, I, I, P, I, I, I, P, P, Z, P]),
+                "sp_attn_fwd_partial": (I, [P, P, P, P, P, I, I, I, I, I, I, I, P, P, Z, P]),
+                "sp_merge_partials": (I, [P, P, I, P, P, I, I, I, I, I, P]),
+                "sp_seq_to_head_relayout": (I, [P, P, I, I, I, I, I, I, P]),
+                "sp_head_to_seq_relayout": (I, [P, P, I, I, I, I, I, I, P]),
+                "sp_build_tile_list": (I, [P, I, I, P, P, P, P]),
+                "sp_status_string": (ctypes.c_char_p, [I]),
+                "sp_check_device_error": (I, [P]),
+                "sp_check_device_error_bits": (I, [P, P]),
+                "sp_set_wait_timeout_ns": (None, [U64]),
+                "sp_debug_wait_timeout": (I, [U64, P]),
+                "sp_version": (ctypes.c_char_p, []),
+            }
+            for name, (res, args) in sig.items():
+                f = getattr(L, name)
+                f.restype = res
+                f.argtypes = args
+            _lib = L
+    return _lib
+
+
+def _check(fn: str, status: int):
+    if status != SP_OK:
+        raise SpError(fn, status)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _ptr_array(ts):
+    arr = (ctypes.c_void_p * len(ts))(*[_ptr(t) for t in ts])
+    return ctypes.cast(arr, ctypes.c_void_p), arr
+
+
+def _need(cond, msg):
+    if not cond:
+        raise ValueError(msg)
+
+
+def _bshd(t, name, dtype=torch.bfloat16):
+    _need(t.dim() == 4, f"{name} must be [B, S, H, D]")
+    _need(t.dtype == dtype, f"{name} must be {dtype}")
+    _need(t.is_cuda and t.is_contiguous(), f"{name} must be a contiguous CUDA tensor")
+
+
+# ------------------------------------------------------------------------------------------------------
+def sp_status_string(status: int) -> str:
+    return lib().sp_status_string(int(status)).decode()
+
+
+def sp_version() -> str:
+    return lib().sp_version().decode()
+
+
+def sp_attn_fwd_workspace_bytes(B, S, H, D, n_kv_blocks=1, has_mask=False) -> int:
+    return int(lib().sp_attn_fwd_workspace_bytes(B, S, H, D, n_kv_blocks, int(bool(has_mask))))
+
+
+def sp_attn_fwd(q, k, v, o, lse=None, head_chunks=None, n_kv_blocks=1, causal=False, block_mask=None,
+                workspace=None, stream=None):
+    """Exact attention of q, k, v (bf16 [B,S,H,D]) into o (bf16) and lse (fp32 [B,H,S] or None).
+
+    The workspace, when the configuration needs one and none is given, is allocated here with torch
+    (device memory is the caller's: the library itself never allocates)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _bshd(t, n)
+    B, S, H, D = q.shape
+    if lse is not None:
+        _need(lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, S),
+              "lse must be contiguous fp32 [B, H, S]")
+    if block_mask is not None:
+        _need(block_mask.dtype == torch.uint8 and block_mask.is_contiguous(), "block_mask must be uint8")
+    ws_bytes = sp_attn_fwd_workspace_bytes(B, S, H, D, n_kv_blocks, block_mask is not None)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    hc = None
+    n_hc = 0
+    if head_chunks is not None:
+        n_hc = len(head_chunks)
+        hc = (ctypes.c_int * n_hc)(*[int(c) for c in head_chunks])
+    st = lib().sp_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, S, H, D,
+                           ctypes.cast(hc, ctypes.c_void_p) if hc is not None else None, n_hc,
+                           int(n_kv_blocks), int(bool(causal)), _ptr(block_mask), _ptr(workspace),
+                           0 if workspace is None else workspace.numel() * workspace.element_size(),
+                           _stream(stream))
+    _check("sp_attn_fwd", st)
+    return o, lse
+
+
+def sp_attn_fwd_partial(q, k, v, o_part, lse_part, kv_begin, kv_end, causal=False, block_mask=None,
+                        workspace=None, stream=None):
+    """One KV block [kv_begin, kv_end) for every query: fp32 o_part [B,S,H,D], fp32 lse_part [B,H,S]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bshd(t, n)
+    _bshd(o_part, "o_part", torch.float32)
+    B, S, H, D = q.shape
+    _need(lse_part.dtype == torch.float32 and tuple(lse_part.shape) == (B, H, S), "lse_part must be fp32 [B,H,S]")
+    ws_bytes = sp_attn_fwd_workspace_bytes(B, S, H, D, 1, block_mask is not None)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    st = lib().sp_attn_fwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(o_part), _ptr(lse_part), B, S, H, D,
+                                   int(kv_begin), int(kv_end), int(bool(causal)), _ptr(block_mask),
+                                   _ptr(workspace),
+                                   0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                   _stream(stream))
+    _check("sp_attn_fwd_partial", st)
+    return o_part, lse_part
+
+
+def sp_merge_partials(o_parts, lse_parts, o, lse=None, stream=None):
+    """Log-sum-exp re-merge of n fp32 partials into o (bf16 or fp32 [B,S,H,D]) and lse (fp32 [B,H,S])."""
+    n = len(o_parts)
+    _need(n == len(lse_parts) and n >= 1, "need n >= 1 matching partials")
+    B, S, H, D = o_parts[0].shape
+    dt = SP_F32 if o.dtype == torch.float32 else SP_BF16
+    _need(o.dtype in (torch.float32, torch.bfloat16), "o must be fp32 or bf16")
+    for t in o_parts:
+        _need(t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == (B, S, H, D), "bad o_part")
+    for t in lse_parts:
+        _need(t.dtype == torch.float32 and t.is_contiguous() and tuple(t.shape) == (B, H, S), "bad lse_part")
+    op, _keep1 = _ptr_array(o_parts)
+    lp, _keep2 = _ptr_array(lse_parts)
+    st = lib().sp_merge_partials(op, lp, n, _ptr(o), _ptr(lse), dt, B, S, H, D, _stream(stream))
+    _check("sp_merge_partials", st)
+    return o, lse
+
+
+def sp_seq_to_head_relayout(in_ranks, out_ranks, S=None, H=None, stream=None):
+    """P rank buffers [B, S/P, H, D] -> P rank buffers [B, S, H/P, D] (bit-exact)."""
+    P = len(in_ranks)
+    B, Sl, H_, D = in_ranks[0].shape
+    S = Sl * P if S is None else S
+    H = H_ if H is None else H
+    ip, _k1 = _ptr_array(in_ranks)
+    op, _k2 = _ptr_array(out_ranks)
+    st = lib().sp_seq_to_head_relayout(ip, op, P, B, S, H, D, in_ranks[0].element_size(), _stream(stream))
+    _check("sp_seq_to_head_relayout", st)
+    return out_ranks
+
+
+def sp_head_to_seq_relayout(in_ranks, out_ranks, S=None, H=None, stream=None):
+    """P rank buffers [B, S, H/P, D] -> P rank buffers [B, S/P, H, D] (bit-exact)."""
+    P = len(in_ranks)
+    B, S_, Hl, D = in_ranks[0].shape
+    S = S_ if S is None else S
+    H = Hl * P if H is None else H
+    ip, _k1 = _ptr_array(in_ranks)
+    op, _k2 = _ptr_array(out_ranks)
+    st = lib().sp_head_to_seq_relayout(ip, op, P, B, S, H, D, in_ranks[0].element_size(), _stream(stream))
+    _check("sp_head_to_seq_relayout", st)
+    return out_ranks
+
+
+def sp_build_tile_list(block_mask, S, row_ptr, col_idx, counts, stream=None):
+    """CSR of the kept key tiles of a uint8 [H, T, T] block mask (T = ceil(S/128))."""
+    H = block_mask.shape[0]
+    st = lib().sp_build_tile_list(_ptr(block_mask), H, S, _ptr(row_ptr), _ptr(col_idx), _ptr(counts),
+                                  _stream(stream))
+    _check("sp_build_tile_list", st)
+    return row_ptr, col_idx
+
+
+def sp_check_device_error(stream=None) -> int:
+    """Synchronise the stream; return SP_ERR_TIMEOUT if a bounded device wait expired since the last check."""
+    return int(lib().sp_check_device_error(_stream(stream)))
+
+
+def sp_check_device_error_bits(stream=None):
+    """(status, bits): the raw device error word, one bit per kind of wait that expired."""
+    bits = ctypes.c_uint(0)
+    st = lib().sp_check_device_error_bits(_stream(stream), ctypes.byref(bits))
+    return int(st), int(bits.value)
+
+
+def sp_set_wait_timeout_ns(ns: int) -> None:
+    lib().sp_set_wait_timeout_ns(int(ns))
+
+
+def sp_debug_wait_timeout(timeout_ns: int, stream=None) -> None:
+    _check("sp_debug_wait_timeout", lib().sp_debug_wait_timeout(int(timeout_ns), _stream(stream)))
+
+
+def declared_symbols():
+    """The entry points include/sp_attn.h declares (parsed from the header)."""
+    import re
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^\s*(?:[\w\*\s]+?)\b(sp_\w+)\s*\(", text, re.M)))

@@ -1,0 +1,153 @@
+"""The three full-size launch configurations, as steps the benchmark times and the tests check.
+
+Each step owns its device buffers (allocated once with torch), and ``run()`` enqueues one pass of its
+part of the path on the current stream through the C ABI; nothing here computes anything itself.
+
+UlyssesStep   video-DiT shape: Q, K, V arrive as P sequence shards (one buffer per simulated rank);
+              seq -> head relayout of each; attention of every rank on its H/P heads, with the global
+              head chunks split at the rank boundaries; head -> seq relayout of O back to sequence shards.
+RingStep      long causal shape: 8 contiguous KV blocks, one partial launch each (every query against one
+              block, fp32 partials), then the log-sum-exp re-merge into bf16 O and fp32 LSE.
+SparseStep    block-sparse DiT shape: tile-list build from the mask, then one attention launch that
+              skips dropped tiles.
+"""
+from __future__ import annotations
+
+import torch
+
+from . import spattn
+from .synth import TILE, Workload, split_seq
+
+
+def rank_chunks(chunks, H, P):
+    """Split a global head-chunk list at the rank boundaries (multiples of H/P).  Each rank gets the
+    chunks inside its head range; a chunk that straddles a boundary is cut there."""
+    Hl = H // P
+    out = [[] for _ in range(P)]
+    h0 = 0
+    for c in chunks:
+        a, e = h0, h0 + c
+        while a < e:
+            r = a // Hl
+            cut = min(e, (r + 1) * Hl)
+            out[r].append(cut - a)
+            a = cut
+        h0 = e
+    return out
+
+
+class UlyssesStep:
+    def __init__(self, w: Workload, q, k, v, device="cuda"):
+        self.w = w
+        P, B, S, H, D = w.ranks, w.B, w.S, w.H, w.D
+        self.P, self.Hl = P, H // P
+        self.chunks = rank_chunks(w.head_chunks or (H,), H, P)
+        self.q_seq = [t.to(device) for t in split_seq(q, P)]
+        self.k_seq = [t.to(device) for t in split_seq(k, P)]
+        self.v_seq = [t.to(device) for t in split_seq(v, P)]
+        shard = (B, S, self.Hl, D)
+        self.q_head = [torch.empty(shard, dtype=torch.bfloat16, device=device) for _ in range(P)]
+        self.k_head = [torch.empty(shard, dtype=torch.bfloat16, device=device) for _ in range(P)]
+        self.v_head = [torch.empty(shard, dtype=torch.bfloat16, device=device) for _ in range(P)]
+        self.o_head = [torch.empty(shard, dtype=torch.bfloat16, device=device) for _ in range(P)]
+        self.lse = [torch.empty((B, self.Hl, S), dtype=torch.float32, device=device) for _ in range(P)]
+        self.o_seq = [torch.empty((B, S // P, H, D), dtype=torch.bfloat16, device=device) for _ in range(P)]
+        self.launches = 3 + P + 1
+        self.flops = w.flops()
+        self.relayout_bytes = 4 * 2 * B * S * H * D * 2  # 4 tensors, each read once and written once
+
+    def relayout_in(self, stream=None):
+        spattn.sp_seq_to_head_relayout(self.q_seq, self.q_head, stream=stream)
+        spattn.sp_seq_to_head_relayout(self.k_seq, self.k_head, stream=stream)
+        spattn.sp_seq_to_head_relayout(self.v_seq, self.v_head, stream=stream)
+
+    def attention(self, stream=None):
+        for r in range(self.P):
+            spattn.sp_attn_fwd(self.q_head[r], self.k_head[r], self.v_head[r], self.o_head[r], self.lse[r],
+                               head_chunks=self.chunks[r], stream=stream)
+
+    def relayout_out(self, stream=None):
+        spattn.sp_head_to_seq_relayout(self.o_head, self.o_seq, stream=stream)
+
+    def run(self, stream=None):
+        self.relayout_in(stream)
+        self.attention(stream)
+        self.relayout_out(stream)
+
+    def lse_full(self):
+        return torch.cat(self.lse, dim=1)
+
+    def inputs(self):
+        return self.q_seq + self.k_seq + self.v_seq
+
+    def outputs(self):
+        return self.o_seq
+
+
+class RingStep:
+    def __init__(self, w: Workload, q, k, v, device="cuda"):
+        self.w = w
+        B, S, H, D = w.B, w.S, w.H, w.D
+        self.q, self.k, self.v = q.to(device), k.to(device), v.to(device)
+        n = w.n_kv_blocks
+        self.blk = (S + n - 1) // n
+        self.o_parts = [torch.empty((B, S, H, D), dtype=torch.float32, device=device) for _ in range(n)]
+        self.l_parts = [torch.empty((B, H, S), dtype=torch.float32, device=device) for _ in range(n)]
+        self.o = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty((B, H, S), dtype=torch.float32, device=device)
+        self.launches = n + 1
+        self.flops = w.flops()
+        # merge: read n fp32 partials (O and LSE), write bf16 O and fp32 LSE
+        self.merge_bytes = n * (B * S * H * D * 4 + B * H * S * 4) + B * S * H * D * 2 + B * H * S * 4
+
+    def attention(self, stream=None):
+        S = self.w.S
+        for i in range(self.w.n_kv_blocks):
+            a, e = i * self.blk, min(S, (i + 1) * self.blk)
+            spattn.sp_attn_fwd_partial(self.q, self.k, self.v, self.o_parts[i], self.l_parts[i], a, e,
+                                       causal=self.w.causal, stream=stream)
+
+    def merge(self, stream=None):
+        spattn.sp_merge_partials(self.o_parts, self.l_parts, self.o, self.lse, stream=stream)
+
+    def run(self, stream=None):
+        self.attention(stream)
+        self.merge(stream)
+
+    def workspace_for_fwd(self):
+        w = self.w
+        n = spattn.sp_attn_fwd_workspace_bytes(w.B, w.S, w.H, w.D, w.n_kv_blocks, False)
+        return torch.empty(n, dtype=torch.uint8, device=self.q.device)
+
+    def inputs(self):
+        return [self.q, self.k, self.v]
+
+    def outputs(self):
+        return [self.o]
+
+
+class SparseStep:
+    def __init__(self, w: Workload, q, k, v, mask, device="cuda"):
+        self.w = w
+        B, S, H, D = w.B, w.S, w.H, w.D
+        self.q, self.k, self.v = q.to(device), k.to(device), v.to(device)
+        self.mask = mask.to(device)
+        self.kept_tiles = int(mask.to(torch.int64).sum())
+        self.density = self.kept_tiles / float(mask.numel())
+        self.o = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty((B, H, S), dtype=torch.float32, device=device)
+        self.ws = torch.empty(spattn.sp_attn_fwd_workspace_bytes(B, S, H, D, 1, True), dtype=torch.uint8,
+                              device=device)
+        self.launches = 3 + 1
+        # algorithmic FLOPs: 4 * D * 128 * 128 per kept tile and batch (QK^T and PV, 2 FLOPs per MAC)
+        self.flops = 4.0 * B * D * TILE * TILE * self.kept_tiles
+
+    def run(self, stream=None):
+        spattn.sp_attn_fwd(self.q, self.k, self.v, self.o, self.lse, block_mask=self.mask,
+                           workspace=self.ws, stream=stream)
+
+    def inputs(self):
+        return [self.q, self.k, self.v]
+
+    def outputs(self):
+        return [self.o]

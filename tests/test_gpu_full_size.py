@@ -1,0 +1,80 @@
+"""The full-size workloads, in the launch configuration the benchmark times, checked on sampled query
+rows against the oracle (which evaluates those rows one by one over all keys)."""
+import pytest
+import torch
+
+import oracle
+from tests.helpers import assert_close, to64
+from sequence_head_attention_b200 import spattn, synth
+from sequence_head_attention_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+N_ROWS = 96
+
+
+def _oracle_rows(q, k, v, rows, **kw):
+    return oracle.attention(to64(q), to64(k), to64(v), rows=rows, **kw)
+
+
+def _sampled(o, lse, rows):
+    r = torch.tensor(rows, device=o.device)
+    return o[:, r], lse[:, :, r]
+
+
+def test_video_dit_ulysses_step():
+    w = synth.WORKLOADS["video_dit"]
+    q, k, v = synth.qkv(w.B, w.S, w.H, w.D, seed=0, scale=w.scale)
+    rows = synth.sample_rows(w.S, N_ROWS, seed=0)
+    ref = _oracle_rows(q, k, v, rows)
+    # attention on the full 40-head tensors with the uneven head chunks
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, w.H, w.S), device="cuda")
+    spattn.sp_attn_fwd(qd, kd, vd, o, lse, head_chunks=list(w.head_chunks))
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    o_s, l_s = _sampled(o, lse, rows)
+    assert_close(o_s, ref[0], l_s, ref[1])
+    # the Ulysses step the benchmark times: seq shards -> head shards -> per-rank attention -> back
+    step = workloads.UlyssesStep(w, q, k, v)
+    step.run()
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    o_full = torch.cat(step.o_seq, dim=1)
+    assert torch.equal(o_full, o)  # same per-head arithmetic, bitwise
+    lse_full = step.lse_full()
+    assert torch.equal(lse_full, lse)
+
+
+def test_ring_causal_partials_and_merge():
+    w = synth.WORKLOADS["ring_causal"]
+    q, k, v = synth.qkv(w.B, w.S, w.H, w.D, seed=0, scale=w.scale)
+    blk = w.S // w.n_kv_blocks
+    rows = synth.sample_rows(w.S, N_ROWS, seed=1, must=[blk - 1, blk, 4 * blk, 4 * blk - 1, w.S - blk])
+    ref = _oracle_rows(q, k, v, rows, causal=True)
+    step = workloads.RingStep(w, q, k, v)
+    step.run()
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    o_s, l_s = _sampled(step.o, step.lse, rows)
+    assert_close(o_s, ref[0], l_s, ref[1])
+    # one call with n_kv_blocks = 8 does the same partials and merge
+    o2 = torch.empty_like(step.o)
+    l2 = torch.empty_like(step.lse)
+    spattn.sp_attn_fwd(step.q, step.k, step.v, o2, l2, n_kv_blocks=w.n_kv_blocks, causal=True,
+                       workspace=step.workspace_for_fwd())
+    assert torch.equal(o2, step.o) and torch.equal(l2, step.lse)
+
+
+def test_block_sparse_dit():
+    w = synth.WORKLOADS["block_sparse"]
+    q, k, v = synth.qkv(w.B, w.S, w.H, w.D, seed=0, scale=w.scale)
+    mask = synth.block_mask(w.H, w.S, seed=0)
+    T = mask.shape[-1]
+    rows = synth.sample_rows(w.S, N_ROWS, seed=2, must=[128 * t + 3 for t in range(0, T, 9)])
+    ref = _oracle_rows(q, k, v, rows, block_mask=mask.numpy())
+    step = workloads.SparseStep(w, q, k, v, mask)
+    step.run()
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    o_s, l_s = _sampled(step.o, step.lse, rows)
+    assert_close(o_s, ref[0], l_s, ref[1])
