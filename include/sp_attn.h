@@ -150,6 +150,30 @@ SP_API sp_status sp_head_to_seq_relayout(const void* const* in_ranks, void* cons
                                   int S, int H, int D, int elem_bytes, sp_stream stream);
 
 /*
+ * Block-sparse attention that allocates nothing, for callers that cannot call cudaMalloc (a serving
+ * path that must not block on the device synchronisation an allocation may cause, a plug-in handed
+ * tensors by a framework that owns all device memory, a real-time loop that forbids allocation after
+ * start-up).  The pages have no counterpart for this entry point: it exists for those callers only.
+ *
+ * Computes exactly what sp_attn_fwd computes with this block_mask, one head chunk and n_kv_blocks = 1
+ * (same kernels, same results).  The scratch that sp_attn_fwd takes from the caller's workspace (the
+ * mask's compacted tile list) lives instead in a fixed array inside the library, 12,714,240 bytes, which
+ * every GPU that loads the library keeps until the process exits.  Limits: H * ceil(S/128) <=
+ * SP_NOALLOC_MAX_TILE_ROWS and H * ceil(S/128)^2 <= SP_NOALLOC_MAX_TILES; larger problems return
+ * SP_ERR_UNSUPPORTED with nothing launched.
+ * The first call on a device looks up that array's device address (cudaGetSymbolAddress with the
+ * device current); make that first call before any stream capture.  Every call on a device shares the
+ * array and leaves its tile list in it (nothing needs to start at zero: each call rewrites what it
+ * reads), so calls whose execution overlaps on the GPU race; order them on one stream or with events.
+ * Arguments as in sp_attn_fwd; block_mask is required.
+ */
+#define SP_NOALLOC_MAX_TILE_ROWS 16384
+#define SP_NOALLOC_MAX_TILES (3 * 1024 * 1024)
+SP_API sp_status sp_attn_fwd_sparse_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                            int B, int S, int H, int D, int causal, const uint8_t* block_mask,
+                                            sp_stream stream);
+
+/*
  * Compacted tile list of a block mask, the form in which the attention kernels skip dropped tiles
  * ("db-SP", abstract: dense blocks irregularly distributed in a per-head mask).
  *   block_mask device uint8 [H, T, T], T = ceil(S/128); nonzero = keep.

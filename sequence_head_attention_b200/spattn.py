@@ -53,6 +53,7 @@ def lib() -> ctypes.CDLL:
                 "sp_seq_to_head_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_head_to_seq_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_build_tile_list": (I, [P, I, I, P, P, P, P]),
+                "sp_attn_fwd_sparse_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, P, P]),
                 "sp_status_string": (ctypes.c_char_p, [I]),
                 "sp_check_device_error": (I, [P]),
                 "sp_check_device_error_bits": (I, [P, P]),
@@ -211,6 +212,22 @@ def sp_head_to_seq_relayout(in_ranks, out_ranks, S=None, H=None, stream=None):
     st = lib().sp_head_to_seq_relayout(ip, op, P, B, S, H, D, in_ranks[0].element_size(), _stream(stream))
     _check("sp_head_to_seq_relayout", st)
     return out_ranks
+
+
+def sp_attn_fwd_sparse_noalloc(q, k, v, o, lse, block_mask, causal=False, stream=None):
+    """Block-sparse attention with no workspace: for callers that cannot allocate device memory.
+
+    Same result as sp_attn_fwd(..., block_mask=block_mask); the mask's tile list goes into a fixed
+    array inside the library instead (size limits and the no-overlap rule in include/sp_attn.h)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _bshd(t, n)
+    B, S, H, D = q.shape
+    _need(block_mask is not None and block_mask.dtype == torch.uint8 and block_mask.is_contiguous(),
+          "block_mask must be a contiguous uint8 tensor")
+    st = lib().sp_attn_fwd_sparse_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, S, H, D,
+                                          int(bool(causal)), _ptr(block_mask), _stream(stream))
+    _check("sp_attn_fwd_sparse_noalloc", st)
+    return o, lse
 
 
 def sp_build_tile_list(block_mask, S, row_ptr, col_idx, counts, stream=None):
