@@ -185,12 +185,14 @@ def calibrated_oracle_baseline(wname, q, k, v, mask, target_s=15.0):
 
 
 # ----------------------------------------------------------------------------------------------------
-def build_inputs(wname: str, seed: int, seq_len: int = 0):
+def build_inputs(wname: str, seed: int, seq_len: int = 0, ranks: int = 0):
     import dataclasses
     from sequence_head_attention_b200 import synth
     w = synth.WORKLOADS[wname]
     if seq_len:
         w = dataclasses.replace(w, S=seq_len)
+    if ranks:
+        w = dataclasses.replace(w, ranks=ranks)
     q, k, v = synth.qkv(w.B, w.S, w.H, w.D, seed=seed, scale=w.scale)
     mask = synth.block_mask(w.H, w.S, seed=seed) if w.sparse else None
     return w, q, k, v, mask
@@ -251,7 +253,7 @@ def run_ours(args):
     init_dist("nccl", timeout_s=180)
     spattn.lib()  # fail now if the library is missing
 
-    w, q, k, v, mask = build_inputs(args.workload, seed=rank, seq_len=args.seq_len)
+    w, q, k, v, mask = build_inputs(args.workload, seed=rank, seq_len=args.seq_len, ranks=args.ranks)
     if args.workload == "video_dit":
         step = workloads.UlyssesStep(w, q, k, v, device=dev)
     elif args.workload == "ring_causal":
@@ -400,6 +402,8 @@ def main(argv=None):
     ap.add_argument("--ref-rows", type=int, default=16, help="query rows per reference step")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override S (profiling captures on a smaller case; not a benchmark number)")
+    ap.add_argument("--ranks", type=int, default=0,
+                    help="override the simulated rank count of video_dit (profiling captures only)")
     args = ap.parse_args(argv)
     if args.impl == "reference":
         return run_reference(args)
