@@ -128,6 +128,25 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
+def recorded_traffic():
+    """DRAM bytes per attention launch from the committed ncu summary, if it was taken on the current
+    kernel sources (their sha256 is recorded beside it); otherwise None."""
+    import hashlib
+    import re
+    path = os.path.join(ROOT, "profiles", "attn_fwd_kernel_video_dit.md")
+    try:
+        text = open(path).read()
+        h = hashlib.sha256()
+        for f in ("attn_fwd.cu", "sp_ptx.cuh"):
+            with open(os.path.join(ROOT, "sequence_head_attention_b200", "csrc", f), "rb") as fh:
+                h.update(fh.read())
+        sha = re.search(r"kernel_sources_sha256: ([0-9a-f]{64})", text).group(1)
+        val = int(re.search(r"traffic_bytes_per_launch: (\d+)", text).group(1))
+    except (OSError, AttributeError, ValueError):
+        return None
+    return val if sha == h.hexdigest() else None
+
+
 def measured_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -338,7 +357,9 @@ def run_ours(args):
     achieved = flops_launch / (attn_ms / 1000.0) / 1e12
     kernels["attention"] = {"tflops": achieved, "ms_per_launch": attn_ms}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops_sustained"], "traffic": None,
+                "frac": achieved / peaks["bf16_tflops_sustained"],
+                "traffic": recorded_traffic() if args.workload == "video_dit" and not args.seq_len and not args.ranks else None,
+                "traffic_unit": "bytes per launch (dram read + write, ncu, profiles/attn_fwd_kernel_video_dit.md)",
                 "peak_kind": f"{peaks['source']} bf16 dense, sustained (kernel timed inside a long step)",
                 "frac_of_burst_peak": achieved / peaks["bf16_tflops"]}
 

@@ -211,6 +211,14 @@ SP_API void sp_set_wait_timeout_ns(unsigned long long ns);
  */
 SP_API sp_status sp_debug_wait_timeout(unsigned long long timeout_ns, sp_stream stream);
 
+/*
+ * Evaluates, on the GPU, the exponential 2^x that the attention kernels compute on the FMA pipe for part
+ * of each softmax row (range split x = n + f, a minimax cubic for 2^f, 2^n through the exponent), for
+ * testing it against CUDA's exp2f.  x, y: device fp32 arrays of n elements, n even.  Inputs below -125
+ * are clamped to -125.
+ */
+SP_API sp_status sp_debug_exp2_poly(const float* x, float* y, int n, sp_stream stream);
+
 /* Library version string. */
 SP_API const char* sp_version(void);
 

@@ -193,6 +193,11 @@ sp_status sp_debug_wait_timeout(unsigned long long timeout_ns, sp_stream stream)
   return launch_debug_wait(timeout_ns, as_stream(stream));
 }
 
+sp_status sp_debug_exp2_poly(const float* x, float* y, int n, sp_stream stream) {
+  if (!x || !y || n < 0 || (n & 1)) return SP_ERR_INVALID_ARG;
+  return launch_debug_exp2_poly(x, y, n, as_stream(stream));
+}
+
 sp_status sp_build_tile_list(const uint8_t* block_mask, int H, int S, int32_t* row_ptr, int32_t* col_idx,
                              int32_t* counts, sp_stream stream) {
   if (!block_mask || !row_ptr || !col_idx || !counts || H < 1 || S < 1) return SP_ERR_INVALID_ARG;

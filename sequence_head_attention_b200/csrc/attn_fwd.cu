@@ -12,15 +12,20 @@
 //   CTA; they share every K/V tile that both need.
 //   warp 8      TMA producer: Q tiles of both lanes, then K_j, V_j tiles into a ring of shared-memory
 //               slots (128B-swizzled, the tensor cores' canonical layout).
-//   warp 9      MMA issuer (one thread): S_t = Q_t K_j^T into TMEM (fp32), and O_t += P_t V_j with P_t
-//               read from TMEM and V_j from shared memory; tcgen05.commit signals completions.
+//   warps 9,10  MMA issuers, one per lane: S_t = Q_t K_j^T into TMEM (fp32), and O_t += P_t V_j with
+//               P_t read from TMEM and V_j from shared memory; tcgen05.commit signals completions.
 //   warps 0-7   softmax, 4 warps per lane: thread r owns query row r of its lane's tile, loads its row
 //               of S from TMEM (so every row reduction stays inside one thread), keeps the running
 //               maximum m and sum l, writes P = exp(S - m) as bf16 back into TMEM over S, rescales
 //               the O row in TMEM when the maximum grows by more than 2^8, and finally writes
-//               O / l and lse = (m + log2 l) ln 2.
+//               O / l and lse = (m + log2 l) ln 2.  The two lanes take turns at the exponentials
+//               (ping-pong), so each has the MUFU unit to itself while the tensor core runs the
+//               other lane's MMAs.
+//   warp 11     idle (it completes the third warpgroup, which gives its registers to the softmax).
 //   TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256, 256+D), O_1 [256+D, 256+2D); P_t
-//   overwrites the first 64 columns of S_t.
+//   overwrites the first 64 columns of S_t.  Each lane's issuer queues S_t(j+1) right behind
+//   O_t += P_t(j) V_j: MMAs from one thread execute in issue order, so S_t(j+1) cannot overwrite P_t(j)
+//   before the P V has read it.
 // Every barrier wait is bounded in time; on expiry the kernel records an error and returns cleanly.
 #include <climits>
 #include <cstdint>
@@ -33,10 +38,22 @@ namespace spattn {
 namespace {
 
 constexpr int kTile = 128;
-constexpr int kThreads = 320;
+// 12 warps: 0-7 softmax (two warpgroups), 8 TMA producer, 9 and 10 MMA issuers (lanes 0 and 1),
+// 11 idle.  Launched with
+// kRegsLaunch registers per thread; the producer/MMA warpgroup gives registers back (kRegsControl)
+// and the softmax warpgroups take them (kRegsSoftmax): 128 * 104 + 256 * 200 = 384 * 168.
+constexpr int kThreads = 384;
 constexpr int kWarpProducer = 8;
-constexpr int kWarpMma = 9;
+constexpr int kWarpMma = 9;  // MMA issuer of lane 0; kWarpMma + 1 issues for lane 1
+constexpr int kRegsLaunch = 168;
+constexpr uint32_t kRegsControl = 104;
+constexpr uint32_t kRegsSoftmax = 200;
+static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and l are rescaled when m grows by > 2^8
+#ifndef SP_EXP2_POLY_PAIRS
+#define SP_EXP2_POLY_PAIRS 0  // of every 8 pairs of exponentials, this many run on the FMA pipe
+#endif
+constexpr int kPolyPairs = SP_EXP2_POLY_PAIRS;
 
 template <int D>
 struct Cfg {
@@ -47,8 +64,8 @@ struct Cfg {
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2], drain, and
-  // two 8-byte slots for the o_done counters
-  static constexpr int kNumBars = 2 + 2 * kStages + 9;
+  // 8-byte slots for the o_done[2] and turn[2] counters
+  static constexpr int kNumBars = 2 + 2 * kStages + 11;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
@@ -58,7 +75,7 @@ struct Cfg {
 };
 
 struct Bars {
-  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, pv_done0, o_done0, drain;
+  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, pv_done0, o_done0, turn0, drain;
   __device__ uint32_t kv_full(int s) const { return kv_full0 + 8u * s; }
   __device__ uint32_t kv_empty(int s) const { return kv_empty0 + 8u * s; }
   __device__ uint32_t s_full(int t) const { return s_full0 + 8u * t; }
@@ -66,6 +83,11 @@ struct Bars {
   __device__ uint32_t pv_done(int t) const { return pv_done0 + 8u * t; }
   // o_done[t]: a counter, +1 per softmax warp of lane t per finished item (epilogue reads of O done)
   __device__ uint32_t o_done(int t) const { return o_done0 + 8u * t; }
+  // turn[t]: a counter, +1 per softmax warp of lane t per union step it has finished (or skipped).  The
+  // two lanes take turns at their exponentials (ping-pong), so each has the MUFU unit to itself while
+  // the tensor core runs the other lane's MMAs; a monotonic count cannot alias however far a lane that
+  // skips steps runs ahead.
+  __device__ uint32_t turn(int t) const { return turn0 + 8u * t; }
 };
 
 struct Item {
@@ -183,7 +205,8 @@ struct StepIter {
 };
 
 // ------------------------------------------------------------------------------------------------
-// Producer: one thread issues all TMA loads.
+// Producer: one warp walks the work in lockstep (all values warp-uniform); one elected lane issues the
+// TMA loads.
 // ------------------------------------------------------------------------------------------------
 template <int D>
 __device__ void run_producer(const AttnParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
@@ -191,6 +214,7 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tq, const C
                              volatile int* abort_flag) {
   using C = Cfg<D>;
   const uint32_t sbase = smem_u32(smem);
+  const uint64_t tmo = p.timeout_ns;
   uint32_t q_empty_ph = 0;
   int ring = 0;
   int n_item = 0;
@@ -199,161 +223,188 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tq, const C
   for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++n_item) {
     const Item it = decode_item(p, w);
     if (n_item > 0) {
-      ok = mbar_wait(bars.q_empty, q_empty_ph, p.timeout_ns, ERR_TIMEOUT_Q_EMPTY, abort_flag, p.err);
+      ok = warp_mbar_wait(bars.q_empty, q_empty_ph, tmo, ERR_TIMEOUT_Q_EMPTY, abort_flag, p.err);
       q_empty_ph ^= 1;
       if (!ok) break;
     }
-    mbar_arrive_expect_tx(bars.q_full, 2 * C::kTileBytes);
+    if (elect_one_sync()) {
+      mbar_arrive_expect_tx(bars.q_full, 2 * C::kTileBytes);
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
+      for (int t = 0; t < 2; ++t)
 #pragma unroll
-      for (int c = 0; c < C::kSub; ++c)
-        tma_load_4d(sbase + C::kQOff + t * C::kTileBytes + c * 16384, tq, bars.q_full, 64 * c, it.h,
-                    it.q_start[t], it.b);
+        for (int c = 0; c < C::kSub; ++c)
+          tma_load_4d(sbase + C::kQOff + t * C::kTileBytes + c * 16384, tq, bars.q_full, 64 * c, it.h,
+                      it.q_start[t], it.b);
+    }
+    __syncwarp();
     last_q_item = n_item;
     StepIter st;
     st.init(p, it);
     int kv_start;
     bool k0, k1;
-    while (st.next(kv_start, k0, k1)) {
+    while (ok && st.next(kv_start, k0, k1)) {
 #pragma unroll
       for (int kv = 0; kv < 2; ++kv) {
         const int slot = ring % C::kStages;
         const int lap = ring / C::kStages;
         if (lap > 0) {
-          ok = mbar_wait(bars.kv_empty(slot), (lap - 1) & 1, p.timeout_ns, ERR_TIMEOUT_KV_EMPTY, abort_flag, p.err);
+          ok = warp_mbar_wait(bars.kv_empty(slot), (lap - 1) & 1, tmo, ERR_TIMEOUT_KV_EMPTY, abort_flag, p.err);
           if (!ok) break;
         }
-        mbar_arrive_expect_tx(bars.kv_full(slot), C::kTileBytes);
-        const CUtensorMap* tm = kv == 0 ? tk : tv;
+        if (elect_one_sync()) {
+          mbar_arrive_expect_tx(bars.kv_full(slot), C::kTileBytes);
+          const CUtensorMap* tm = kv == 0 ? tk : tv;
 #pragma unroll
-        for (int c = 0; c < C::kSub; ++c)
-          tma_load_4d(sbase + C::kKVOff + slot * C::kTileBytes + c * 16384, tm, bars.kv_full(slot), 64 * c,
-                      it.h, kv_start, it.b);
+          for (int c = 0; c < C::kSub; ++c)
+            tma_load_4d(sbase + C::kKVOff + slot * C::kTileBytes + c * 16384, tm, bars.kv_full(slot), 64 * c,
+                        it.h, kv_start, it.b);
+        }
+        __syncwarp();
         ++ring;
       }
-      if (!ok) break;
     }
   }
   if (*abort_flag) {
     // Do not leave copies in flight into shared memory: wait (bounded) for the most recent load of
     // every slot and for the last Q load.
-    const uint64_t tmo = p.timeout_ns;
     for (int pos = max(0, ring - C::kStages); pos < ring; ++pos)
-      mbar_wait(bars.kv_full(pos % C::kStages), (pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, nullptr, p.err);
-    if (last_q_item >= 0) mbar_wait(bars.q_full, last_q_item & 1, tmo, ERR_TIMEOUT_Q_FULL, nullptr, p.err);
+      warp_mbar_wait(bars.kv_full(pos % C::kStages), (pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, nullptr, p.err);
+    if (last_q_item >= 0) warp_mbar_wait(bars.q_full, last_q_item & 1, tmo, ERR_TIMEOUT_Q_FULL, nullptr, p.err);
   }
 }
 
 // ------------------------------------------------------------------------------------------------
-// MMA issuer: one thread.
+// MMA issuers: one warp per lane walks the work in lockstep (all values warp-uniform, so descriptors
+// stay in uniform registers); one elected lane issues the tcgen05 instructions.  With a warp per lane,
+// one lane's waits (for its P, or for its previous P V) never hold up the other lane's MMAs; the tensor
+// core interleaves the two lanes.  Shared K/V slots and the Q buffer are released when both lanes are
+// done with them (the "empty" barriers count two arrivals; a lane that skips a tile arrives directly).
 // ------------------------------------------------------------------------------------------------
 template <int D>
-__device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, uint32_t tmem,
+__device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, uint32_t tmem_in, int t,
                         volatile int* abort_flag) {
   using C = Cfg<D>;
   const uint32_t sbase = smem_u32(smem);
   const uint64_t tmo = p.timeout_ns;
-  uint32_t q_full_ph = 0;
-  uint32_t p_full_ph[2] = {0, 0}, pv_done_ph[2] = {0, 0};
-  bool pv_pending[2] = {false, false};
+  const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_in, 0);  // provably warp-uniform
+  // Descriptors of K-step 0; later K-steps add their byte offset / 16 to the start-address field.
+  const uint64_t q_desc = smem_desc_sw128(sbase + C::kQOff + t * C::kTileBytes, 16, 1024);
+  const uint64_t kv_desc0 = smem_desc_sw128(sbase + C::kKVOff, 16, 1024);
+  const uint64_t v_desc0 = smem_desc_sw128(sbase + C::kKVOff, 16384, 1024);
+  const uint32_t s_tmem = tmem + C::kColS + t * 128;  // S_t, and P_t over its first 64 columns
+  const uint32_t o_tmem = tmem + C::kColO + t * D;
+  const uint32_t s_full = bars.s_full(t), p_full = bars.p_full(t), pv_done = bars.pv_done(t);  // pv_done: for the epilogue
+  uint32_t q_full_ph = 0, p_full_ph = 0;
   int ring = 0;
   int n_item = 0;
   bool ok = true;
   for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++n_item) {
     const Item it = decode_item(p, w);
-    ok = mbar_wait(bars.q_full, q_full_ph, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
+    ok = warp_mbar_wait(bars.q_full, q_full_ph, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
     q_full_ph ^= 1;
     if (!ok) break;
     tc_fence_after();
     // O_t may be overwritten by this item's first P V only after the 4 softmax warps of lane t have
     // read out the previous item's O: o_done[t] counts 4 per finished item.
-    bool need_odone[2] = {n_item > 0, n_item > 0};
-    bool first_pv[2] = {true, true};
+    bool need_odone = n_item > 0;
+    bool first_pv = true;
     StepIter st;
     st.init(p, it);
-    bool prev_has = false, prev_keep[2] = {false, false};
+    bool prev_has = false, prev_keep = false;
     int prev_v_pos = 0;
-    bool prev_v_waited = false;
     for (;;) {
       int kv_start;
-      bool keep[2];
-      const bool has = st.next(kv_start, keep[0], keep[1]);
+      bool k0, k1;
+      const bool has = st.next(kv_start, k0, k1);
+      const bool keep = has && (t ? k1 : k0);
       const int k_pos = ring;
-      bool k_waited = false;
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (prev_has && prev_keep[t]) {
-          if (!prev_v_waited) {
-            ok = mbar_wait(bars.kv_full(prev_v_pos % C::kStages), (prev_v_pos / C::kStages) & 1, tmo,
-                           ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
-            if (!ok) break;
-            prev_v_waited = true;
+      // O_t += P_t V_{j-1} for the previous step (or release V_{j-1} if this lane did not use it).
+      if (prev_has) {
+        const int vs = prev_v_pos % C::kStages;
+        if (prev_keep) {
+          ok = warp_mbar_wait(bars.kv_full(vs), (prev_v_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
+                              abort_flag, p.err);
+          if (ok && need_odone) {
+            ok = warp_counter_wait(bars.o_done(t), 4u * (uint32_t)n_item, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err);
+            need_odone = false;
           }
-          if (need_odone[t]) {
-            ok = counter_wait(bars.o_done(t), 4u * (uint32_t)n_item, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err);
-            need_odone[t] = false;
-            if (!ok) break;
+          if (ok) {
+            ok = warp_mbar_wait(p_full, p_full_ph, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
+            p_full_ph ^= 1;
           }
-          ok = mbar_wait(bars.p_full(t), p_full_ph[t], tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
-          p_full_ph[t] ^= 1;
           if (!ok) break;
           tc_fence_after();
-          const uint32_t v_addr = sbase + C::kKVOff + (prev_v_pos % C::kStages) * C::kTileBytes;
+          const uint64_t v_desc = v_desc0 + (uint64_t)((vs * C::kTileBytes) >> 4);
+          const uint32_t acc0 = first_pv ? 0u : 1u;
+          if (elect_one_sync()) {
 #pragma unroll
-          for (int kk = 0; kk < kTile / 16; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(v_addr + kk * 2048, 16384, 1024);
-            mma_ts(tmem + C::kColO + t * D, tmem + C::kColS + t * 128 + kk * 8, bdesc, C::kIdescPV,
-                   (first_pv[t] && kk == 0) ? 0u : 1u);
+            for (int kk = 0; kk < kTile / 16; ++kk)
+              mma_ts(o_tmem, s_tmem + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
+            mma_commit(pv_done);
+            mma_commit(bars.kv_empty(vs));
           }
-          first_pv[t] = false;
-          mma_commit(bars.pv_done(t));
-          pv_pending[t] = true;
-        }
-        if (has && keep[t]) {
-          if (!k_waited) {
-            ok = mbar_wait(bars.kv_full(k_pos % C::kStages), (k_pos / C::kStages) & 1, tmo,
-                           ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
-            if (!ok) break;
-            k_waited = true;
-            tc_fence_after();
-          }
-          if (pv_pending[t]) {
-            ok = mbar_wait(bars.pv_done(t), pv_done_ph[t], tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err);
-            pv_done_ph[t] ^= 1;
-            pv_pending[t] = false;
-            if (!ok) break;
-            tc_fence_after();
-          }
-          const uint32_t q_addr = sbase + C::kQOff + t * C::kTileBytes;
-          const uint32_t k_addr = sbase + C::kKVOff + (k_pos % C::kStages) * C::kTileBytes;
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk / 4) * 16384 + (kk % 4) * 32;
-            const uint64_t adesc = smem_desc_sw128(q_addr + off, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(k_addr + off, 16, 1024);
-            mma_ss(tmem + C::kColS + t * 128, adesc, bdesc, C::kIdescS, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(bars.s_full(t));
+          __syncwarp();
+          first_pv = false;
+        } else {
+          // Not used by this lane: still wait for its load, so that this warp consumes every phase
+          // of every slot in order (a skipped phase would let a later parity wait see a stale one).
+          ok = warp_mbar_wait(bars.kv_full(vs), (prev_v_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
+                              abort_flag, p.err);
+          if (!ok) break;
+          if (elect_one_sync()) mbar_arrive(bars.kv_empty(vs));
+          __syncwarp();
         }
       }
-      if (!ok) break;
-      if (prev_has) mma_commit(bars.kv_empty(prev_v_pos % C::kStages));
       if (!has) break;
-      mma_commit(bars.kv_empty(k_pos % C::kStages));
+      // S_t = Q_t K_j^T.  It overwrites P_t, which the P V just issued reads: tcgen05.mma operations
+      // issued by one thread execute in issue order, so no wait is needed here, and the commit below
+      // (which fires once all earlier MMAs of this thread are complete) also tells the softmax that
+      // O_t is no longer being written.
+      const int ks = k_pos % C::kStages;
+      if (keep) {
+        ok = warp_mbar_wait(bars.kv_full(ks), (k_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t k_desc = kv_desc0 + (uint64_t)((ks * C::kTileBytes) >> 4);
+        if (elect_one_sync()) {
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+            mma_ss(s_tmem, q_desc + off, k_desc + off, C::kIdescS, kk > 0 ? 1u : 0u);
+          }
+          mma_commit(s_full);
+          mma_commit(bars.kv_empty(ks));
+        }
+        __syncwarp();
+      } else {
+        ok = warp_mbar_wait(bars.kv_full(ks), (k_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+        if (!ok) break;
+        if (elect_one_sync()) mbar_arrive(bars.kv_empty(ks));
+        __syncwarp();
+      }
       ring += 2;
       prev_has = true;
-      prev_keep[0] = keep[0];
-      prev_keep[1] = keep[1];
+      prev_keep = keep;
       prev_v_pos = k_pos + 1;
-      prev_v_waited = false;
     }
     if (!ok) break;
-    mma_commit(bars.q_empty);  // every S MMA that read this item's Q tiles has been issued
+    if (elect_one_sync()) mma_commit(bars.q_empty);  // this lane's S MMAs of the item are all issued
+    __syncwarp();
   }
   // Drain: nothing of ours may still run on the tensor cores when TMEM is released.
-  mma_commit(bars.drain);
-  mbar_wait(bars.drain, 0, tmo, ERR_TIMEOUT_DRAIN, nullptr, p.err);
+  if (elect_one_sync()) mma_commit(bars.drain);
+  __syncwarp();
+  warp_mbar_wait(bars.drain, 0, tmo, ERR_TIMEOUT_DRAIN, nullptr, p.err);
+}
+
+// Ping-pong between the two softmax lanes: lane 0 starts the exponentials of union step u once lane 1 is
+// done with step u - 1 (turn[1] >= 4u), lane 1 once lane 0 is done with step u (turn[0] >= 4(u + 1)).
+__device__ __forceinline__ bool take_turn(const Bars& bars, int lane_t, uint32_t u, uint64_t tmo,
+                                          volatile int* abort_flag, unsigned int* err) {
+  return warp_counter_wait(bars.turn(lane_t ^ 1), 4u * (lane_t ? u + 1u : u), tmo, ERR_TIMEOUT_TURN, abort_flag, err);
+}
+__device__ __forceinline__ void pass_turn(const Bars& bars, int lane_t) {
+  smem_counter_add_release(bars.turn(lane_t), 1u);
 }
 
 // ------------------------------------------------------------------------------------------------
@@ -373,6 +424,7 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, uint32_t tmem
   const float scale_log2 = p.scale_log2;
   uint32_t s_full_ph = 0;
   uint32_t total_pv = 0;
+  uint32_t union_step = 0;  // union steps walked so far, over all items (identical in both lanes)
   bool ok = true;
 
   for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
@@ -388,7 +440,12 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, uint32_t tmem
     int kv_start;
     bool k0, k1;
     while (st.next(kv_start, k0, k1)) {
-      if (!(lane_t == 0 ? k0 : k1)) continue;
+      const uint32_t u = union_step++;
+      if (!(lane_t == 0 ? k0 : k1)) {  // this lane skips the step: its turn is over at once
+        __syncwarp();
+        if (lane == 0) pass_turn(bars, lane_t);
+        continue;
+      }
       ok = mbar_wait(bars.s_full(lane_t), s_full_ph, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err);
       ok = __all_sync(0xffffffffu, ok);
       s_full_ph ^= 1;
@@ -398,6 +455,7 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, uint32_t tmem
 #pragma unroll
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
       tmem_wait_ld();
+#define SV(i) __uint_as_float(sr[(i) >> 5][(i) & 31])
       // Keys past the KV range, past S, or (causal) after this query: -inf.
       const int n_valid = lim_row - kv_start;
       if (__any_sync(0xffffffffu, n_valid < kTile)) {
@@ -407,11 +465,20 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, uint32_t tmem
           for (int e = 0; e < 32; ++e)
             if (c * 32 + e >= n_valid) sr[c][e] = __float_as_uint(-INFINITY);
       }
-      float mx = -INFINITY;
+      // Row maximum: eight independent chains of three-input maxima, then a small tree.
+      float mx8[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(SV(2 * k), SV(2 * k + 1));
 #pragma unroll
-        for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(sr[c][e]));
+      for (int i = 16; i < 128; i += 16)
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = fmax3f(mx8[k], SV(i + 2 * k), SV(i + 2 * k + 1));
+      const float mx = fmax3f(fmax3f(mx8[0], mx8[1], mx8[2]), fmax3f(mx8[3], mx8[4], mx8[5]),
+                              fmaxf(mx8[6], mx8[7]));
+      // Ping-pong: lane 0 starts step u's exponentials once lane 1 is done with step u - 1, lane 1 once
+      // lane 0 is done with step u.
+      ok = take_turn(bars, lane_t, u, tmo, abort_flag, p.err);
+      if (!ok) break;
       const float m_tile = mx * scale_log2;
       const bool grow = m_tile > m_used + kRescaleThreshold;
       float alpha = 1.f;
@@ -421,8 +488,9 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, uint32_t tmem
         m_used = m_tile;
       }
       if (n_kept > 0 && __any_sync(0xffffffffu, grow)) {
-        // O row *= alpha.  The previous O += P V of this lane has completed: S_t was only issued
-        // after it, and its next one waits for this thread's P.
+        // O row *= alpha.  The previous O += P V of this lane has completed (the S_t commit that
+        // signalled this step fires only after every earlier MMA of its issuer), and the next one
+        // waits for this thread's P.
 #pragma unroll 1
         for (int c = 0; c < D / 16; ++c) {
           uint32_t o[16];
@@ -434,29 +502,44 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, uint32_t tmem
         }
       }
       const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
-      float rowsum = 0.f;
-      // P (bf16, two per column) over the first 64 columns of S_t: the A operand of O += P V.  Each
-      // half is stored as soon as it is packed, so its registers are free for the next half.
+      const f2 sc2 = {scale_log2, scale_log2};
+      const f2 nm2 = {neg_m, neg_m};
+      f2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+      // P = 2^(s * scale - m), bf16, two per column over the first 64 columns of S_t: the A operand of
+      // O += P V.  Each quarter is stored as soon as it is packed.  Of every 8 pairs, kPolyPairs go
+      // through the FMA-pipe polynomial and the rest through ex2.approx, so neither pipe saturates.
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t pk[32];
+      for (int quarter = 0; quarter < 4; ++quarter) {
+        uint32_t pk[16];
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2)
-#pragma unroll
-          for (int e = 0; e < 32; e += 2) {
-            const int c = half * 2 + c2;
-            const float p0 = ex2_approx(fmaf(__uint_as_float(sr[c][e]), scale_log2, neg_m));
-            const float p1 = ex2_approx(fmaf(__uint_as_float(sr[c][e + 1]), scale_log2, neg_m));
-            rowsum += p0 + p1;
-            pk[c2 * 16 + (e >> 1)] = pack_bf16x2(p0, p1);
+        for (int e = 0; e < 32; e += 2) {
+          const int i = quarter * 32 + e;
+          const f2 x = ffma2(f2{SV(i), SV(i + 1)}, sc2, nm2);
+          f2 pr;
+          if (((e >> 1) & 7) >= 8 - kPolyPairs) {
+            pr = exp2_poly2(x);
+          } else {
+            pr.x = ex2_approx(x.x);
+            pr.y = ex2_approx(x.y);
           }
-        tmem_st32(tS + half * 32, pk);
+          acc[(e >> 1) & 3] = fadd2(acc[(e >> 1) & 3], pr);
+          pk[e >> 1] = pack_bf16x2(pr.x, pr.y);
+        }
+        tmem_st16(tS + quarter * 16, pk);
       }
+#undef SV
+      const f2 acc01 = fadd2(acc[0], acc[1]);
+      const f2 acc23 = fadd2(acc[2], acc[3]);
+      const f2 acc4 = fadd2(acc01, acc23);
+      const float rowsum = acc4.x + acc4.y;
       l += rowsum;
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars.p_full(lane_t));
+      if (lane == 0) {
+        mbar_arrive(bars.p_full(lane_t));
+        pass_turn(bars, lane_t);
+      }
       ++n_kept;
       ++total_pv;
     }
@@ -470,7 +553,9 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, uint32_t tmem
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        const float inv_l = l > 0.f ? 1.f / l : 0.f;
+        // A row that never saw a visible key is exactly 0 (the FMA-pipe exponentials of its masked
+        // entries are tiny but not zero).
+        const float inv_l = (l > 0.f && m_used != -INFINITY) ? 1.f / l : 0.f;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -506,7 +591,7 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, uint32_t tmem
       }
       if (row_ok && p.lse)
         p.lse[((size_t)it.b * p.H + it.h) * p.S + q_row] =
-            l > 0.f ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+            (l > 0.f && m_used != -INFINITY) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
     tc_fence_before();
     __syncwarp();
@@ -531,7 +616,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   bars.p_full0 = bars.s_full0 + 16;
   bars.pv_done0 = bars.p_full0 + 16;
   bars.o_done0 = bars.pv_done0 + 16;
-  bars.drain = bars.o_done0 + 16;
+  bars.turn0 = bars.o_done0 + 16;
+  bars.drain = bars.turn0 + 16;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   const int warp = threadIdx.x >> 5;
@@ -539,19 +625,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(bars.q_full, 1);
-    mbar_init(bars.q_empty, 1);
+    mbar_init(bars.q_empty, 2);  // one arrival per MMA warp
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bars.kv_full(s), 1);
-      mbar_init(bars.kv_empty(s), 1);
+      mbar_init(bars.kv_empty(s), 2);  // one arrival per MMA warp
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bars.s_full(t), 1);
       mbar_init(bars.p_full(t), 4);   // one arrival per softmax warp
       mbar_init(bars.pv_done(t), 1);
     }
-    *reinterpret_cast<volatile uint32_t*>(smem + C::kBarOff + (bars.o_done0 - bar0)) = 0u;
-    *reinterpret_cast<volatile uint32_t*>(smem + C::kBarOff + (bars.o_done0 - bar0) + 8) = 0u;
-    mbar_init(bars.drain, 1);
+    for (int k = 0; k < 4; ++k)  // o_done[0..1], turn[0..1] counters
+      *reinterpret_cast<volatile uint32_t*>(smem + C::kBarOff + (bars.o_done0 - bar0) + 8 * k) = 0u;
+    mbar_init(bars.drain, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -570,12 +656,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
 
   if (warp < 8) {
+    regs_inc<kRegsSoftmax>();
     run_softmax<D>(p, bars, tmem, warp >> 2, abort_flag);
-  } else if (warp == kWarpProducer) {
-    if (lane == 0) run_producer<D>(p, &tq, &tk, &tv, smem, bars, abort_flag);
-    __syncwarp();
   } else {
-    if (lane == 0) run_mma<D>(p, smem, bars, tmem, abort_flag);
+    regs_dec<kRegsControl>();
+    if (warp == kWarpProducer) {
+      run_producer<D>(p, &tq, &tk, &tv, smem, bars, abort_flag);
+    } else if (warp == kWarpMma || warp == kWarpMma + 1) {
+      run_mma<D>(p, smem, bars, tmem, warp - kWarpMma, abort_flag);
+    }
     __syncwarp();
   }
   tc_fence_before();
@@ -606,6 +695,19 @@ sp_status launch_attn(const AttnParams& p_in, const void* q, const void* k, cons
   const int grid = p.n_items < num_sms(dev) ? p.n_items : num_sms(dev);
   const int smem = attn_smem_bytes(p.D);
   cudaError_t e;
+  // The warpgroups re-divide the registers the CTA was launched with; a kernel built with another
+  // per-thread count would make that division wait forever, so it is never launched.
+  {
+    static int regs_ok[kMaxDevices][2] = {};
+    int& ok = regs_ok[dev][p.D == 128 ? 1 : 0];
+    if (ok == 0) {
+      cudaFuncAttributes fa;
+      e = p.D == 128 ? cudaFuncGetAttributes(&fa, attn_fwd_kernel<128>) : cudaFuncGetAttributes(&fa, attn_fwd_kernel<64>);
+      if (e != cudaSuccess) return SP_ERR_CUDA;
+      ok = fa.numRegs == kRegsLaunch ? 1 : -1;
+    }
+    if (ok < 0) return SP_ERR_UNSUPPORTED;
+  }
   if (p.D == 128) {
     static bool attr_set[kMaxDevices] = {};
     if (!attr_set[dev]) {

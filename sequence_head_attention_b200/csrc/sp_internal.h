@@ -53,5 +53,6 @@ sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, i
 sp_status launch_tile_list(const uint8_t* mask, int H, int T, int32_t* row_ptr, int32_t* col_idx,
                            int32_t* counts, cudaStream_t stream);
 sp_status launch_debug_wait(unsigned long long timeout_ns, cudaStream_t stream);
+sp_status launch_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
 
 }  // namespace spattn

@@ -22,7 +22,8 @@ enum : unsigned int {
   ERR_TIMEOUT_O_FREE = 1u << 7,
   ERR_TIMEOUT_DRAIN = 1u << 8,
   ERR_TIMEOUT_DEBUG = 1u << 9,
-  ERR_ANY_TIMEOUT = 0x3ffu,
+  ERR_TIMEOUT_TURN = 1u << 10,
+  ERR_ANY_TIMEOUT = 0x7ffu,
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -55,6 +56,8 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t byt
                : "memory");
 }
 
+// One test of the phase; if it has not completed, the thread may sleep inside the instruction until
+// it completes or about kSuspendNs pass (so waiting warps do not take issue slots from working ones).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -115,6 +118,29 @@ __device__ __forceinline__ bool counter_wait(uint32_t addr, uint32_t target, uin
   }
 }
 
+// One lane of a converged warp (the same lane every time while the whole warp is active).
+__device__ __forceinline__ bool elect_one_sync() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred P1;\n\t"
+      "elect.sync _|P1, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, P1;\n\t}"
+      : "+r"(pred));
+  return pred != 0;
+}
+
+// Warp-wide forms of the waits: every lane polls, and the warp agrees on the outcome.
+__device__ __forceinline__ bool warp_mbar_wait(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                               unsigned int code, volatile int* abort_flag, unsigned int* err) {
+  const bool ok = mbar_wait(bar, parity, timeout_ns, code, abort_flag, err);
+  return __all_sync(0xffffffffu, ok);
+}
+__device__ __forceinline__ bool warp_counter_wait(uint32_t addr, uint32_t target, uint64_t timeout_ns,
+                                                  unsigned int code, volatile int* abort_flag, unsigned int* err) {
+  const bool ok = counter_wait(addr, target, timeout_ns, code, abort_flag, err);
+  return __all_sync(0xffffffffu, ok);
+}
+
 // ------------------------------------------------------------------------------------------------
 // TMA (tiled tensor copies global -> shared, completion counted in bytes on an mbarrier).  Loads only;
 // no multicast form is used anywhere in this library.
@@ -146,6 +172,16 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 
+// Register re-allocation between warpgroups (all warps of a warpgroup execute the same one).
+template <uint32_t N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -153,15 +189,15 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc]
+// D[tmem] (+)= A[smem desc] * B[smem desc].  No "memory" clobber: the MMA reads shared memory
+// asynchronously, and its ordering against the barrier waits and commits (all volatile asm) is kept.
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                        uint32_t accumulate) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // D[tmem] (+)= A[tmem] * B[smem desc]
@@ -171,14 +207,12 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // Arrive once on `bar` when every tcgen05 operation this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-               : "memory");
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar));
 }
 
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
@@ -263,6 +297,66 @@ __device__ __forceinline__ float ex2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// Three-input maximum (one instruction on sm_100a).
+__device__ __forceinline__ float fmax3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// Pairs of fp32 processed by the packed (.f32x2) FMA-pipe instructions of sm_100a.
+struct f2 {
+  float x, y;
+};
+
+__device__ __forceinline__ f2 ffma2(f2 a, f2 b, f2 c) {
+  f2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ f2 fadd2(f2 a, f2 b) {
+  f2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// 2^x for a pair, on the FMA pipe instead of the MUFU unit.  x = n + f with n = round(x) (added to a
+// 1.5 * 2^23 offset, whose low mantissa bits then hold n) and f in [-1/2, 1/2]; 2^f by a cubic whose
+// coefficients are the minimax (Remez) fit with relative weight of 2^f on [-1/2, 1/2] produced by
+// csrc/fit_exp2_poly.py (max relative error 7.5e-5 in this fp32 evaluation); 2^n enters through the
+// exponent field.  x is clamped to >= -125 so the exponent never wraps.
+__device__ __forceinline__ f2 exp2_poly2(f2 x) {
+  const f2 kOff = {12582912.0f, 12582912.0f};   // 1.5 * 2^23
+  const f2 kNegOff = {-12582912.0f, -12582912.0f};
+  const f2 c0 = {9.999280572e-01f, 9.999280572e-01f};
+  const f2 c1 = {6.932609677e-01f, 6.932609677e-01f};
+  const f2 c2 = {2.426111251e-01f, 2.426111251e-01f};
+  const f2 c3 = {5.517166853e-02f, 5.517166853e-02f};
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const f2 j = fadd2(x, kOff);
+  const f2 n = fadd2(j, kNegOff);
+  const f2 f = ffma2(n, f2{-1.0f, -1.0f}, x);  // x - n, exact
+  f2 q = ffma2(c3, f, c2);
+  q = ffma2(q, f, c1);
+  q = ffma2(q, f, c0);
+  f2 r;
+  r.x = __int_as_float(__float_as_int(q.x) + (__float_as_int(j.x) << 23));
+  r.y = __int_as_float(__float_as_int(q.y) + (__float_as_int(j.y) << 23));
+  return r;
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

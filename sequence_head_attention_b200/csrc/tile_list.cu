@@ -91,7 +91,24 @@ __global__ void debug_wait_kernel(unsigned long long timeout_ns, unsigned int* e
   }
 }
 
+// Evaluates the attention kernel's FMA-pipe exponential on n inputs (pairs; n even), for testing it
+// against CUDA's exp2f.
+__global__ void debug_exp2_poly_kernel(const float* x, float* y, int n_pairs) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_pairs) return;
+  const f2 r = exp2_poly2(f2{x[2 * i], x[2 * i + 1]});
+  y[2 * i] = r.x;
+  y[2 * i + 1] = r.y;
+}
+
 }  // namespace
+
+sp_status launch_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream) {
+  const int pairs = n / 2;
+  if (pairs == 0) return SP_OK;
+  debug_exp2_poly_kernel<<<(pairs + 255) / 256, 256, 0, stream>>>(x, y, pairs);
+  return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+}
 
 sp_status launch_tile_list(const uint8_t* mask, int H, int T, int32_t* row_ptr, int32_t* col_idx,
                            int32_t* counts, cudaStream_t stream) {

@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
                 "sp_check_device_error_bits": (I, [P, P]),
                 "sp_set_wait_timeout_ns": (None, [U64]),
                 "sp_debug_wait_timeout": (I, [U64, P]),
+                "sp_debug_exp2_poly": (I, [P, P, I, P]),
                 "sp_version": (ctypes.c_char_p, []),
             }
             for name, (res, args) in sig.items():
@@ -257,6 +258,13 @@ def sp_set_wait_timeout_ns(ns: int) -> None:
 
 def sp_debug_wait_timeout(timeout_ns: int, stream=None) -> None:
     _check("sp_debug_wait_timeout", lib().sp_debug_wait_timeout(int(timeout_ns), _stream(stream)))
+
+
+def sp_debug_exp2_poly(x, y, stream=None):
+    """The kernels' FMA-pipe 2^x on a CUDA fp32 tensor x (even length) into y."""
+    _need(x.dtype == torch.float32 and y.dtype == torch.float32 and x.numel() % 2 == 0, "fp32, even length")
+    _check("sp_debug_exp2_poly", lib().sp_debug_exp2_poly(_ptr(x), _ptr(y), x.numel(), _stream(stream)))
+    return y
 
 
 def declared_symbols():
