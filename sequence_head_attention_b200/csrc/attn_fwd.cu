@@ -27,6 +27,7 @@
 //   O_t += P_t(j) V_j: MMAs from one thread execute in issue order, so S_t(j+1) cannot overwrite P_t(j)
 //   before the P V has read it.
 // Every barrier wait is bounded in time; on expiry the kernel records an error and returns cleanly.
+#include <atomic>
 #include <climits>
 #include <cstdint>
 
@@ -49,6 +50,11 @@ constexpr int kRegsLaunch = 168;
 constexpr uint32_t kRegsControl = 104;
 constexpr uint32_t kRegsSoftmax = 200;
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
+constexpr int kItemRing = 8;     // work-item ids in flight between the producer and the other roles
+constexpr int kSchedSlots = 64;  // launch-rotated work counters, so concurrent launches never share one
+// Per-launch work counters [next item, CTAs finished], kSchedSlots pairs handed out in rotation.  A
+// launch leaves its pair at zero when its last CTA ends.
+__device__ unsigned int g_attn_sched[2 * kSchedSlots];
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and l are rescaled when m grows by > 2^8
 #ifndef SP_EXP2_POLY_PAIRS
 #define SP_EXP2_POLY_PAIRS 0  // of every 8 pairs of exponentials, this many run on the FMA pipe
@@ -67,7 +73,8 @@ struct Cfg {
   // 8-byte slots for the o_done[2] and turn[2] counters
   static constexpr int kNumBars = 2 + 2 * kStages + 11;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + alignment slack
+  // misc: TMEM base, abort flag, published-item count, per-warp item-read counts, the item ring
+  static constexpr int kSmemBytes = kMiscOff + 96 + 1024;  // + alignment slack
   static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
   static constexpr uint32_t kColS = 0;
@@ -98,8 +105,9 @@ struct Item {
 };
 
 __device__ __forceinline__ Item decode_item(const AttnParams& p, int w) {
-  // Items are ordered by head chunk, then batch, then head, then query-tile pair (heaviest first when
-  // causal, so that the round-robin assignment to CTAs interleaves long and short items).
+  // Items are ordered by head chunk, then batch, then head, then query-tile pair, so that the CTAs
+  // running at the same time share one head's K/V in L2.  When causal, a head's pairs run longest
+  // first, so that the last items of a launch, claimed by whichever CTA is free, are the short ones.
   int c = 0;
   while (c + 1 < p.n_chunks && w >= p.chunk_item0[c + 1]) ++c;
   const int r = w - p.chunk_item0[c];
@@ -205,12 +213,35 @@ struct StepIter {
 };
 
 // ------------------------------------------------------------------------------------------------
+// Work distribution: every CTA starts with item blockIdx.x; after that the producer warp claims items
+// from a per-launch counter in global memory (dynamic: a CTA that drew short items takes more), and
+// publishes the claimed ids, in order, into a ring in shared memory that the other roles read.
+// -1 marks the end.  The ring slot of item n is reused for item n + kItemRing only after each of the
+// eight softmax warps has read it: every softmax warp counts its reads in a word of its own (a sum
+// over warps would not do, since on items without keys the warps of a lane do not wait for one another
+// and one may read ahead of another by more than the ring holds).  The MMA warps need no count: the
+// producer loads item n's Q only after both of them are done with item n - 1.
+// ------------------------------------------------------------------------------------------------
+struct ItemRing {
+  uint32_t pub;    // shared address: number of item ids published
+  uint32_t used0;  // shared address: items read by softmax warp 0; warp k at +4k
+  volatile int* ids;
+};
+
+__device__ __forceinline__ bool ring_read(const ItemRing& r, int n, int& w, uint64_t tmo, volatile int* abort_flag,
+                                          unsigned int* err) {
+  if (!warp_counter_wait(r.pub, (uint32_t)(n + 1), tmo, ERR_TIMEOUT_ITEM, abort_flag, err)) return false;
+  w = r.ids[n % kItemRing];
+  return true;
+}
+
+// ------------------------------------------------------------------------------------------------
 // Producer: one warp walks the work in lockstep (all values warp-uniform); one elected lane issues the
 // TMA loads.
 // ------------------------------------------------------------------------------------------------
 template <int D>
 __device__ void run_producer(const AttnParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
-                             const CUtensorMap* tv, uint8_t* smem, const Bars& bars,
+                             const CUtensorMap* tv, uint8_t* smem, const Bars& bars, const ItemRing& ir,
                              volatile int* abort_flag) {
   using C = Cfg<D>;
   const uint32_t sbase = smem_u32(smem);
@@ -220,7 +251,28 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tq, const C
   int n_item = 0;
   int last_q_item = -1;
   bool ok = true;
-  for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++n_item) {
+  int w = blockIdx.x;
+  for (;; ++n_item) {
+    if (n_item > 0) {  // claim the next item
+      int claimed = 0;
+      if (elect_one_sync()) claimed = (int)gridDim.x + (int)atomicAdd(p.sched, 1u);
+      w = __shfl_sync(0xffffffffu, claimed, __ffs(__ballot_sync(0xffffffffu, claimed != 0)) - 1);
+    }
+    const bool done = w >= p.n_items;
+    // publish it (the slot's previous item must have been read by every softmax warp)
+    if (n_item >= kItemRing) {
+      const uint32_t need = (uint32_t)(n_item - kItemRing + 1);
+#pragma unroll 1
+      for (int k = 0; k < 8 && ok; ++k)
+        ok = warp_counter_wait(ir.used0 + 4u * k, need, tmo, ERR_TIMEOUT_ITEM_FREE, abort_flag, p.err);
+      if (!ok) break;
+    }
+    if (elect_one_sync()) {
+      ir.ids[n_item % kItemRing] = done ? -1 : w;
+      smem_counter_add_release(ir.pub, 1u);
+    }
+    __syncwarp();
+    if (done) break;
     const Item it = decode_item(p, w);
     if (n_item > 0) {
       ok = warp_mbar_wait(bars.q_empty, q_empty_ph, tmo, ERR_TIMEOUT_Q_EMPTY, abort_flag, p.err);
@@ -281,8 +333,8 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tq, const C
 // done with them (the "empty" barriers count two arrivals; a lane that skips a tile arrives directly).
 // ------------------------------------------------------------------------------------------------
 template <int D>
-__device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, uint32_t tmem_in, int t,
-                        volatile int* abort_flag) {
+__device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, const ItemRing& ir, uint32_t tmem_in,
+                        int t, volatile int* abort_flag) {
   using C = Cfg<D>;
   const uint32_t sbase = smem_u32(smem);
   const uint64_t tmo = p.timeout_ns;
@@ -298,7 +350,10 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, ui
   int ring = 0;
   int n_item = 0;
   bool ok = true;
-  for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x, ++n_item) {
+  for (;; ++n_item) {
+    int w;
+    ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err);
+    if (!ok || w < 0) break;
     const Item it = decode_item(p, w);
     ok = warp_mbar_wait(bars.q_full, q_full_ph, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
     q_full_ph ^= 1;
@@ -411,7 +466,7 @@ __device__ __forceinline__ void pass_turn(const Bars& bars, int lane_t) {
 // Softmax + epilogue: 4 warps per lane, one query row per thread.
 // ------------------------------------------------------------------------------------------------
 template <int D>
-__device__ void run_softmax(const AttnParams& p, const Bars& bars, uint32_t tmem, int lane_t,
+__device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRing& ir, uint32_t tmem, int lane_t,
                             volatile int* abort_flag) {
   using C = Cfg<D>;
   const int warp = threadIdx.x >> 5;
@@ -427,7 +482,12 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, uint32_t tmem
   uint32_t union_step = 0;  // union steps walked so far, over all items (identical in both lanes)
   bool ok = true;
 
-  for (int w = blockIdx.x; w < p.n_items && ok; w += gridDim.x) {
+  for (int n_item = 0;; ++n_item) {
+    int w;
+    ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err);
+    if (!ok || w < 0) break;
+    __syncwarp();
+    if (lane == 0) smem_counter_add_release(ir.used0 + 4u * warp, 1u);  // this warp is done with the slot
     const Item it = decode_item(p, w);
     StepIter st;
     st.init(p, it);
@@ -620,6 +680,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   bars.drain = bars.turn0 + 16;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  ItemRing ir;
+  ir.pub = smem_u32(smem + C::kMiscOff + 8);
+  ir.used0 = smem_u32(smem + C::kMiscOff + 16);
+  ir.ids = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 48);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
@@ -639,6 +703,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<volatile uint32_t*>(smem + C::kBarOff + (bars.o_done0 - bar0) + 8 * k) = 0u;
     mbar_init(bars.drain, 2);
     *abort_flag = 0;
+    *reinterpret_cast<volatile uint32_t*>(smem + C::kMiscOff + 8) = 0u;  // items published
+    for (int k = 0; k < 8; ++k)                                          // items read, per softmax warp
+      *reinterpret_cast<volatile uint32_t*>(smem + C::kMiscOff + 16 + 4 * k) = 0u;
     fence_mbar_init();
   }
   if (warp == kWarpProducer && lane == 0) {
@@ -657,13 +724,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     regs_inc<kRegsSoftmax>();
-    run_softmax<D>(p, bars, tmem, warp >> 2, abort_flag);
+    run_softmax<D>(p, bars, ir, tmem, warp >> 2, abort_flag);
   } else {
     regs_dec<kRegsControl>();
     if (warp == kWarpProducer) {
-      run_producer<D>(p, &tq, &tk, &tv, smem, bars, abort_flag);
+      run_producer<D>(p, &tq, &tk, &tv, smem, bars, ir, abort_flag);
     } else if (warp == kWarpMma || warp == kWarpMma + 1) {
-      run_mma<D>(p, smem, bars, tmem, warp - kWarpMma, abort_flag);
+      run_mma<D>(p, smem, bars, ir, tmem, warp - kWarpMma, abort_flag);
     }
     __syncwarp();
   }
@@ -672,6 +739,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
+  }
+  // The last CTA to finish returns this launch's work counter to zero for the next launch that draws
+  // the same slot (every CTA has made its last claim before it gets here).
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(p.sched, 0u);
+      atomicExch(p.sched + 1, 0u);
+    }
   }
 }
 
@@ -692,6 +768,16 @@ sp_status launch_attn(const AttnParams& p_in, const void* q, const void* k, cons
   if (p.n_items <= 0) return SP_OK;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SP_ERR_CUDA;
+  {
+    static unsigned int* sched_base[kMaxDevices] = {};
+    static std::atomic<unsigned int> launch_seq{0};
+    if (!sched_base[dev]) {
+      void* ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_attn_sched) != cudaSuccess || !ptr) return SP_ERR_CUDA;
+      sched_base[dev] = static_cast<unsigned int*>(ptr);
+    }
+    p.sched = sched_base[dev] + 2 * (launch_seq.fetch_add(1) % kSchedSlots);
+  }
   const int grid = p.n_items < num_sms(dev) ? p.n_items : num_sms(dev);
   const int smem = attn_smem_bytes(p.D);
   cudaError_t e;

@@ -6,8 +6,9 @@
 // framework owning every allocation and exposing no allocator, or a hard-real-time loop that forbids
 // allocation after start-up.  Such a caller can provide inputs and outputs but no workspace.
 //
-// The only scratch the block-sparse path needs is the compacted tile list of the mask (row offsets,
-// per-row counts and kept key-tile indices).  Here it lives in g_noalloc_scratch below: a file-scope
+// Besides the attention kernel's work counters (a small static array of its own, shared by every
+// launch), the only scratch the block-sparse path needs is the compacted tile list of the mask (row
+// offsets, per-row counts and kept key-tile indices).  Here it lives in g_noalloc_scratch below: a file-scope
 // device array that every GPU which loads this library holds until the process exits.  The array is
 // shared by every call on a device, so calls whose execution overlaps on the GPU (different streams, or
 // threads without ordering between them) race on it and must be serialised by the caller.  Nothing in

@@ -33,7 +33,8 @@ struct AttnParams {
   int chunk_h0[kMaxChunks + 1];     // first head of each chunk, chunk_h0[n_chunks] = H
   int chunk_item0[kMaxChunks + 1];  // first work item of each chunk
   unsigned long long timeout_ns;
-  unsigned int* err;  // device error word of this device
+  unsigned int* err;    // device error word of this device
+  unsigned int* sched;  // this launch's work counter pair [next item, CTAs finished] (set by launch_attn)
 };
 
 // Device properties and driver entry points (cached per device).

@@ -202,3 +202,26 @@ def test_many_items_per_cta_with_empty_lanes(causal, kv, mask_heads_empty):
     assert st == spattn.SP_OK, hex(bits)
     r = torch.tensor(rows, device="cuda")
     assert_close(o[:, r], ref[0], lse[:, :, r], ref[1])
+
+
+def test_concurrent_launches_on_two_streams():
+    """Two launches in flight at once on different streams draw different work counters; each result
+    equals the same launch run alone, and repeated launches (counters reused after their reset) agree."""
+    B, S, H, D = 1, 4096, 8, 128
+    qa, ka, va = (t.cuda() for t in synth.qkv(B, S, H, D, seed=31, scale=0.5))
+    qb, kb, vb = (t.cuda() for t in synth.qkv(B, S, H, D, seed=32, scale=0.5))
+    ref_a, ref_b = gpu_attn(qa, ka, va, causal=True), gpu_attn(qb, kb, vb)
+    s1, s2 = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+    outs = []
+    for _ in range(70):  # more launches than there are counter slots
+        oa = torch.empty_like(ref_a[0]); la = torch.empty_like(ref_a[1])
+        ob = torch.empty_like(ref_b[0]); lb = torch.empty_like(ref_b[1])
+        spattn.sp_attn_fwd(qa, ka, va, oa, la, causal=True, stream=s1)
+        spattn.sp_attn_fwd(qb, kb, vb, ob, lb, stream=s2)
+        outs.append((oa, la, ob, lb))
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    for oa, la, ob, lb in outs:
+        assert torch.equal(oa, ref_a[0]) and torch.equal(la, ref_a[1])
+        assert torch.equal(ob, ref_b[0]) and torch.equal(lb, ref_b[1])
