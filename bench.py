@@ -273,8 +273,9 @@ def run_ours(args):
     spattn.lib()  # fail now if the library is missing
 
     w, q, k, v, mask = build_inputs(args.workload, seed=rank, seq_len=args.seq_len, ranks=args.ranks)
+    fused = args.workload == "video_dit" and args.ulysses == "fused"
     if args.workload == "video_dit":
-        step = workloads.UlyssesStep(w, q, k, v, device=dev)
+        step = workloads.UlyssesStep(w, q, k, v, device=dev, fused=fused)
     elif args.workload == "ring_causal":
         step = workloads.RingStep(w, q, k, v, device=dev)
     else:
@@ -284,7 +285,11 @@ def run_ours(args):
 
     def timed_step(marks):
         """One step with events around the phases: returns nothing; marks collects (name, ev0, ev1)."""
-        if args.workload == "video_dit":
+        if fused:
+            for r in range(step.P):
+                a = E(); a.record(stream); step.attention_rank_fused(r); b = E(); b.record(stream)
+                marks.append(("attn", a, b))
+        elif args.workload == "video_dit":
             a = E(); a.record(stream); step.relayout_in(); b = E(); b.record(stream)
             marks.append(("relayout", a, b))
             for r in range(step.P):
@@ -340,10 +345,21 @@ def run_ours(args):
     if args.workload == "video_dit":
         attn_ms = statistics.mean(phase["attn"])
         flops_launch = step.flops / step.P
-        rl_ms = sum(phase["relayout"]) / args.steps  # both relayout phases of one step
+        if fused:
+            # The fused step has no relayout pass; the relayout kernels (the unfused path's copies) are
+            # timed here on their own, after the timed region, for their HBM figures.
+            rl = []
+            for _ in range(args.steps):
+                a = E(); a.record(stream); step.relayout_in(); step.relayout_out(); b = E(); b.record(stream)
+                rl.append((a, b))
+            torch.cuda.synchronize(dev)
+            rl_ms = statistics.mean(x.elapsed_time(y) for x, y in rl)
+        else:
+            rl_ms = sum(phase["relayout"]) / args.steps  # both relayout phases of one step
         rl_gbs = step.relayout_bytes / (rl_ms / 1000.0) / 1e9
         kernels["relayout"] = {"gbs": rl_gbs, "ms_per_step": rl_ms, "bytes_per_step": step.relayout_bytes,
-                               "frac_of_measured_hbm": rl_gbs / peaks["hbm_gbs"]}
+                               "frac_of_measured_hbm": rl_gbs / peaks["hbm_gbs"],
+                               "in_timed_step": not fused}
     elif args.workload == "ring_causal":
         attn_ms = statistics.mean(phase["attn_all"])
         flops_launch = step.flops
@@ -395,6 +411,9 @@ def run_ours(args):
         cpu = calibrated_oracle_baseline(args.workload, q, k, v, mask, target_s=args.cpu_seconds)
 
     extra = {}
+    if args.workload == "video_dit":
+        extra = {"ulysses": "attention on the sequence shards, relayouts folded into the kernel" if fused
+                 else "seq->head relayout, per-rank attention, head->seq relayout"}
     if args.workload == "block_sparse":
         extra = {"mask_density": step.density, "kept_tiles": step.kept_tiles}
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -417,6 +436,9 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=["video_dit", "ring_causal", "block_sparse", "tiny_dense", "megatron"],
                     default="video_dit", help="tiny_dense / megatron: reference arm only (parity-size cases)")
+    ap.add_argument("--ulysses", choices=["fused", "relayout"], default="fused",
+                    help="video_dit step: attention straight on the sequence shards (fused), or the seq->head "
+                         "relayout, per-rank attention and head->seq relayout")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

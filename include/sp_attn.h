@@ -68,6 +68,8 @@ typedef void* sp_stream;
 /* Largest number of partials sp_merge_partials combines in one call, and of relayout ranks. */
 #define SP_MAX_PARTS 64
 #define SP_MAX_RANKS 64
+/* Largest number of sequence shards sp_attn_fwd_seq_sharded reads and writes directly. */
+#define SP_MAX_SHARDS 8
 
 /*
  * Bytes of device workspace sp_attn_fwd / sp_attn_fwd_partial need for these sizes.
@@ -148,6 +150,33 @@ SP_API sp_status sp_seq_to_head_relayout(const void* const* in_ranks, void* cons
 /* The exact inverse: in_ranks[r] [B, S, H/P, D] -> out_ranks[r] [B, S/P, H, D].  Same requirements. */
 SP_API sp_status sp_head_to_seq_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B,
                                   int S, int H, int D, int elem_bytes, sp_stream stream);
+
+/*
+ * One Ulysses rank's attention straight on the sequence shards, with both relayouts folded into the
+ * kernel ("HCMS: ... Ulysses ... all-to-all", abstract: each rank attends over the whole sequence for its
+ * share of the heads; "LLM Lab Notes 05", section 2: per head q @ k^T / sqrt(d), softmax, @ v).  It
+ * computes what sp_seq_to_head_relayout of Q, K and V, sp_attn_fwd of the rank's heads [h0, h0 + n_heads)
+ * with these head chunks, then sp_head_to_seq_relayout of O compute, but no head-sharded copy is ever
+ * written: query and key tiles lie on each shard's own 128-row grid (a shard's last tile may be short),
+ * each is loaded from its shard, and each O row is written into the shard that owns it.  When S/P is a
+ * multiple of 128 the grids coincide and the result is bit for bit that of the three calls; otherwise
+ * the keys are grouped into different tiles, so the result differs from theirs by rounding only.
+ *
+ * q_shards, k_shards, v_shards  host arrays of P device pointers, bf16 [B, S/P, H, D]: shard r holds
+ *                               positions [r*S/P, (r+1)*S/P) of every head.
+ * o_shards  host array of P device pointers, bf16 [B, S/P, H, D]; heads [h0, h0 + n_heads) of every
+ *           row are written, the other heads are left untouched (so P calls with disjoint head ranges
+ *           fill them all).  No overlap with any input.
+ * lse       device fp32 [B, H, S] (every head of the whole sequence; rows of heads [h0, h0 + n_heads)
+ *           written), or NULL.
+ * head_chunks  host int[n_head_chunks], each > 0, summing to n_heads (NULL: one chunk).
+ * Requires 1 <= P <= SP_MAX_SHARDS, S % P == 0, 0 <= h0, h0 + n_heads <= H, D in {64, 128}, 16-byte
+ * aligned pointers.  No block mask.  Errors as sp_attn_fwd.
+ */
+SP_API sp_status sp_attn_fwd_seq_sharded(const void* const* q_shards, const void* const* k_shards,
+                                         const void* const* v_shards, void* const* o_shards, float* lse, int P,
+                                         int B, int S, int H, int D, int h0, int n_heads, const int* head_chunks,
+                                         int n_head_chunks, int causal, sp_stream stream);
 
 /*
  * Block-sparse attention that allocates nothing, for callers that cannot call cudaMalloc (a serving

@@ -65,6 +65,8 @@ bool sizes_ok(int B, int S, int H, int D) {
 
 cudaStream_t as_stream(sp_stream s) { return reinterpret_cast<cudaStream_t>(s); }
 
+sp_status count_items(AttnParams& p);
+
 sp_status fill_attn_params(AttnParams& p, int B, int S, int H, int D, int kv_begin, int kv_end,
                            int causal, const int* chunk_h0, int n_chunks) {
   p = AttnParams{};
@@ -84,14 +86,18 @@ sp_status fill_attn_params(AttnParams& p, int B, int S, int H, int D, int kv_beg
   p.err = device_error_word();
   if (!p.err) return SP_ERR_CUDA;
   p.n_chunks = n_chunks;
+  for (int c = 0; c <= n_chunks; ++c) p.chunk_h0[c] = chunk_h0[c];
+  return count_items(p);
+}
+
+// Work items per head chunk (B * heads * n_qpairs each) and in all.
+sp_status count_items(AttnParams& p) {
   long long items = 0;
-  for (int c = 0; c < n_chunks; ++c) {
-    p.chunk_h0[c] = chunk_h0[c];
+  for (int c = 0; c < p.n_chunks; ++c) {
     p.chunk_item0[c] = (int)items;
-    items += (long long)B * (chunk_h0[c + 1] - chunk_h0[c]) * p.n_qpairs;
+    items += (long long)p.B * (p.chunk_h0[c + 1] - p.chunk_h0[c]) * p.n_qpairs;
   }
-  p.chunk_h0[n_chunks] = chunk_h0[n_chunks];
-  p.chunk_item0[n_chunks] = (int)items;
+  p.chunk_item0[p.n_chunks] = (int)items;
   if (items > 0x7fffffffLL) return SP_ERR_INVALID_ARG;
   p.n_items = (int)items;
   return SP_OK;
@@ -356,6 +362,72 @@ static sp_status relayout_common(const void* const* in_ranks, void* const* out_r
       if (a0 < b1 && b0 < a1) return SP_ERR_INVALID_ARG;
     }
   return launch_relayout(in_ranks, out_ranks, P, B, S, H, D, elem_bytes, seq_to_head, as_stream(stream));
+}
+
+sp_status sp_attn_fwd_seq_sharded(const void* const* q_shards, const void* const* k_shards,
+                                  const void* const* v_shards, void* const* o_shards, float* lse, int P, int B,
+                                  int S, int H, int D, int h0, int n_heads, const int* head_chunks,
+                                  int n_head_chunks, int causal, sp_stream stream) {
+  if (!sizes_ok(B, S, H, D)) return SP_ERR_INVALID_ARG;
+  if (!q_shards || !k_shards || !v_shards || !o_shards || P < 1 || P > SP_MAX_SHARDS || S % P != 0)
+    return SP_ERR_INVALID_ARG;
+  if (h0 < 0 || n_heads < 1 || (long long)h0 + n_heads > H) return SP_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SP_ERR_INVALID_ARG;
+  if (lse && !aligned16(lse)) return SP_ERR_INVALID_ARG;
+  for (int r = 0; r < P; ++r) {
+    if (!q_shards[r] || !k_shards[r] || !v_shards[r] || !o_shards[r]) return SP_ERR_INVALID_ARG;
+    if (!aligned16(q_shards[r]) || !aligned16(k_shards[r]) || !aligned16(v_shards[r]) || !aligned16(o_shards[r]))
+      return SP_ERR_INVALID_ARG;
+  }
+  // no output shard may overlap an input shard
+  const size_t shard_bytes = (size_t)B * (S / P) * H * D * 2;
+  for (int r = 0; r < P; ++r)
+    for (int i = 0; i < P; ++i)
+      for (const void* in : {q_shards[i], k_shards[i], v_shards[i]}) {
+        const uintptr_t a0 = reinterpret_cast<uintptr_t>(o_shards[r]), b0 = reinterpret_cast<uintptr_t>(in);
+        if (a0 < b0 + shard_bytes && b0 < a0 + shard_bytes) return SP_ERR_INVALID_ARG;
+      }
+  // head chunks of [h0, h0 + n_heads): contiguous, in order, each > 0, summing to n_heads
+  int c0[kMaxChunks + 1];
+  int n_chunks = 1;
+  c0[0] = h0;
+  c0[1] = h0 + n_heads;
+  if (head_chunks) {
+    if (n_head_chunks < 1 || n_head_chunks > kMaxChunks) return SP_ERR_INVALID_ARG;
+    long long acc = 0;
+    for (int c = 0; c < n_head_chunks; ++c) {
+      if (head_chunks[c] < 1) return SP_ERR_INVALID_ARG;
+      c0[c] = h0 + (int)acc;
+      acc += head_chunks[c];
+      if (acc > n_heads) return SP_ERR_INVALID_ARG;
+    }
+    if (acc != n_heads) return SP_ERR_INVALID_ARG;
+    c0[n_head_chunks] = h0 + n_heads;
+    n_chunks = n_head_chunks;
+  } else if (n_head_chunks != 0 && n_head_chunks != 1) {
+    return SP_ERR_INVALID_ARG;
+  }
+  AttnParams p;
+  sp_status s = fill_attn_params(p, B, S, H, D, 0, S, causal, c0, n_chunks);
+  if (s != SP_OK) return s;
+  p.o = o_shards[0];
+  p.o_f32 = 0;
+  p.lse = lse;
+  p.n_shards = P;
+  p.shard_rows = S / P;
+  p.tiles_per_shard = (p.shard_rows + SP_TILE - 1) / SP_TILE;
+  p.pairs_per_shard = (p.tiles_per_shard + 1) / 2;
+  p.n_qpairs = P * p.pairs_per_shard;
+  p.n_kv_tiles = P * p.tiles_per_shard;
+  s = count_items(p);
+  if (s != SP_OK) return s;
+  for (int r = 0; r < P; ++r) {
+    p.q_shard[r] = q_shards[r];
+    p.k_shard[r] = k_shards[r];
+    p.v_shard[r] = v_shards[r];
+    p.o_shard[r] = o_shards[r];
+  }
+  return launch_attn_sharded(p, as_stream(stream));
 }
 
 sp_status sp_seq_to_head_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,

@@ -18,9 +18,9 @@
 //               of S from TMEM (so every row reduction stays inside one thread), keeps the running
 //               maximum m and sum l, writes P = exp(S - m) as bf16 back into TMEM over S, rescales
 //               the O row in TMEM when the maximum grows by more than 2^8, and finally writes
-//               O / l and lse = (m + log2 l) ln 2.  The two lanes take turns at the exponentials
-//               (ping-pong), so each has the MUFU unit to itself while the tensor core runs the
-//               other lane's MMAs.
+//               O / l and lse = (m + log2 l) ln 2.  The two lanes run independently: while one
+//               lane's warps compute exponentials, the tensor core runs the other lane's MMAs, and
+//               when both are in their softmax phase the two warps per SMSP hide each other's latency.
 //   warp 11     idle (it completes the third warpgroup, which gives its registers to the softmax).
 //   TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256, 256+D), O_1 [256+D, 256+2D); P_t
 //   overwrites the first 64 columns of S_t.  Each lane's issuer queues S_t(j+1) right behind
@@ -70,8 +70,8 @@ struct Cfg {
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
   // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2], drain, and
-  // 8-byte slots for the o_done[2] and turn[2] counters
-  static constexpr int kNumBars = 2 + 2 * kStages + 11;
+  // 8-byte slots for the o_done[2] counters
+  static constexpr int kNumBars = 2 + 2 * kStages + 9;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // misc: TMEM base, abort flag, published-item count, per-warp item-read counts, the item ring
   static constexpr int kSmemBytes = kMiscOff + 96 + 1024;  // + alignment slack
@@ -82,7 +82,7 @@ struct Cfg {
 };
 
 struct Bars {
-  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, pv_done0, o_done0, turn0, drain;
+  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, pv_done0, o_done0, drain;
   __device__ uint32_t kv_full(int s) const { return kv_full0 + 8u * s; }
   __device__ uint32_t kv_empty(int s) const { return kv_empty0 + 8u * s; }
   __device__ uint32_t s_full(int t) const { return s_full0 + 8u * t; }
@@ -90,17 +90,14 @@ struct Bars {
   __device__ uint32_t pv_done(int t) const { return pv_done0 + 8u * t; }
   // o_done[t]: a counter, +1 per softmax warp of lane t per finished item (epilogue reads of O done)
   __device__ uint32_t o_done(int t) const { return o_done0 + 8u * t; }
-  // turn[t]: a counter, +1 per softmax warp of lane t per union step it has finished (or skipped).  The
-  // two lanes take turns at their exponentials (ping-pong), so each has the MUFU unit to itself while
-  // the tensor core runs the other lane's MMAs; a monotonic count cannot alias however far a lane that
-  // skips steps runs ahead.
-  __device__ uint32_t turn(int t) const { return turn0 + 8u * t; }
 };
 
 struct Item {
   int b, h, qp;
-  int q_start[2];
-  int q_last[2];
+  int shard;       // sequence shard holding both query tiles (0 when not sharded)
+  int q_start[2];  // first row of each lane's query tile (global position)
+  int q_last[2];   // last row of each lane's tile that exists (global position)
+  int q_end;       // one past the last row of the shard (rows from here on belong to the next shard)
   bool valid[2];
 };
 
@@ -119,19 +116,30 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p, int w) {
   it.h = p.chunk_h0[c] + r2 / p.n_qpairs;
   const int qq = r2 % p.n_qpairs;
   it.qp = p.causal ? (p.n_qpairs - 1 - qq) : qq;
+  // Query tiles are laid on each shard's own 128-row grid (one shard: the global grid); a shard's last
+  // tile may be short, and pairs never cross shards.
+  it.shard = it.qp / p.pairs_per_shard;
+  const int lp = it.qp - it.shard * p.pairs_per_shard;
+  it.q_end = min(p.S, (it.shard + 1) * p.shard_rows);
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    it.q_start[t] = (2 * it.qp + t) * kTile;
-    it.valid[t] = it.q_start[t] < p.S;
-    it.q_last[t] = min(p.S, it.q_start[t] + kTile) - 1;
+    const int lt = 2 * lp + t;
+    it.q_start[t] = it.shard * p.shard_rows + lt * kTile;
+    it.valid[t] = lt < p.tiles_per_shard && it.q_start[t] < it.q_end;
+    it.q_last[t] = min(it.q_end, it.q_start[t] + kTile) - 1;
   }
   return it;
 }
 
-// Walks the key tiles a work item needs, in increasing key order, with which lanes need each.
+// Walks the key tiles a work item needs, in increasing key order, with which lanes need each.  Dense
+// key tiles lie on each shard's own grid as the query tiles do (a shard's last tile may be short).
 struct StepIter {
-  bool sparse, causal;
+  bool sparse, causal, sharded;
   int kv_begin;
+  int shard_rows, tiles_per_shard;
+  int r, lt;       // shard and tile within it of the next dense tile (sharded)
+  int shard;       // shard of the tile next() returned last (0 when not sharded)
+  int key_end;     // one past that shard's last row (INT_MAX when not sharded)
   int q_last0, q_last1;
   bool v0, v1;
   int j, n_dense;
@@ -155,14 +163,25 @@ struct StepIter {
     v0 = it.valid[0];
     v1 = it.valid[1];
     sparse = p.row_ptr != nullptr;
+    sharded = p.n_shards > 1;
+    shard_rows = p.shard_rows;
+    tiles_per_shard = p.tiles_per_shard;
     j = 0;
+    r = lt = 0;
+    shard = 0;
+    key_end = INT_MAX;
     if (!sparse) {
       n_dense = 0;
       if (v0 || v1) {
         n_dense = p.n_kv_tiles;
         if (causal) {
           const int ql = v1 ? q_last1 : q_last0;
-          n_dense = ql < p.kv_begin ? 0 : min(p.n_kv_tiles, (ql - p.kv_begin) / kTile + 1);
+          if (sharded) {  // the tile of key ql on its shard's grid (kv_begin is 0 here)
+            const int r = ql / shard_rows;
+            n_dense = min(p.n_kv_tiles, r * tiles_per_shard + (ql - r * shard_rows) / kTile + 1);
+          } else {
+            n_dense = ql < p.kv_begin ? 0 : min(p.n_kv_tiles, (ql - p.kv_begin) / kTile + 1);
+          }
         }
       }
       return;
@@ -195,7 +214,17 @@ struct StepIter {
   __device__ __forceinline__ bool next(int& kv_start, bool& k0, bool& k1) {
     if (!sparse) {
       if (j >= n_dense) return false;
-      kv_start = kv_begin + j * kTile;
+      if (sharded) {  // walk the shards' grids without dividing
+        kv_start = r * shard_rows + lt * kTile;
+        shard = r;
+        key_end = (r + 1) * shard_rows;
+        if (++lt == tiles_per_shard) {
+          lt = 0;
+          ++r;
+        }
+      } else {
+        kv_start = kv_begin + j * kTile;
+      }
       ++j;
       k0 = v0 && (!causal || kv_start <= q_last0);
       k1 = v1 && (!causal || kv_start <= q_last1);
@@ -236,13 +265,23 @@ __device__ __forceinline__ bool ring_read(const ItemRing& r, int n, int& w, uint
 }
 
 // ------------------------------------------------------------------------------------------------
+// Sequence shards: the tensor maps of every shard of Q, K and V (one shard when the tensors are not
+// split).  Every tile lies on one shard's grid, so it is one TMA box of that shard; the rows of a short
+// last tile past the shard's end read as zero and are masked (keys) or not written (queries).
+// ------------------------------------------------------------------------------------------------
+struct TMaps {
+  CUtensorMap q[kMaxShards];
+  CUtensorMap k[kMaxShards];
+  CUtensorMap v[kMaxShards];
+};
+
+// ------------------------------------------------------------------------------------------------
 // Producer: one warp walks the work in lockstep (all values warp-uniform); one elected lane issues the
 // TMA loads.
 // ------------------------------------------------------------------------------------------------
 template <int D>
-__device__ void run_producer(const AttnParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
-                             const CUtensorMap* tv, uint8_t* smem, const Bars& bars, const ItemRing& ir,
-                             volatile int* abort_flag) {
+__device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem, const Bars& bars,
+                             const ItemRing& ir, volatile int* abort_flag) {
   using C = Cfg<D>;
   const uint32_t sbase = smem_u32(smem);
   const uint64_t tmo = p.timeout_ns;
@@ -280,13 +319,14 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tq, const C
       if (!ok) break;
     }
     if (elect_one_sync()) {
+      const int y0 = it.shard * p.shard_rows;  // the pair's shard starts at this global row
       mbar_arrive_expect_tx(bars.q_full, 2 * C::kTileBytes);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
         for (int c = 0; c < C::kSub; ++c)
-          tma_load_4d(sbase + C::kQOff + t * C::kTileBytes + c * 16384, tq, bars.q_full, 64 * c, it.h,
-                      it.q_start[t], it.b);
+          tma_load_4d(sbase + C::kQOff + t * C::kTileBytes + c * 16384, &tm.q[it.shard], bars.q_full, 64 * c, it.h,
+                      it.q_start[t] - y0, it.b);
     }
     __syncwarp();
     last_q_item = n_item;
@@ -305,11 +345,11 @@ __device__ void run_producer(const AttnParams& p, const CUtensorMap* tq, const C
         }
         if (elect_one_sync()) {
           mbar_arrive_expect_tx(bars.kv_full(slot), C::kTileBytes);
-          const CUtensorMap* tm = kv == 0 ? tk : tv;
+          const CUtensorMap* map = kv == 0 ? &tm.k[st.shard] : &tm.v[st.shard];
 #pragma unroll
           for (int c = 0; c < C::kSub; ++c)
-            tma_load_4d(sbase + C::kKVOff + slot * C::kTileBytes + c * 16384, tm, bars.kv_full(slot), 64 * c,
-                        it.h, kv_start, it.b);
+            tma_load_4d(sbase + C::kKVOff + slot * C::kTileBytes + c * 16384, map, bars.kv_full(slot), 64 * c,
+                        it.h, kv_start - st.shard * p.shard_rows, it.b);
         }
         __syncwarp();
         ++ring;
@@ -452,16 +492,6 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
   warp_mbar_wait(bars.drain, 0, tmo, ERR_TIMEOUT_DRAIN, nullptr, p.err);
 }
 
-// Ping-pong between the two softmax lanes: lane 0 starts the exponentials of union step u once lane 1 is
-// done with step u - 1 (turn[1] >= 4u), lane 1 once lane 0 is done with step u (turn[0] >= 4(u + 1)).
-__device__ __forceinline__ bool take_turn(const Bars& bars, int lane_t, uint32_t u, uint64_t tmo,
-                                          volatile int* abort_flag, unsigned int* err) {
-  return warp_counter_wait(bars.turn(lane_t ^ 1), 4u * (lane_t ? u + 1u : u), tmo, ERR_TIMEOUT_TURN, abort_flag, err);
-}
-__device__ __forceinline__ void pass_turn(const Bars& bars, int lane_t) {
-  smem_counter_add_release(bars.turn(lane_t), 1u);
-}
-
 // ------------------------------------------------------------------------------------------------
 // Softmax + epilogue: 4 warps per lane, one query row per thread.
 // ------------------------------------------------------------------------------------------------
@@ -479,7 +509,6 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
   const float scale_log2 = p.scale_log2;
   uint32_t s_full_ph = 0;
   uint32_t total_pv = 0;
-  uint32_t union_step = 0;  // union steps walked so far, over all items (identical in both lanes)
   bool ok = true;
 
   for (int n_item = 0;; ++n_item) {
@@ -500,12 +529,7 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
     int kv_start;
     bool k0, k1;
     while (st.next(kv_start, k0, k1)) {
-      const uint32_t u = union_step++;
-      if (!(lane_t == 0 ? k0 : k1)) {  // this lane skips the step: its turn is over at once
-        __syncwarp();
-        if (lane == 0) pass_turn(bars, lane_t);
-        continue;
-      }
+      if (!(lane_t == 0 ? k0 : k1)) continue;  // this lane skips the step
       ok = mbar_wait(bars.s_full(lane_t), s_full_ph, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err);
       ok = __all_sync(0xffffffffu, ok);
       s_full_ph ^= 1;
@@ -516,8 +540,9 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
       for (int c = 0; c < 4; ++c) tmem_ld32(tS + c * 32, sr[c]);
       tmem_wait_ld();
 #define SV(i) __uint_as_float(sr[(i) >> 5][(i) & 31])
-      // Keys past the KV range, past S, or (causal) after this query: -inf.
-      const int n_valid = lim_row - kv_start;
+      // Keys past the KV range, past S, past the end of the tile's shard, or (causal) after this query:
+      // -inf.
+      const int n_valid = min(lim_row, st.key_end) - kv_start;
       if (__any_sync(0xffffffffu, n_valid < kTile)) {
 #pragma unroll
         for (int c = 0; c < 4; ++c)
@@ -535,10 +560,6 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
         for (int k = 0; k < 8; ++k) mx8[k] = fmax3f(mx8[k], SV(i + 2 * k), SV(i + 2 * k + 1));
       const float mx = fmax3f(fmax3f(mx8[0], mx8[1], mx8[2]), fmax3f(mx8[3], mx8[4], mx8[5]),
                               fmaxf(mx8[6], mx8[7]));
-      // Ping-pong: lane 0 starts step u's exponentials once lane 1 is done with step u - 1, lane 1 once
-      // lane 0 is done with step u.
-      ok = take_turn(bars, lane_t, u, tmo, abort_flag, p.err);
-      if (!ok) break;
       const float m_tile = mx * scale_log2;
       const bool grow = m_tile > m_used + kRescaleThreshold;
       float alpha = 1.f;
@@ -596,18 +617,22 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bars.p_full(lane_t));
-        pass_turn(bars, lane_t);
-      }
+      if (lane == 0) mbar_arrive(bars.p_full(lane_t));
       ++n_kept;
       ++total_pv;
     }
     if (!ok) break;
     // Epilogue: O / l and lse for the rows of this lane.
     if (lane_valid) {
-      const bool row_ok = q_row < p.S;
-      const size_t o_idx = (((size_t)it.b * p.S + q_row) * p.H + it.h) * D;
+      const bool row_ok = q_row < it.q_end;  // inside S and inside the pair's shard
+      void* obase = p.o;
+      int orow = q_row, orows = p.S;
+      if (p.n_shards > 1) {  // the pair's sequence shard
+        obase = p.o_shard[it.shard];
+        orow = q_row - it.shard * p.shard_rows;
+        orows = p.shard_rows;
+      }
+      const size_t o_idx = (((size_t)it.b * orows + orow) * p.H + it.h) * D;
       if (n_kept > 0) {
         ok = mbar_wait(bars.pv_done(lane_t), (total_pv - 1) & 1, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err);
         ok = __all_sync(0xffffffffu, ok);
@@ -623,14 +648,14 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
           tmem_wait_ld();
           if (row_ok) {
             if (p.o_f32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + o_idx + c * 32);
+              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(obase) + o_idx + c * 32);
 #pragma unroll
               for (int e = 0; e < 8; ++e)
                 dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
                                      __uint_as_float(o[4 * e + 2]) * inv_l,
                                      __uint_as_float(o[4 * e + 3]) * inv_l);
             } else {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + o_idx + c * 32);
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(obase) + o_idx + c * 32);
 #pragma unroll
               for (int e = 0; e < 4; ++e)
                 dst[e] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * e]) * inv_l, __uint_as_float(o[8 * e + 1]) * inv_l),
@@ -642,10 +667,10 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
         }
       } else if (row_ok) {
         if (p.o_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(p.o) + o_idx);
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(obase) + o_idx);
           for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
         } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.o) + o_idx);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(obase) + o_idx);
           for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
@@ -661,8 +686,7 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
 
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_fwd_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                    const __grid_constant__ CUtensorMap tv, const __grid_constant__ AttnParams p) {
+    attn_fwd_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ AttnParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -676,8 +700,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   bars.p_full0 = bars.s_full0 + 16;
   bars.pv_done0 = bars.p_full0 + 16;
   bars.o_done0 = bars.pv_done0 + 16;
-  bars.turn0 = bars.o_done0 + 16;
-  bars.drain = bars.turn0 + 16;
+  bars.drain = bars.o_done0 + 16;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   ItemRing ir;
@@ -699,7 +722,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars.p_full(t), 4);   // one arrival per softmax warp
       mbar_init(bars.pv_done(t), 1);
     }
-    for (int k = 0; k < 4; ++k)  // o_done[0..1], turn[0..1] counters
+    for (int k = 0; k < 2; ++k)  // o_done[0..1] counters
       *reinterpret_cast<volatile uint32_t*>(smem + C::kBarOff + (bars.o_done0 - bar0) + 8 * k) = 0u;
     mbar_init(bars.drain, 2);
     *abort_flag = 0;
@@ -709,9 +732,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     fence_mbar_init();
   }
   if (warp == kWarpProducer && lane == 0) {
-    tma_prefetch_desc(&tq);
-    tma_prefetch_desc(&tk);
-    tma_prefetch_desc(&tv);
+    for (int r = 0; r < p.n_shards; ++r) {
+      tma_prefetch_desc(&tm.q[r]);
+      tma_prefetch_desc(&tm.k[r]);
+      tma_prefetch_desc(&tm.v[r]);
+    }
   }
   if (warp == kWarpMma) {
     tmem_alloc(smem_u32(tmem_holder), 512);
@@ -728,7 +753,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     regs_dec<kRegsControl>();
     if (warp == kWarpProducer) {
-      run_producer<D>(p, &tq, &tk, &tv, smem, bars, ir, abort_flag);
+      run_producer<D>(p, tm, smem, bars, ir, abort_flag);
     } else if (warp == kWarpMma || warp == kWarpMma + 1) {
       run_mma<D>(p, smem, bars, ir, tmem, warp - kWarpMma, abort_flag);
     }
@@ -761,10 +786,29 @@ int attn_smem_bytes(int D) { return D == 128 ? Cfg<128>::kSmemBytes : Cfg<64>::k
 sp_status launch_attn(const AttnParams& p_in, const void* q, const void* k, const void* v,
                       cudaStream_t stream) {
   AttnParams p = p_in;
-  CUtensorMap tq, tk, tv;
-  if (!encode_bshd_tmap(&tq, q, p.B, p.S, p.H, p.D) || !encode_bshd_tmap(&tk, k, p.B, p.S, p.H, p.D) ||
-      !encode_bshd_tmap(&tv, v, p.B, p.S, p.H, p.D))
-    return SP_ERR_CUDA;
+  p.n_shards = 1;
+  p.shard_rows = p.S;
+  p.tiles_per_shard = (p.S + kTile - 1) / kTile;
+  p.pairs_per_shard = p.n_qpairs;
+  p.q_shard[0] = q;
+  p.k_shard[0] = k;
+  p.v_shard[0] = v;
+  p.o_shard[0] = p.o;
+  return launch_attn_sharded(p, stream);
+}
+
+sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
+  AttnParams p = p_in;
+  if (p.n_shards < 1 || p.n_shards > kMaxShards || p.shard_rows < 1 || (long long)p.n_shards * p.shard_rows != p.S ||
+      p.tiles_per_shard != (p.shard_rows + kTile - 1) / kTile || p.pairs_per_shard != (p.tiles_per_shard + 1) / 2 ||
+      p.n_qpairs != p.n_shards * p.pairs_per_shard)
+    return SP_ERR_INVALID_ARG;
+  TMaps tm{};  // the kernel argument (copied at launch)
+  for (int r = 0; r < p.n_shards; ++r)
+    if (!encode_bshd_tmap(&tm.q[r], p.q_shard[r], p.B, p.shard_rows, p.H, p.D) ||
+        !encode_bshd_tmap(&tm.k[r], p.k_shard[r], p.B, p.shard_rows, p.H, p.D) ||
+        !encode_bshd_tmap(&tm.v[r], p.v_shard[r], p.B, p.shard_rows, p.H, p.D))
+      return SP_ERR_CUDA;
   if (p.n_items <= 0) return SP_OK;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SP_ERR_CUDA;
@@ -801,7 +845,7 @@ sp_status launch_attn(const AttnParams& p_in, const void* q, const void* k, cons
       if (e != cudaSuccess) return SP_ERR_CUDA;
       attr_set[dev] = true;
     }
-    attn_fwd_kernel<128><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+    attn_fwd_kernel<128><<<grid, kThreads, smem, stream>>>(tm, p);
   } else {
     static bool attr_set[kMaxDevices] = {};
     if (!attr_set[dev]) {
@@ -809,7 +853,7 @@ sp_status launch_attn(const AttnParams& p_in, const void* q, const void* k, cons
       if (e != cudaSuccess) return SP_ERR_CUDA;
       attr_set[dev] = true;
     }
-    attn_fwd_kernel<64><<<grid, kThreads, smem, stream>>>(tq, tk, tv, p);
+    attn_fwd_kernel<64><<<grid, kThreads, smem, stream>>>(tm, p);
   }
   return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
 }

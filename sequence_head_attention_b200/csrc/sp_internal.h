@@ -12,6 +12,7 @@ namespace spattn {
 
 constexpr int kMaxDevices = 64;
 constexpr int kMaxChunks = 128;
+constexpr int kMaxShards = SP_MAX_SHARDS;  // sequence shards one attention launch reads and writes directly
 
 // Parameters of one attention launch (all H heads, all S queries, keys in [kv_begin, kv_lim)).
 struct AttnParams {
@@ -35,6 +36,17 @@ struct AttnParams {
   unsigned long long timeout_ns;
   unsigned int* err;    // device error word of this device
   unsigned int* sched;  // this launch's work counter pair [next item, CTAs finished] (set by launch_attn)
+  // Sequence sharding.  n_shards == 1: Q, K, V and O are the single [B, S, H, D] tensors (o above).
+  // n_shards > 1: each is split along S into n_shards buffers [B, shard_rows, H, D] (row s lives in
+  // shard s / shard_rows at local row s % shard_rows); o is unused and O rows go to o_shard.
+  int n_shards;
+  int shard_rows;
+  int tiles_per_shard;  // ceil(shard_rows / 128): query and key tiles lie on each shard's own grid
+  int pairs_per_shard;  // ceil(tiles_per_shard / 2); n_qpairs = n_shards * pairs_per_shard
+  const void* q_shard[kMaxShards];
+  const void* k_shard[kMaxShards];
+  const void* v_shard[kMaxShards];
+  void* o_shard[kMaxShards];
 };
 
 // Device properties and driver entry points (cached per device).
@@ -47,6 +59,8 @@ unsigned int* device_error_word();  // address of the current device's error wor
 int attn_smem_bytes(int D);
 sp_status launch_attn(const AttnParams& p, const void* q, const void* k, const void* v,
                       cudaStream_t stream);
+// As launch_attn, with Q, K, V (and O) given as the sequence shards in p (n_shards, shard_rows, *_shard).
+sp_status launch_attn_sharded(const AttnParams& p, cudaStream_t stream);
 sp_status launch_merge(const float* const* o_parts, const float* const* lse_parts, int n, void* o,
                        float* lse, int o_f32, int B, int S, int H, int D, cudaStream_t stream);
 sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,

@@ -22,7 +22,7 @@ enum : unsigned int {
   ERR_TIMEOUT_O_FREE = 1u << 7,
   ERR_TIMEOUT_DRAIN = 1u << 8,
   ERR_TIMEOUT_DEBUG = 1u << 9,
-  ERR_TIMEOUT_TURN = 1u << 10,
+  // 1u << 10: unused
   ERR_TIMEOUT_ITEM = 1u << 11,       // waiting for the next work-item id
   ERR_TIMEOUT_ITEM_FREE = 1u << 12,  // waiting for a work-item slot to be read by every role
   ERR_ANY_TIMEOUT = 0x1fffu,

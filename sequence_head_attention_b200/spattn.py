@@ -52,6 +52,7 @@ def lib() -> ctypes.CDLL:
                 "sp_merge_partials": (I, [P, P, I, P, P, I, I, I, I, I, P]),
                 "sp_seq_to_head_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_head_to_seq_relayout": (I, [P, P, I, I, I, I, I, I, P]),
+                "sp_attn_fwd_seq_sharded": (I, [P, P, P, P, P, I, I, I, I, I, I, I, P, I, I, P]),
                 "sp_build_tile_list": (I, [P, I, I, P, P, P, P]),
                 "sp_attn_fwd_sparse_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, P, P]),
                 "sp_status_string": (ctypes.c_char_p, [I]),
@@ -213,6 +214,40 @@ def sp_head_to_seq_relayout(in_ranks, out_ranks, S=None, H=None, stream=None):
     st = lib().sp_head_to_seq_relayout(ip, op, P, B, S, H, D, in_ranks[0].element_size(), _stream(stream))
     _check("sp_head_to_seq_relayout", st)
     return out_ranks
+
+
+def sp_attn_fwd_seq_sharded(q_shards, k_shards, v_shards, o_shards, lse=None, heads=None, head_chunks=None,
+                            causal=False, stream=None):
+    """One Ulysses rank's attention on the sequence shards (bf16 [B, S/P, H, D] each, P of them):
+    heads [h0, h0 + n) with heads=(h0, n) (default: all), written into the heads of o_shards; lse is
+    fp32 [B, H, S] over all heads (rows of the computed heads written) or None.  Bit-identical to the
+    seq -> head relayout, sp_attn_fwd on those heads, and the head -> seq relayout."""
+    P = len(q_shards)
+    _need(P >= 1 and len(k_shards) == P and len(v_shards) == P and len(o_shards) == P, "P shards of each")
+    for group, n in ((q_shards, "q"), (k_shards, "k"), (v_shards, "v"), (o_shards, "o")):
+        for i, t in enumerate(group):
+            _bshd(t, f"{n}_shards[{i}]")
+            _need(t.shape == q_shards[0].shape, "all shards must have the same shape")
+    B, Sl, H, D = q_shards[0].shape
+    S = Sl * P
+    h0, n = (0, H) if heads is None else (int(heads[0]), int(heads[1]))
+    if lse is not None:
+        _need(lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, S),
+              "lse must be contiguous fp32 [B, H, S]")
+    hc = None
+    n_hc = 0
+    if head_chunks is not None:
+        n_hc = len(head_chunks)
+        hc = (ctypes.c_int * n_hc)(*[int(c) for c in head_chunks])
+    qp, _k1 = _ptr_array(q_shards)
+    kp, _k2 = _ptr_array(k_shards)
+    vp, _k3 = _ptr_array(v_shards)
+    op, _k4 = _ptr_array(o_shards)
+    st = lib().sp_attn_fwd_seq_sharded(qp, kp, vp, op, _ptr(lse), P, B, S, H, D, h0, n,
+                                       ctypes.cast(hc, ctypes.c_void_p) if hc is not None else None, n_hc,
+                                       int(bool(causal)), _stream(stream))
+    _check("sp_attn_fwd_seq_sharded", st)
+    return o_shards, lse
 
 
 def sp_attn_fwd_sparse_noalloc(q, k, v, o, lse, block_mask, causal=False, stream=None):

@@ -6,6 +6,8 @@ part of the path on the current stream through the C ABI; nothing here computes 
 UlyssesStep   video-DiT shape: Q, K, V arrive as P sequence shards (one buffer per simulated rank);
               seq -> head relayout of each; attention of every rank on its H/P heads, with the global
               head chunks split at the rank boundaries; head -> seq relayout of O back to sequence shards.
+              With fused=True each rank's attention reads the sequence shards and writes O into them
+              directly (sp_attn_fwd_seq_sharded), with the same result and no relayout pass.
 RingStep      long causal shape: 8 contiguous KV blocks, one partial launch each (every query against one
               block, fp32 partials), then the log-sum-exp re-merge into bf16 O and fp32 LSE.
 SparseStep    block-sparse DiT shape: tile-list build from the mask, then one attention launch that
@@ -37,8 +39,9 @@ def rank_chunks(chunks, H, P):
 
 
 class UlyssesStep:
-    def __init__(self, w: Workload, q, k, v, device="cuda"):
+    def __init__(self, w: Workload, q, k, v, device="cuda", fused=False):
         self.w = w
+        self.fused = fused
         P, B, S, H, D = w.ranks, w.B, w.S, w.H, w.D
         self.P, self.Hl = P, H // P
         self.chunks = rank_chunks(w.head_chunks or (H,), H, P)
@@ -52,7 +55,8 @@ class UlyssesStep:
         self.o_head = [torch.empty(shard, dtype=torch.bfloat16, device=device) for _ in range(P)]
         self.lse = [torch.empty((B, self.Hl, S), dtype=torch.float32, device=device) for _ in range(P)]
         self.o_seq = [torch.empty((B, S // P, H, D), dtype=torch.bfloat16, device=device) for _ in range(P)]
-        self.launches = 3 + P + 1
+        self.lse_all = torch.empty((B, H, S), dtype=torch.float32, device=device)  # fused path
+        self.launches = P if fused else 3 + P + 1
         self.flops = w.flops()
         self.relayout_bytes = 4 * 2 * B * S * H * D * 2  # 4 tensors, each read once and written once
 
@@ -69,13 +73,21 @@ class UlyssesStep:
     def relayout_out(self, stream=None):
         spattn.sp_head_to_seq_relayout(self.o_head, self.o_seq, stream=stream)
 
+    def attention_rank_fused(self, r, stream=None):
+        spattn.sp_attn_fwd_seq_sharded(self.q_seq, self.k_seq, self.v_seq, self.o_seq, self.lse_all,
+                                       heads=(r * self.Hl, self.Hl), head_chunks=self.chunks[r], stream=stream)
+
     def run(self, stream=None):
+        if self.fused:
+            for r in range(self.P):
+                self.attention_rank_fused(r, stream)
+            return
         self.relayout_in(stream)
         self.attention(stream)
         self.relayout_out(stream)
 
     def lse_full(self):
-        return torch.cat(self.lse, dim=1)
+        return self.lse_all if self.fused else torch.cat(self.lse, dim=1)
 
     def inputs(self):
         return self.q_seq + self.k_seq + self.v_seq

@@ -24,7 +24,9 @@ def _sampled(o, lse, rows):
 def test_video_dit_ulysses_step():
     w = synth.WORKLOADS["video_dit"]
     q, k, v = synth.qkv(w.B, w.S, w.H, w.D, seed=0, scale=w.scale)
-    rows = synth.sample_rows(w.S, N_ROWS, seed=0)
+    sr = w.S // w.ranks  # rows per sequence shard: each shard's first and last rows, and its short last tile
+    rows = synth.sample_rows(w.S, N_ROWS, seed=0,
+                             must=[x for r in range(w.ranks) for x in (r * sr, r * sr + 63 * 128, (r + 1) * sr - 1)])
     ref = _oracle_rows(q, k, v, rows)
     # attention on the full 40-head tensors with the uneven head chunks
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
@@ -43,6 +45,16 @@ def test_video_dit_ulysses_step():
     assert torch.equal(o_full, o)  # same per-head arithmetic, bitwise
     lse_full = step.lse_full()
     assert torch.equal(lse_full, lse)
+    # the same step with the relayouts folded into the attention kernel (shards of 8190 rows, tiled on
+    # their own grids: 63 full tiles and one of 126 rows each)
+    fused = workloads.UlyssesStep(w, q, k, v, fused=True)
+    fused.run()
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    o_fused = torch.cat(fused.o_seq, dim=1)
+    o_s, l_s = _sampled(o_fused, fused.lse_full(), rows)
+    assert_close(o_s, ref[0], l_s, ref[1])
+    assert_close(o_fused, o, fused.lse_full(), lse)
 
 
 def test_ring_causal_partials_and_merge():
