@@ -260,6 +260,28 @@ def run_reference(args):
     return 0
 
 
+def dbsp_ranks_report(step, P, reps, stream, E):
+    """Block-sparse attention split over P simulated sequence-parallel ranks, by the contiguous head split
+    of Ulysses and by the db-SP plan: each rank's item-list launch is timed on its own (CUDA events), and
+    a parallel step would take the slowest rank's time."""
+    import torch
+    out = {"ranks": P, "how": "per-rank item-list launches timed one by one on this GPU; step = slowest rank"}
+    for name, planned in (("head_split", False), ("planned", True)):
+        lists, imb = step.rank_items(P, planned)
+        for items in lists:  # warm-up
+            step.run_items(items)
+        marks = []
+        for _ in range(reps):
+            for r, items in enumerate(lists):
+                a = E(); a.record(stream); step.run_items(items); b = E(); b.record(stream)
+                marks.append((r, a, b))
+        torch.cuda.synchronize()
+        per_rank = [statistics.mean(a.elapsed_time(b) for rr, a, b in marks if rr == r) for r in range(P)]
+        out[name] = {"imbalance": imb, "rank_ms": per_rank, "max_rank_ms": max(per_rank)}
+    out["speedup_of_plan"] = out["head_split"]["max_rank_ms"] / out["planned"]["max_rank_ms"]
+    return out
+
+
 def run_ours(args):
     import torch
     from sequence_head_attention_b200 import spattn, workloads
@@ -370,6 +392,8 @@ def run_ours(args):
     else:
         attn_ms = statistics.mean(phase["attn"])
         flops_launch = step.flops
+        if args.dbsp_ranks > 1:
+            kernels["dbsp"] = dbsp_ranks_report(step, args.dbsp_ranks, max(3, args.steps // 2), stream, E)
     achieved = flops_launch / (attn_ms / 1000.0) / 1e12
     kernels["attention"] = {"tflops": achieved, "ms_per_launch": attn_ms}
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
@@ -449,6 +473,9 @@ def main(argv=None):
     ap.add_argument("--ulysses", choices=["fused", "relayout"], default="fused",
                     help="video_dit step: attention straight on the sequence shards (fused), or the seq->head "
                          "relayout, per-rank attention and head->seq relayout")
+    ap.add_argument("--dbsp-ranks", type=int, default=4,
+                    help="block_sparse: also time the work split over this many simulated ranks, head split "
+                         "vs db-SP plan (0: off)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -179,6 +179,42 @@ SP_API sp_status sp_attn_fwd_seq_sharded(const void* const* q_shards, const void
                                          int n_head_chunks, int causal, sp_stream stream);
 
 /*
+ * db-SP work partition ("db-SP: ... Sparsity-Aware Sequence Parallelism ...", abstract: dual-level
+ * partitioning over heads and blocks balancing block-sparse attention; the page gives neither the imbalance
+ * formula nor the algorithm, so these are this library's reading).  Host functions on host arrays; no GPU.
+ *
+ * Work unit: (head h, query-tile pair qp), qp < NP = ceil(T/2), T = ceil(S/128): the kernel's work item.
+ * Unit u = h * NP + qp costs the 128 x 128 tiles its two query-tile rows keep (keys j <= i when causal).
+ *
+ * sp_dbsp_unit_costs  block_mask: host u8 [H, T, T] or NULL (dense); cost: host int64 [H * NP] (out).
+ * sp_dbsp_plan        cost [H * NP] -> unit_rank [H * NP] (out, host): level 1 places whole heads, longest
+ *                     first, on the least loaded rank; level 2 moves single units from the most to the
+ *                     least loaded rank while a unit with 0 < cost < (max - min load) exists (the one with
+ *                     2 cost closest to the gap).  Ties: lower head / unit / rank first.  rank_load [P]
+ *                     and imbalance (max load / mean load) are optional outputs.  1 <= P <= SP_MAX_RANKS.
+ * sp_dbsp_rank_items  the kernel item ids of rank `rank` for batch size B, (b * H + h) * NP + qp, longest
+ *                     unit first; items may be NULL to query the count (*n_items), else capacity must hold it.
+ */
+SP_API sp_status sp_dbsp_unit_costs(const uint8_t* block_mask, int H, int T, int causal, long long* cost);
+SP_API sp_status sp_dbsp_plan(const long long* cost, int H, int NP, int P, int* unit_rank, long long* rank_load,
+                              double* imbalance);
+SP_API sp_status sp_dbsp_rank_items(const long long* cost, const int* unit_rank, int B, int H, int NP, int rank,
+                                    int* items, int capacity, int* n_items);
+
+/*
+ * Attention over an explicit list of work items: exactly what sp_attn_fwd (one head chunk, one KV block)
+ * writes for those items' rows, and nothing else (other rows of o and lse are left untouched).
+ * items: device int [n_items], ids (b * H + h) * ceil(ceil(S/128)/2) + qp of the one-chunk layout (e.g.
+ * from sp_dbsp_rank_items); each names query tiles 2 qp and 2 qp + 1 of head h, batch b.  An id outside
+ * that range is skipped and reported by sp_check_device_error as SP_ERR_INVALID_ARG.  Items are claimed in
+ * list order.  Workspace and the other arguments as in sp_attn_fwd (n_kv_blocks = 1).
+ */
+SP_API sp_status sp_attn_fwd_items(const void* q, const void* k, const void* v, void* o, float* lse, int B, int S,
+                                   int H, int D, const int* items, int n_items, int causal,
+                                   const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
+                                   sp_stream stream);
+
+/*
  * Block-sparse attention that allocates nothing, for callers that cannot call cudaMalloc (a serving
  * path that must not block on the device synchronisation an allocation may cause, a plug-in handed
  * tensors by a framework that owns all device memory, a real-time loop that forbids allocation after

@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libspattn.so")
 BUILD_DIR = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "attn_fwd.cu", "merge.cu", "relayout.cu", "tile_list.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "attn_fwd.cu", "merge.cu", "relayout.cu", "tile_list.cu", "noalloc.cu", "dbsp_plan.cpp"]
 HEADERS = ["sp_internal.h", "sp_ptx.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",
@@ -33,7 +33,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     objs = []
     for src in SOURCES:
         s = os.path.join(CSRC, src)
-        o = os.path.join(BUILD_DIR, src.replace(".cu", ".o"))
+        o = os.path.join(BUILD_DIR, os.path.splitext(src)[0] + ".o")
         objs.append(o)
         if force or _stale(o, [s] + hdrs):
             cmd = [NVCC] + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", s, "-o", o]

@@ -189,7 +189,8 @@ sp_status sp_check_device_error_bits(sp_stream stream, unsigned int* bits) {
   if (cudaMemcpyFromSymbol(&v, g_sp_error, sizeof(v)) != cudaSuccess) return SP_ERR_CUDA;
   if (v != 0 && cudaMemcpyToSymbol(g_sp_error, &zero, sizeof(zero)) != cudaSuccess) return SP_ERR_CUDA;
   if (bits) *bits = v;
-  return (v & ERR_ANY_TIMEOUT) ? SP_ERR_TIMEOUT : SP_OK;
+  if (v & ERR_ANY_TIMEOUT) return SP_ERR_TIMEOUT;
+  return (v & ERR_BAD_ITEM) ? SP_ERR_INVALID_ARG : SP_OK;
 }
 
 sp_status sp_check_device_error(sp_stream stream) { return sp_check_device_error_bits(stream, nullptr); }
@@ -428,6 +429,41 @@ sp_status sp_attn_fwd_seq_sharded(const void* const* q_shards, const void* const
     p.o_shard[r] = o_shards[r];
   }
   return launch_attn_sharded(p, as_stream(stream));
+}
+
+sp_status sp_attn_fwd_items(const void* q, const void* k, const void* v, void* o, float* lse, int B, int S, int H,
+                            int D, const int* items, int n_items, int causal, const uint8_t* block_mask,
+                            void* workspace, size_t workspace_bytes, sp_stream stream) {
+  if (!sizes_ok(B, S, H, D)) return SP_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || n_items < 0 || (n_items > 0 && !items)) return SP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || (lse && !aligned16(lse)))
+    return SP_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SP_ERR_INVALID_ARG;
+  const WsLayout wl = ws_layout(B, S, H, D, 1, block_mask != nullptr);
+  if (wl.total > 0 && (!workspace || workspace_bytes < wl.total || !aligned16(workspace)))
+    return SP_ERR_INVALID_ARG;
+  if (n_items == 0) return SP_OK;
+  cudaStream_t st = as_stream(stream);
+  AttnParams p;
+  int h0[2] = {0, H};
+  sp_status s = fill_attn_params(p, B, S, H, D, 0, S, causal, h0, 1);
+  if (s != SP_OK) return s;
+  p.item_space = p.n_items;
+  p.item_list = items;
+  p.n_items = n_items;
+  p.o = o;
+  p.o_f32 = 0;
+  p.lse = lse;
+  if (block_mask) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* row_ptr = reinterpret_cast<int32_t*>(ws + wl.row_ptr);
+    int32_t* col_idx = reinterpret_cast<int32_t*>(ws + wl.col_idx);
+    s = launch_tile_list(block_mask, H, p.mask_T, row_ptr, col_idx, reinterpret_cast<int32_t*>(ws + wl.counts), st);
+    if (s != SP_OK) return s;
+    p.row_ptr = row_ptr;
+    p.col_idx = col_idx;
+  }
+  return launch_attn(p, q, k, v, st);
 }
 
 sp_status sp_seq_to_head_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,

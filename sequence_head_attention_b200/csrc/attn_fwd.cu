@@ -99,9 +99,16 @@ struct Item {
   int q_last[2];   // last row of each lane's tile that exists (global position)
   int q_end;       // one past the last row of the shard (rows from here on belong to the next shard)
   bool valid[2];
+  bool id_ok;      // false: the item list named an item that does not exist
 };
 
 __device__ __forceinline__ Item decode_item(const AttnParams& p, int w) {
+  bool id_ok = true;
+  if (p.item_list) {  // an explicit list: ids of the one-chunk layout, query-tile pair as given
+    w = __ldg(p.item_list + w);
+    id_ok = w >= 0 && w < p.item_space;
+    if (!id_ok) w = 0;
+  }
   // Items are ordered by head chunk, then batch, then head, then query-tile pair, so that the CTAs
   // running at the same time share one head's K/V in L2.  When causal, a head's pairs run longest
   // first, so that the last items of a launch, claimed by whichever CTA is free, are the short ones.
@@ -115,7 +122,7 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p, int w) {
   const int r2 = r - it.b * per_b;
   it.h = p.chunk_h0[c] + r2 / p.n_qpairs;
   const int qq = r2 % p.n_qpairs;
-  it.qp = p.causal ? (p.n_qpairs - 1 - qq) : qq;
+  it.qp = (p.causal && !p.item_list) ? (p.n_qpairs - 1 - qq) : qq;
   // Query tiles are laid on each shard's own 128-row grid (one shard: the global grid); a shard's last
   // tile may be short, and pairs never cross shards.
   it.shard = it.qp / p.pairs_per_shard;
@@ -128,6 +135,8 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p, int w) {
     it.valid[t] = lt < p.tiles_per_shard && it.q_start[t] < it.q_end;
     it.q_last[t] = min(it.q_end, it.q_start[t] + kTile) - 1;
   }
+  it.id_ok = id_ok;
+  if (!id_ok) it.valid[0] = it.valid[1] = false;  // nothing computed, nothing written
   return it;
 }
 
@@ -313,6 +322,7 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
     __syncwarp();
     if (done) break;
     const Item it = decode_item(p, w);
+    if (!it.id_ok && elect_one_sync()) atomicOr(p.err, ERR_BAD_ITEM);
     if (n_item > 0) {
       ok = warp_mbar_wait(bars.q_empty, q_empty_ph, tmo, ERR_TIMEOUT_Q_EMPTY, abort_flag, p.err);
       q_empty_ph ^= 1;

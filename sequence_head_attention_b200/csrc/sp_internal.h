@@ -27,6 +27,9 @@ struct AttnParams {
   void* o;          // bf16 or fp32 BSHD
   int o_f32;
   float* lse;       // [B, H, S] or nullptr
+  const int* item_list; // device list of work-item ids (nullptr: items 0 .. n_items-1); ids index the
+                        // one-chunk layout (b * H + h) * n_qpairs + qp, and ids outside it are skipped
+  int item_space;       // number of valid ids (B * H * n_qpairs) when item_list is set
   const int* row_ptr;  // block-sparse tile list (nullptr: dense)
   const int* col_idx;
   int mask_T;          // ceil(S/128)

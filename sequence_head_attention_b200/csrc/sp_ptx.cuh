@@ -26,6 +26,7 @@ enum : unsigned int {
   ERR_TIMEOUT_ITEM = 1u << 11,       // waiting for the next work-item id
   ERR_TIMEOUT_ITEM_FREE = 1u << 12,  // waiting for a work-item slot to be read by every role
   ERR_ANY_TIMEOUT = 0x1fffu,
+  ERR_BAD_ITEM = 1u << 16,           // an item list named a work item that does not exist (skipped)
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {

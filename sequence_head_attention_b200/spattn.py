@@ -53,6 +53,10 @@ def lib() -> ctypes.CDLL:
                 "sp_seq_to_head_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_head_to_seq_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_attn_fwd_seq_sharded": (I, [P, P, P, P, P, I, I, I, I, I, I, I, P, I, I, P]),
+                "sp_attn_fwd_items": (I, [P, P, P, P, P, I, I, I, I, P, I, I, P, P, Z, P]),
+                "sp_dbsp_unit_costs": (I, [P, I, I, I, P]),
+                "sp_dbsp_plan": (I, [P, I, I, I, P, P, P]),
+                "sp_dbsp_rank_items": (I, [P, P, I, I, I, I, P, I, P]),
                 "sp_build_tile_list": (I, [P, I, I, P, P, P, P]),
                 "sp_attn_fwd_sparse_noalloc": (I, [P, P, P, P, P, I, I, I, I, I, P, P]),
                 "sp_status_string": (ctypes.c_char_p, [I]),
@@ -248,6 +252,73 @@ def sp_attn_fwd_seq_sharded(q_shards, k_shards, v_shards, o_shards, lse=None, he
                                        int(bool(causal)), _stream(stream))
     _check("sp_attn_fwd_seq_sharded", st)
     return o_shards, lse
+
+
+def sp_dbsp_unit_costs(block_mask, H, T, causal=False):
+    """Host: kept tiles per (head, query-tile pair) unit, int64 [H, ceil(T/2)] (block_mask: host uint8
+    [H, T, T] tensor or array, or None for dense)."""
+    import numpy as np
+    NP = (T + 1) // 2
+    cost = np.zeros((H, NP), dtype=np.int64)
+    m = None
+    if block_mask is not None:
+        m = np.ascontiguousarray(block_mask.cpu().numpy() if isinstance(block_mask, torch.Tensor) else block_mask,
+                                 dtype=np.uint8)
+        _need(m.shape == (H, T, T), "block_mask must be [H, T, T]")
+    st = lib().sp_dbsp_unit_costs(None if m is None else m.ctypes.data, H, T, int(bool(causal)), cost.ctypes.data)
+    _check("sp_dbsp_unit_costs", st)
+    return cost
+
+
+def sp_dbsp_plan(cost, P):
+    """Host: (unit_rank int32 [H, NP], rank_load int64 [P], imbalance) of the two-level partition."""
+    import numpy as np
+    cost = np.ascontiguousarray(cost, dtype=np.int64)
+    H, NP = cost.shape
+    unit_rank = np.zeros((H, NP), dtype=np.int32)
+    load = np.zeros(P, dtype=np.int64)
+    imb = ctypes.c_double(0.0)
+    st = lib().sp_dbsp_plan(cost.ctypes.data, H, NP, int(P), unit_rank.ctypes.data, load.ctypes.data,
+                            ctypes.byref(imb))
+    _check("sp_dbsp_plan", st)
+    return unit_rank, load, imb.value
+
+
+def sp_dbsp_rank_items(cost, unit_rank, B, rank):
+    """Host: int32 kernel item ids of one rank, longest unit first."""
+    import numpy as np
+    cost = np.ascontiguousarray(cost, dtype=np.int64)
+    unit_rank = np.ascontiguousarray(unit_rank, dtype=np.int32)
+    H, NP = cost.shape
+    n = ctypes.c_int(0)
+    _check("sp_dbsp_rank_items", lib().sp_dbsp_rank_items(cost.ctypes.data, unit_rank.ctypes.data, B, H, NP,
+                                                          int(rank), None, 0, ctypes.byref(n)))
+    items = np.zeros(max(n.value, 1), dtype=np.int32)
+    _check("sp_dbsp_rank_items", lib().sp_dbsp_rank_items(cost.ctypes.data, unit_rank.ctypes.data, B, H, NP,
+                                                          int(rank), items.ctypes.data, n.value, ctypes.byref(n)))
+    return items[:n.value]
+
+
+def sp_attn_fwd_items(q, k, v, o, lse, items, causal=False, block_mask=None, workspace=None, stream=None):
+    """Attention of the listed work items only (items: device int32 tensor of item ids)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _bshd(t, n)
+    B, S, H, D = q.shape
+    _need(items.dtype == torch.int32 and items.is_cuda and items.is_contiguous(), "items must be CUDA int32")
+    if lse is not None:
+        _need(lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, S),
+              "lse must be contiguous fp32 [B, H, S]")
+    if block_mask is not None:
+        _need(block_mask.dtype == torch.uint8 and block_mask.is_contiguous(), "block_mask must be uint8")
+    ws_bytes = sp_attn_fwd_workspace_bytes(B, S, H, D, 1, block_mask is not None)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    st = lib().sp_attn_fwd_items(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, S, H, D, _ptr(items),
+                                 items.numel(), int(bool(causal)), _ptr(block_mask), _ptr(workspace),
+                                 0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                 _stream(stream))
+    _check("sp_attn_fwd_items", st)
+    return o, lse
 
 
 def sp_attn_fwd_sparse_noalloc(q, k, v, o, lse, block_mask, causal=False, stream=None):

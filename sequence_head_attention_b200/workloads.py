@@ -158,6 +158,28 @@ class SparseStep:
         spattn.sp_attn_fwd(self.q, self.k, self.v, self.o, self.lse, block_mask=self.mask,
                            workspace=self.ws, stream=stream)
 
+    def rank_items(self, P: int, planned: bool):
+        """Device item lists of P simulated sequence-parallel ranks: the db-SP two-level plan, or the
+        contiguous head split of Ulysses (rank r takes heads [r H/P, (r+1) H/P)).  Returns (lists,
+        imbalance ratio)."""
+        import numpy as np
+        w = self.w
+        T = (w.S + TILE - 1) // TILE
+        cost = spattn.sp_dbsp_unit_costs(self.mask.cpu(), w.H, T, w.causal)
+        if planned:
+            unit_rank, load, imb = spattn.sp_dbsp_plan(cost, P)
+        else:
+            unit_rank = np.repeat((np.arange(w.H) * P // w.H)[:, None], cost.shape[1], axis=1).astype(np.int32)
+            load = np.array([cost[unit_rank == r].sum() for r in range(P)])
+            imb = float(load.max() * P / load.sum())
+        lists = [torch.from_numpy(spattn.sp_dbsp_rank_items(cost, unit_rank, w.B, r)).to(self.q.device)
+                 for r in range(P)]
+        return lists, imb
+
+    def run_items(self, items, stream=None):
+        spattn.sp_attn_fwd_items(self.q, self.k, self.v, self.o, self.lse, items, causal=self.w.causal,
+                                 block_mask=self.mask, workspace=self.ws, stream=stream)
+
     def inputs(self):
         return [self.q, self.k, self.v]
 

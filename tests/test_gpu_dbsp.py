@@ -1,0 +1,69 @@
+"""Per-rank attention over planned work-item lists (sp_attn_fwd_items): the ranks' launches together write
+exactly what one launch writes (bitwise: each item's arithmetic is the same), which matches the oracle."""
+import pytest
+import torch
+
+import oracle
+from tests.helpers import assert_close, to64
+from sequence_head_attention_b200 import spattn, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _ranks_launch(q, k, v, cost, unit_rank, P, causal, mask):
+    B, S, H, D = q.shape
+    o = torch.full((B, S, H, D), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, H, S), float("nan"), device="cuda")
+    for r in range(P):
+        items = torch.from_numpy(spattn.sp_dbsp_rank_items(cost, unit_rank, B, r)).cuda()
+        spattn.sp_attn_fwd_items(q, k, v, o, lse, items, causal=causal, block_mask=mask)
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    return o, lse
+
+
+@pytest.mark.parametrize("B,S,H,D,P,causal,sparse", [
+    (1, 2048, 8, 128, 4, False, True), (2, 1000, 3, 64, 2, True, True), (1, 1536, 6, 128, 3, True, False),
+])
+def test_planned_ranks_equal_one_launch_and_oracle(B, S, H, D, P, causal, sparse):
+    q, k, v = (t.cuda() for t in synth.qkv(B, S, H, D, seed=S + P, scale=0.5))
+    T = (S + 127) // 128
+    mask_cpu = synth.block_mask(H, S, seed=P) if sparse else None
+    mask = None if mask_cpu is None else mask_cpu.cuda()
+    cost = spattn.sp_dbsp_unit_costs(mask_cpu, H, T, causal)
+    unit_rank, _, _ = spattn.sp_dbsp_plan(cost, P)
+    o, lse = _ranks_launch(q, k, v, cost, unit_rank, P, causal, mask)
+    o1 = torch.empty_like(o)
+    l1 = torch.empty_like(lse)
+    spattn.sp_attn_fwd(q, k, v, o1, l1, causal=causal, block_mask=mask)
+    torch.cuda.synchronize()
+    assert torch.equal(o, o1) and torch.equal(lse, l1)
+    ref = oracle.attention(to64(q.cpu()), to64(k.cpu()), to64(v.cpu()), causal=causal,
+                           block_mask=None if mask_cpu is None else mask_cpu.numpy())
+    assert_close(o, ref[0], lse, ref[1])
+
+
+def test_unknown_item_is_skipped_and_reported():
+    B, S, H, D = 1, 1024, 2, 128
+    q, k, v = (t.cuda() for t in synth.qkv(B, S, H, D, seed=3, scale=0.5))
+    NP = (S // 128 + 1) // 2
+    o = torch.full((B, S, H, D), 5.0, dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, H, S), 5.0, device="cuda")
+    items = torch.tensor([3, B * H * NP, 0], dtype=torch.int32, device="cuda")  # the middle id does not exist
+    spattn.sp_attn_fwd_items(q, k, v, o, lse, items)
+    assert spattn.sp_check_device_error() == spattn.SP_ERR_INVALID_ARG
+    assert spattn.sp_check_device_error() == spattn.SP_OK  # cleared
+    ref = oracle.attention(to64(q.cpu()), to64(k.cpu()), to64(v.cpu()))
+    # item 0: head 0, rows 0-255; item 3: head 0, rows 768-1023 (NP = 4)
+    for rows in (slice(0, 256), slice(768, 1024)):
+        assert_close(o[:, rows, 0:1], ref[0][:, rows, 0:1], lse[:, 0:1, rows], ref[1][:, 0:1, rows])
+    assert torch.all(o[:, 256:768, 0] == 5.0) and torch.all(o[:, :, 1] == 5.0)
+    assert torch.all(lse[:, 1] == 5.0)
+
+
+def test_empty_item_list_is_a_no_op():
+    q = torch.zeros((1, 256, 1, 64), dtype=torch.bfloat16, device="cuda")
+    o = torch.full_like(q, 2.0)
+    spattn.sp_attn_fwd_items(q, q, q, o, None, torch.zeros(0, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    assert torch.all(o == 2.0)
