@@ -58,8 +58,9 @@ def _load(path: str | None = None):
             lib.orc_seq_to_head.argtypes = [P, P, I, I, I, I, I, I]
             lib.orc_head_to_seq.argtypes = [P, P, I, I, I, I, I, I]
             lib.orc_tile_list.argtypes = [P, I, I, I, P, P, ctypes.c_long]
+            lib.orc_attn_bwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I]
             for f in (lib.orc_attn, lib.orc_attn_probs, lib.orc_merge, lib.orc_seq_to_head,
-                      lib.orc_head_to_seq, lib.orc_tile_list):
+                      lib.orc_head_to_seq, lib.orc_tile_list, lib.orc_attn_bwd):
                 f.restype = ctypes.c_int
             _libs[key] = lib
     return _libs[key]
@@ -114,6 +115,27 @@ def attention(q, k, v, *, causal=False, block_mask=None, tile=TILE, kv_begin=0, 
     if rc:
         raise ValueError(f"orc_attn failed ({rc})")
     return o, lse
+
+
+def attention_bwd(q, k, v, dout, *, causal=False, nthreads=None, lib=None):
+    """Gradients (dq, dk, dv) of the exact attention, in fp64, for an upstream gradient dout of o.
+
+    The backward pass whose speed "CHARM+ ..." (abstract) reports, written as plain calculus on the same
+    definition as :func:`attention` (all keys, optionally causal): dv_j = sum_i p_ij do_i;
+    dp_ij = do_i . v_j; delta_i = sum_j p_ij dp_ij; ds_ij = p_ij (dp_ij - delta_i);
+    dq_i = sum_j ds_ij k_j / sqrt(D); dk_j = sum_i ds_ij q_i / sqrt(D).  All arrays [B, S, H, D]."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, S, H, D = q.shape
+    for t in (k, v, dout):
+        if t.shape != q.shape:
+            raise ValueError("q, k, v, dout must share one [B, S, H, D] shape")
+    dq, dk, dv = np.zeros_like(q), np.zeros_like(q), np.zeros_like(q)
+    nthreads = nthreads or os.cpu_count() or 1
+    rc = _load(lib).orc_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv), B, S, H,
+                              D, int(causal), nthreads)
+    if rc:
+        raise ValueError(f"orc_attn_bwd failed ({rc})")
+    return dq, dk, dv
 
 
 def attention_probs(q, k, v, *, causal=False, block_mask=None, tile=TILE, kv_begin=0, kv_end=None, lib=None):

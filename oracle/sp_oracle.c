@@ -39,6 +39,14 @@
  *                 Byte copies, element by element.
  *  orc_tile_list  The compacted per-(head, query tile) list of kept key tiles of a block mask, in
  *                 increasing key-tile order (CSR: row_ptr, col_idx).
+ *  orc_attn_bwd   The gradients of the attention above (dense or causal, all keys) for an upstream
+ *                 gradient dO of O: the backward pass whose speed the CHARM+ pages report ("CHARM+ ...",
+ *                 abstract: forward and backward speedups).  Plain calculus on the definition: with
+ *                 p_ij the softmax of s_ij = q_i.k_j / sqrt(D) over the allowed j and o_i = sum_j p_ij v_j,
+ *                   dV_j = sum_i p_ij dO_i;   dp_ij = dO_i . v_j;   delta_i = sum_j p_ij dp_ij (= dO_i . o_i);
+ *                   ds_ij = p_ij (dp_ij - delta_i);   dQ_i = sum_j ds_ij k_j / sqrt(D);
+ *                   dK_j = sum_i ds_ij q_i / sqrt(D).
+ *                 Per (batch, head), rows in order, p from the same two-pass softmax as orc_attn.
  *
  * Threads: rows are split over POSIX threads; each row is computed by exactly one thread in a fixed
  * order, so results do not depend on the thread count.
@@ -327,6 +335,97 @@ int orc_head_to_seq(const void* const* in_ranks, void* const* out_ranks, int P, 
  * mask: [H, Tq, Tk] bytes, nonzero = keep.  row_ptr: [H*Tq + 1], col_idx: [nnz] (capacity cap).
  * Row (h, i) lists the kept key tiles j in increasing order.  Returns ORC_EINVAL if cap is too small.
  */
+/* ------------------------------------------------------------------------------------------------ */
+/* Backward: one (batch, head) per task.                                                            */
+/* ------------------------------------------------------------------------------------------------ */
+typedef struct {
+  const double *q, *k, *v, *dout;
+  double *dq, *dk, *dv;
+  int B, S, H, D, causal;
+  int next;
+  pthread_mutex_t mu;
+} bwd_job;
+
+static void bwd_head(bwd_job* J, int b, int h) {
+  const int S = J->S, H = J->H, D = J->D;
+  const double scale = 1.0 / sqrt((double)D);
+#define IDX(t, i, d) ((((size_t)(b) * S + (i)) * H + (h)) * D + (d))
+  double* p = (double*)malloc(sizeof(double) * (size_t)S);
+  double* o = (double*)malloc(sizeof(double) * (size_t)D);
+  for (int j = 0; j < S; ++j)
+    for (int d = 0; d < D; ++d) {
+      J->dk[IDX(k, j, d)] = 0.0;
+      J->dv[IDX(v, j, d)] = 0.0;
+    }
+  for (int i = 0; i < S; ++i) {
+    const int n = J->causal ? i + 1 : S;  /* allowed keys 0 .. n-1 */
+    double m = -INFINITY;
+    for (int j = 0; j < n; ++j) {
+      double s = 0.0;
+      for (int d = 0; d < D; ++d) s += J->q[IDX(q, i, d)] * J->k[IDX(k, j, d)];
+      p[j] = s * scale;
+      if (p[j] > m) m = p[j];
+    }
+    double l = 0.0;
+    for (int j = 0; j < n; ++j) {
+      p[j] = exp(p[j] - m);
+      l += p[j];
+    }
+    for (int j = 0; j < n; ++j) p[j] /= l;
+    for (int d = 0; d < D; ++d) {
+      double acc = 0.0;
+      for (int j = 0; j < n; ++j) acc += p[j] * J->v[IDX(v, j, d)];
+      o[d] = acc;
+    }
+    double delta = 0.0;
+    for (int d = 0; d < D; ++d) delta += J->dout[IDX(dout, i, d)] * o[d];
+    for (int d = 0; d < D; ++d) J->dq[IDX(q, i, d)] = 0.0;
+    for (int j = 0; j < n; ++j) {
+      double dp = 0.0;
+      for (int d = 0; d < D; ++d) dp += J->dout[IDX(dout, i, d)] * J->v[IDX(v, j, d)];
+      const double ds = p[j] * (dp - delta);
+      for (int d = 0; d < D; ++d) {
+        J->dq[IDX(q, i, d)] += ds * J->k[IDX(k, j, d)] * scale;
+        J->dk[IDX(k, j, d)] += ds * J->q[IDX(q, i, d)] * scale;
+        J->dv[IDX(v, j, d)] += p[j] * J->dout[IDX(dout, i, d)];
+      }
+    }
+  }
+#undef IDX
+  free(p);
+  free(o);
+}
+
+static void* bwd_worker(void* arg) {
+  bwd_job* J = (bwd_job*)arg;
+  for (;;) {
+    pthread_mutex_lock(&J->mu);
+    const int t = J->next++;
+    pthread_mutex_unlock(&J->mu);
+    if (t >= J->B * J->H) break;
+    bwd_head(J, t / J->H, t % J->H);
+  }
+  return NULL;
+}
+
+int orc_attn_bwd(const double* q, const double* k, const double* v, const double* dout, double* dq, double* dk,
+                 double* dv, int B, int S, int H, int D, int causal, int nthreads) {
+  if (B < 1 || S < 1 || H < 1 || D < 1 || (causal != 0 && causal != 1)) return ORC_EINVAL;
+  bwd_job J = {q, k, v, dout, dq, dk, dv, B, S, H, D, causal, 0, PTHREAD_MUTEX_INITIALIZER};
+  if (nthreads < 1) nthreads = 1;
+  if (nthreads > B * H) nthreads = B * H;
+  pthread_t th[256];
+  if (nthreads > 256) nthreads = 256;
+  int started = 0;
+  for (int t = 0; t < nthreads; ++t) {
+    if (pthread_create(&th[t], NULL, bwd_worker, &J) != 0) break;
+    ++started;
+  }
+  if (started == 0) bwd_worker(&J);
+  for (int t = 0; t < started; ++t) pthread_join(th[t], NULL);
+  return ORC_OK;
+}
+
 int orc_tile_list(const uint8_t* mask, int H, int Tq, int Tk, int32_t* row_ptr, int32_t* col_idx,
                   long cap) {
   if (H < 1 || Tq < 0 || Tk < 0) return ORC_EINVAL;

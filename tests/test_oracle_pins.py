@@ -436,3 +436,49 @@ def test_planted_mistake_is_caught(name):
             f.write(src.replace(old, new))
         lib = oracle.compile_source(c, os.path.join(d, "libmutant.so"))
         assert not _pins_pass(lib), f"planted mistake {name!r} went unnoticed"
+
+
+# --- backward ------------------------------------------------------------------------------------------
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_bwd_matches_finite_differences(causal):
+    """The gradients equal central differences of L = sum(dO * O) through the forward oracle."""
+    rng = np.random.default_rng(7)
+    B, S, H, D = 1, 6, 2, 3
+    q, k, v, do = (rng.standard_normal((B, S, H, D)) for _ in range(4))
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, causal=causal)
+
+    def loss(qq, kk, vv):
+        return float((do * oracle.attention(qq, kk, vv, causal=causal)[0]).sum())
+
+    eps = 1e-6
+    for x, g, which in ((q, dq, 0), (k, dk, 1), (v, dv, 2)):
+        num = np.zeros_like(x)
+        for idx in np.ndindex(x.shape):
+            args_p = [q, k, v]
+            args_m = [q, k, v]
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += eps
+            xm[idx] -= eps
+            args_p[which], args_m[which] = xp, xm
+            num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+        np.testing.assert_allclose(g, num, atol=1e-7, rtol=1e-6)
+
+
+def test_attention_bwd_invariants_and_single_key():
+    rng = np.random.default_rng(8)
+    B, S, H, D = 2, 9, 3, 5
+    q, k, v, do = (rng.standard_normal((B, S, H, D)) for _ in range(4))
+    for causal in (False, True):
+        dq, dk, dv = oracle.attention_bwd(q, k, v, do, causal=causal)
+        # sum_j ds_ij = 0 for every row, so the key gradients sum to zero; rows of p sum to 1, so the value
+        # gradients sum to the upstream gradients
+        np.testing.assert_allclose(dk.sum(axis=1), 0.0, atol=1e-12)
+        np.testing.assert_allclose(dv.sum(axis=1), do.sum(axis=1), atol=1e-12)
+    # one key: o = v_0 exactly, so dv_0 = do_0 and nothing flows into q or k
+    q1, k1, v1, do1 = (rng.standard_normal((1, 1, 1, 4)) for _ in range(4))
+    dq, dk, dv = oracle.attention_bwd(q1, k1, v1, do1)
+    np.testing.assert_allclose(dv, do1, atol=1e-15)
+    assert np.all(dq == 0) and np.all(dk == 0)
+    # causal: query 0 sees key 0 only, so its gradient does not reach later keys and dq_0 = 0
+    dq, dk, dv = oracle.attention_bwd(q, k, v, do, causal=True)
+    np.testing.assert_allclose(dq[:, 0], 0.0, atol=1e-15)
