@@ -136,6 +136,24 @@ SP_API sp_status sp_merge_partials(const float* const* o_parts, const float* con
                             float* lse, sp_dtype o_dtype, int B, int S, int H, int D, sp_stream stream);
 
 /*
+ * Gradients of the attention of sp_attn_fwd (one head chunk, one KV block, no mask; dense or causal) for
+ * an upstream gradient dout of o: the backward pass whose speed "CHARM+ ..." (abstract) reports next to
+ * the forward's.  With p_ij = exp(q_i.k_j / sqrt(D) - lse_i) over the keys query i sees,
+ *   delta_i = dout_i . o_i,  dv_j = sum_i p_ij dout_i,  ds_ij = p_ij (dout_i . v_j - delta_i),
+ *   dq_i = sum_j ds_ij k_j / sqrt(D),  dk_j = sum_i ds_ij q_i / sqrt(D).
+ * q, k, v, o, dout  device bf16 [B, S, H, D] (o and lse as sp_attn_fwd wrote them for q, k, v);
+ * lse       device fp32 [B, H, S] (natural log);
+ * dq, dk, dv  device bf16 [B, S, H, D] outputs, overlapping nothing else;
+ * workspace  device, sp_attn_bwd_workspace_bytes(B, S, H, D) bytes (the fp32 delta per row).
+ * Three launches on `stream`: delta, then dk and dv (one CTA per key tile), then dq (one per query tile);
+ * p and ds are rounded to bf16 for the tensor cores, accumulation is fp32.  Errors as sp_attn_fwd.
+ */
+SP_API size_t sp_attn_bwd_workspace_bytes(int B, int S, int H, int D);
+SP_API sp_status sp_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, int B, int S, int H, int D, int causal,
+                             void* workspace, size_t workspace_bytes, sp_stream stream);
+
+/*
  * Ulysses relayout, sequence shards -> head shards, between P buffers of one GPU:
  *   in_ranks[r]  device [B, S/P, H, D]   (rank r's slice of the sequence, all heads)
  *   out_ranks[r] device [B, S, H/P, D]   (all positions of heads [r*H/P, (r+1)*H/P))

@@ -12,7 +12,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 OUT = os.path.join(HERE, "libspattn.so")
 BUILD_DIR = os.path.join(HERE, "_build")
-SOURCES = ["api.cu", "attn_fwd.cu", "merge.cu", "relayout.cu", "tile_list.cu", "noalloc.cu", "dbsp_plan.cpp"]
+SOURCES = ["api.cu", "attn_fwd.cu", "merge.cu", "relayout.cu", "tile_list.cu", "noalloc.cu", "dbsp_plan.cpp", "attn_bwd.cu"]
 HEADERS = ["sp_internal.h", "sp_ptx.cuh"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-std=c++17", "-lineinfo",

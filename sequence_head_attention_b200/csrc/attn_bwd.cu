@@ -1,0 +1,482 @@
+// attn_bwd.cu -- gradients of exact multi-head attention on the 5th-generation tensor cores (sm_100a).
+//
+// What it computes (the backward pass of the attention in attn_fwd.cu, whose speed the CHARM+ pages
+// report next to the forward's: "CHARM+ ...", abstract), for an upstream gradient dO of O, with
+// p_ij = exp(q_i.k_j / sqrt(D) - lse_i) over the keys j that query i sees (all, or j <= i when causal):
+//   delta_i = dO_i . O_i
+//   dV_j = sum_i p_ij dO_i,   dp_ij = dO_i . v_j,   ds_ij = p_ij (dp_ij - delta_i)
+//   dK_j = sum_i ds_ij q_i / sqrt(D),   dQ_i = sum_j ds_ij k_j / sqrt(D)
+// lse is the forward's natural-log log-sum-exp, so p is recomputed exactly as the forward normalised it.
+//
+// How: three launches.
+//   bwd_delta_kernel   delta = rowsum(dO * O), fp32 [B, H, S] (HBM-bound, 16-byte loads).
+//   bwd_kernel<D, false>  one CTA per (b, h, key tile of 128): K and V stay in shared memory while the
+//                      query tiles stream through a two-slot ring.  Per query tile, on the tensor cores:
+//                      S^T = K Q^T and dP^T = V dO^T (both operands in shared memory, fp32 in TMEM); the
+//                      four row warps turn them into P^T and dS^T (bf16, written back over S^T and dP^T in
+//                      TMEM); then dV += P^T dO and dK += dS^T Q with the left operand read from TMEM.
+//   bwd_kernel<D, true>   one CTA per (b, h, query tile): Q and dO stay, key tiles stream; S = Q K^T and
+//                      dP = dO V^T, then dS, then dQ += dS K.
+//   Warps: 0 TMA producer, 1 MMA issuer (one elected lane), 2-3 idle, 4-7 the 128 tile rows (one row per
+//   thread: the TMEM lane quadrant of warp w is w % 4).  TMEM: S [0,128), dP [128,256), accumulators
+//   from 256 (dV then dK, or dQ).  The MMA issuer queues the next tile's S and dP right behind the
+//   previous tile's accumulating MMAs: tcgen05 MMAs from one thread execute in order, so the new S cannot
+//   overwrite P before it has been read.
+// Every barrier wait is bounded in time; on expiry the kernel records an error and returns cleanly.
+#include <cuda_bf16.h>
+
+#include <climits>
+#include <cstdint>
+
+#include "sp_internal.h"
+#include "sp_ptx.cuh"
+
+namespace spattn {
+namespace {
+
+constexpr int kBT = 128;           // tile edge
+constexpr int kBwdThreads = 256;   // 8 warps
+constexpr int kWarpLoad = 0, kWarpIssue = 1, kWarpRow0 = 4;
+
+template <int D>
+struct BCfg {
+  static constexpr int kSub = D / 64;
+  static constexpr int kTileBytes = kBT * D * 2;
+  static constexpr int kStages = 2;
+  // resident tiles (K, V or Q, dO) at [0, 2 tiles); then per slot: two streamed tiles and 2 x 128 floats
+  static constexpr int kResOff = 0;
+  static constexpr int kStageOff = 2 * kTileBytes;
+  static constexpr int kStageBytes = 2 * kTileBytes + 1024;
+  static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
+  static constexpr int kNumBars = 1 + 2 * kStages + 4;  // res_full, full[S], empty[S], st_full, p_full, acc_full, drain
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  // one CTA per SM: its TMEM allocation takes all 512 columns
+  static constexpr int kRaw = kMiscOff + 16 + 1024;
+  static constexpr int kSmemBytes = kRaw > 120 * 1024 ? kRaw : 120 * 1024;
+  static constexpr uint32_t kIdescSq = idesc_bf16_f32(128, 128, false, false);  // both operands K-major
+  static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);    // B operand MN-major
+};
+
+struct BwdMaps {
+  CUtensorMap q, k, v, dout;
+};
+
+struct BwdBars {
+  uint32_t res_full, full0, empty0, st_full, p_full, acc_full, drain;
+  __device__ uint32_t full(int s) const { return full0 + 8u * s; }
+  __device__ uint32_t empty(int s) const { return empty0 + 8u * s; }
+};
+
+// The CTA's tile and the range of streamed tiles it walks.
+struct BwdItem {
+  int b, h, tile;      // resident tile index (key tile for dK/dV, query tile for dQ)
+  int first, n_steps;  // streamed tiles first .. first + n_steps - 1
+};
+
+template <bool kDQ>
+__device__ __forceinline__ BwdItem bwd_item(const BwdParams& p) {
+  BwdItem it;
+  const int w = blockIdx.x;
+  it.b = w / (p.H * p.T);
+  it.h = (w / p.T) % p.H;
+  it.tile = w % p.T;
+  if (kDQ) {  // key tiles 0 .. (causal: the query tile's own)
+    it.first = 0;
+    it.n_steps = p.causal ? it.tile + 1 : p.T;
+  } else {    // query tiles (causal: from the key tile's own) .. T-1
+    it.first = p.causal ? it.tile : 0;
+    it.n_steps = p.T - it.first;
+  }
+  return it;
+}
+
+// ------------------------------------------------------------------------------------------------
+template <int D, bool kDQ>
+__device__ void bwd_load(const BwdParams& p, const BwdMaps& tm, const BwdItem& it, uint32_t sbase, uint8_t* smem,
+                         const BwdBars& bars, volatile int* abort_flag) {
+  using C = BCfg<D>;
+  const int lane = threadIdx.x & 31;
+  const uint64_t tmo = p.timeout_ns;
+  const CUtensorMap* res0 = kDQ ? &tm.q : &tm.k;     // resident pair
+  const CUtensorMap* res1 = kDQ ? &tm.dout : &tm.v;
+  const CUtensorMap* str0 = kDQ ? &tm.k : &tm.q;     // streamed pair
+  const CUtensorMap* str1 = kDQ ? &tm.v : &tm.dout;
+  if (elect_one_sync()) {
+    mbar_arrive_expect_tx(bars.res_full, 2 * C::kTileBytes);
+#pragma unroll
+    for (int c = 0; c < C::kSub; ++c) {
+      tma_load_4d(sbase + C::kResOff + c * 16384, res0, bars.res_full, 64 * c, it.h, it.tile * kBT, it.b);
+      tma_load_4d(sbase + C::kResOff + C::kTileBytes + c * 16384, res1, bars.res_full, 64 * c, it.h, it.tile * kBT,
+                  it.b);
+    }
+  }
+  __syncwarp();
+  int issued = 0;
+  bool ok = true;
+  for (int n = 0; n < it.n_steps && ok; ++n) {
+    const int s = n % C::kStages;
+    const int lap = n / C::kStages;
+    if (lap > 0) {
+      ok = warp_mbar_wait(bars.empty(s), (lap - 1) & 1, tmo, ERR_TIMEOUT_KV_EMPTY, abort_flag, p.err);
+      if (!ok) break;
+    }
+    const int t = it.first + n;
+    const uint32_t stage = sbase + C::kStageOff + s * C::kStageBytes;
+    if (!kDQ) {
+      // the streamed query tile's lse (in log2 units) and delta, one per column of S^T; rows past S get
+      // lse = +inf, so their probabilities are exactly 0
+      float* lse2 = reinterpret_cast<float*>(smem + C::kStageOff + s * C::kStageBytes + 2 * C::kTileBytes);
+      float* dlt = lse2 + kBT;
+      const size_t base = ((size_t)it.b * p.H + it.h) * p.S;
+      for (int r = lane; r < kBT; r += 32) {
+        const int row = t * kBT + r;
+        lse2[r] = row < p.S ? __ldg(p.lse + base + row) * 1.4426950408889634f : INFINITY;
+        dlt[r] = row < p.S ? __ldg(p.delta + base + row) : 0.f;
+      }
+      __threadfence_block();
+      __syncwarp();
+    }
+    if (elect_one_sync()) {
+      mbar_arrive_expect_tx(bars.full(s), 2 * C::kTileBytes);
+#pragma unroll
+      for (int c = 0; c < C::kSub; ++c) {
+        tma_load_4d(stage + c * 16384, str0, bars.full(s), 64 * c, it.h, t * kBT, it.b);
+        tma_load_4d(stage + C::kTileBytes + c * 16384, str1, bars.full(s), 64 * c, it.h, t * kBT, it.b);
+      }
+    }
+    __syncwarp();
+    issued = n + 1;
+  }
+  if (*abort_flag) {  // no copy may still be landing when the CTA exits: wait (bounded) for the last ones
+    warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, nullptr, p.err);
+    for (int n = issued > C::kStages ? issued - C::kStages : 0; n < issued; ++n)
+      warp_mbar_wait(bars.full(n % C::kStages), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, nullptr, p.err);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+template <int D, bool kDQ>
+__device__ void bwd_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase, uint32_t tmem_in, const BwdBars& bars,
+                          volatile int* abort_flag) {
+  using C = BCfg<D>;
+  const uint64_t tmo = p.timeout_ns;
+  const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_in, 0);
+  const uint32_t tS = tmem, tdP = tmem + 128, tAcc0 = tmem + 256, tAcc1 = tmem + 256 + D;
+  // K-major descriptors of K-step 0 (the row-major tiles as the MMAs' K-major operands), and MN-major ones
+  // of the streamed tiles as the right operand of the accumulating MMAs.
+  const uint64_t res0_k = smem_desc_sw128(sbase + C::kResOff, 16, 1024);
+  const uint64_t res1_k = smem_desc_sw128(sbase + C::kResOff + C::kTileBytes, 16, 1024);
+  bool ok = warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
+  for (int n = 0; n < it.n_steps && ok; ++n) {
+    const int s = n % C::kStages;
+    const uint32_t stage = sbase + C::kStageOff + s * C::kStageBytes;
+    ok = warp_mbar_wait(bars.full(s), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+    if (!ok) break;
+    tc_fence_after();
+    const uint64_t str0_k = smem_desc_sw128(stage, 16, 1024);
+    const uint64_t str1_k = smem_desc_sw128(stage + C::kTileBytes, 16, 1024);
+    if (elect_one_sync()) {
+      // dK/dV: S^T = K Q^T, dP^T = V dO^T.   dQ: S = Q K^T, dP = dO V^T.
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+        mma_ss(tS, res0_k + off, str0_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
+      }
+#pragma unroll
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+        mma_ss(tdP, res1_k + off, str1_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
+      }
+      mma_commit(bars.st_full);
+    }
+    __syncwarp();
+    ok = warp_mbar_wait(bars.p_full, n & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
+    if (!ok) break;
+    tc_fence_after();
+    const uint32_t acc = n > 0 ? 1u : 0u;
+    if (elect_one_sync()) {
+      // K-steps of 16 rows of the streamed tiles: 8 packed bf16 columns of P / dS, 16 rows of the tile
+      const uint64_t str0_mn = smem_desc_sw128(stage, 16384, 1024);
+      const uint64_t str1_mn = smem_desc_sw128(stage + C::kTileBytes, 16384, 1024);
+      if (kDQ) {
+        // dQ += dS K
+#pragma unroll
+        for (int kk = 0; kk < kBT / 16; ++kk)
+          mma_ts(tAcc0, tdP + kk * 8, str0_mn + (uint64_t)(kk * 128), C::kIdescAcc, kk > 0 ? 1u : acc);
+      } else {
+        // dV += P^T dO, dK += dS^T Q
+#pragma unroll
+        for (int kk = 0; kk < kBT / 16; ++kk)
+          mma_ts(tAcc0, tS + kk * 8, str1_mn + (uint64_t)(kk * 128), C::kIdescAcc, kk > 0 ? 1u : acc);
+#pragma unroll
+        for (int kk = 0; kk < kBT / 16; ++kk)
+          mma_ts(tAcc1, tdP + kk * 8, str0_mn + (uint64_t)(kk * 128), C::kIdescAcc, kk > 0 ? 1u : acc);
+      }
+      mma_commit(bars.empty(s));
+    }
+    __syncwarp();
+  }
+  if (ok && elect_one_sync()) mma_commit(bars.acc_full);
+  __syncwarp();
+  // nothing of ours may still run on the tensor cores when TMEM is released
+  if (elect_one_sync()) mma_commit(bars.drain);
+  __syncwarp();
+  warp_mbar_wait(bars.drain, 0, tmo, ERR_TIMEOUT_DRAIN, nullptr, p.err);
+}
+
+// ------------------------------------------------------------------------------------------------
+template <int D, bool kDQ>
+__device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, uint32_t tmem, const BwdBars& bars,
+                         volatile int* abort_flag) {
+  using C = BCfg<D>;
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int quad = warp & 3;
+  const int r = quad * 32 + lane;                                // row of the resident tile
+  const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+  const uint32_t tS = trow, tdP = trow + 128, tAcc0 = trow + 256, tAcc1 = trow + 256 + D;
+  const uint64_t tmo = p.timeout_ns;
+  const float sl2 = p.scale_log2;
+  const int row = it.tile * kBT + r;                             // global position of this thread's row
+  float lse2_row = 0.f, dlt_row = 0.f;
+  if (kDQ && row < p.S) {
+    const size_t i = ((size_t)it.b * p.H + it.h) * p.S + row;
+    lse2_row = __ldg(p.lse + i) * 1.4426950408889634f;
+    dlt_row = __ldg(p.delta + i);
+  }
+  bool ok = true;
+  for (int n = 0; n < it.n_steps; ++n) {
+    const int t = it.first + n;
+    const float* lse2 = reinterpret_cast<const float*>(smem + C::kStageOff + (n % C::kStages) * C::kStageBytes +
+                                                       2 * C::kTileBytes);
+    const float* dlt = lse2 + kBT;
+    if (!kDQ) {
+      // lse and delta of the streamed tile were stored by the producer before it released the slot's
+      // full barrier: acquire them from that barrier (the slot is refilled only after this step's
+      // P arrives, so the phase cannot have moved on)
+      ok = mbar_wait(bars.full(n % C::kStages), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+    }
+    ok = mbar_wait(bars.st_full, n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    tc_fence_after();
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t s[2][32], dp[2][32];
+      tmem_ld32(tS + 64 * half, s[0]);
+      tmem_ld32(tS + 64 * half + 32, s[1]);
+      tmem_ld32(tdP + 64 * half, dp[0]);
+      tmem_ld32(tdP + 64 * half + 32, dp[1]);
+      tmem_wait_ld();
+      uint32_t pk_p[32], pk_ds[32];
+#pragma unroll
+      for (int e = 0; e < 64; e += 2) {
+        float pr[2], ds[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+          const int c = 64 * half + e + u;  // column: the streamed tile's row
+          const float sv = __uint_as_float(s[(e + u) >> 5][(e + u) & 31]);
+          const float dv = __uint_as_float(dp[(e + u) >> 5][(e + u) & 31]);
+          float pv;
+          if (kDQ) {
+            pv = ex2_approx(sv * sl2 - lse2_row);
+            if (p.causal && t * kBT + c > row) pv = 0.f;  // key after the query
+            ds[u] = pv * (dv - dlt_row);
+          } else {
+            pv = ex2_approx(sv * sl2 - lse2[c]);
+            if (p.causal && t * kBT + c < row) pv = 0.f;  // query before the key
+            ds[u] = pv * (dv - dlt[c]);
+          }
+          pr[u] = pv;
+        }
+        pk_p[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+        pk_ds[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+      }
+      // packed columns [32 half, 32 half + 32) of S and dP: this thread has already read them
+      if (!kDQ) tmem_st32(tS + 32 * half, pk_p);
+      tmem_st32(tdP + 32 * half, pk_ds);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars.p_full);
+  }
+  if (!ok) return;
+  ok = __all_sync(0xffffffffu, mbar_wait(bars.acc_full, 0, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err));
+  if (!ok) return;
+  tc_fence_after();
+  const float scale = p.scale;
+  const size_t out = (((size_t)it.b * p.S + row) * p.H + it.h) * D;
+#pragma unroll
+  for (int which = 0; which < (kDQ ? 1 : 2); ++which) {
+    // dQ: tAcc0, scaled.  dK/dV: dV from tAcc0 unscaled, dK from tAcc1 scaled.
+    const uint32_t tacc = which == 0 ? tAcc0 : tAcc1;
+    const float f = (kDQ || which == 1) ? scale : 1.f;
+    __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(kDQ ? p.dq : (which == 0 ? p.dv : p.dk));
+#pragma unroll 1
+    for (int c = 0; c < D / 32; ++c) {
+      uint32_t a[32];
+      tmem_ld32(tacc + c * 32, a);
+      tmem_wait_ld();
+      if (row < p.S) {
+        uint4* d4 = reinterpret_cast<uint4*>(dst + out + c * 32);
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          d4[e] = make_uint4(pack_bf16x2(__uint_as_float(a[8 * e]) * f, __uint_as_float(a[8 * e + 1]) * f),
+                             pack_bf16x2(__uint_as_float(a[8 * e + 2]) * f, __uint_as_float(a[8 * e + 3]) * f),
+                             pack_bf16x2(__uint_as_float(a[8 * e + 4]) * f, __uint_as_float(a[8 * e + 5]) * f),
+                             pack_bf16x2(__uint_as_float(a[8 * e + 6]) * f, __uint_as_float(a[8 * e + 7]) * f));
+      }
+    }
+  }
+}
+
+template <int D, bool kDQ>
+__global__ void __launch_bounds__(kBwdThreads, 1)
+    bwd_kernel(const __grid_constant__ BwdMaps tm, const __grid_constant__ BwdParams p) {
+  using C = BCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t bar0 = sbase + C::kBarOff;
+  BwdBars bars;
+  bars.res_full = bar0;
+  bars.full0 = bar0 + 8;
+  bars.empty0 = bars.full0 + 8 * C::kStages;
+  bars.st_full = bars.empty0 + 8 * C::kStages;
+  bars.p_full = bars.st_full + 8;
+  bars.acc_full = bars.p_full + 8;
+  bars.drain = bars.acc_full + 8;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
+  const int warp = threadIdx.x >> 5;
+  if (threadIdx.x == 0) {
+    mbar_init(bars.res_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(bars.full(s), 1);
+      mbar_init(bars.empty(s), 1);
+    }
+    mbar_init(bars.st_full, 1);
+    mbar_init(bars.p_full, 4);  // one arrival per row warp
+    mbar_init(bars.acc_full, 1);
+    mbar_init(bars.drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpLoad && (threadIdx.x & 31) == 0) {
+    tma_prefetch_desc(&tm.q);
+    tma_prefetch_desc(&tm.k);
+    tma_prefetch_desc(&tm.v);
+    tma_prefetch_desc(&tm.dout);
+  }
+  if (warp == kWarpIssue) {
+    tmem_alloc(smem_u32(tmem_holder), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const BwdItem it = bwd_item<kDQ>(p);
+  if (warp == kWarpLoad) {
+    bwd_load<D, kDQ>(p, tm, it, sbase, smem, bars, abort_flag);
+  } else if (warp == kWarpIssue) {
+    bwd_issue<D, kDQ>(p, it, sbase, tmem, bars, abort_flag);
+  } else if (warp >= kWarpRow0) {
+    bwd_rows<D, kDQ>(p, it, smem, tmem, bars, abort_flag);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kWarpIssue) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// delta[b, h, i] = sum_d dO[b, i, h, d] * O[b, i, h, d]: D/8 lanes per row, 16-byte loads.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16* __restrict__ o,
+                                                        const __nv_bfloat16* __restrict__ dout,
+                                                        float* __restrict__ delta, int B, int S, int H) {
+  constexpr int kLanes = D / 8;             // lanes per row
+  constexpr int kRowsPerWarp = 32 / kLanes;
+  const long long n_rows = (long long)B * S * H;
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / kLanes, l = lane % kLanes;
+  const long long warps = (long long)gridDim.x * (blockDim.x / 32);
+  for (long long w = (long long)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+       w * kRowsPerWarp < n_rows; w += warps) {
+    const long long rrow = w * kRowsPerWarp + sub;  // (b, s, h) in BSHD order
+    float acc = 0.f;
+    if (rrow < n_rows) {
+      const uint4 a = __ldcs(reinterpret_cast<const uint4*>(o + rrow * D) + l);
+      const uint4 g = __ldcs(reinterpret_cast<const uint4*>(dout + rrow * D) + l);
+      const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
+      const __nv_bfloat162* g2 = reinterpret_cast<const __nv_bfloat162*>(&g);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 x = __bfloat1622float2(a2[e]), y = __bfloat1622float2(g2[e]);
+        acc = fmaf(x.x, y.x, acc);
+        acc = fmaf(x.y, y.y, acc);
+      }
+    }
+#pragma unroll
+    for (int off = kLanes / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (rrow < n_rows && l == 0) {
+      const long long h = rrow % H, bs = rrow / H, s = bs % S, b = bs / S;
+      delta[(b * H + h) * S + s] = acc;
+    }
+  }
+}
+
+template <int D, bool kDQ>
+sp_status launch_bwd_one(const BwdMaps& tm, const BwdParams& p, int grid, cudaStream_t stream) {
+  using C = BCfg<D>;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SP_ERR_CUDA;
+  static bool attr_set[kMaxDevices] = {};
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(bwd_kernel<D, kDQ>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+      return SP_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  bwd_kernel<D, kDQ><<<grid, kBwdThreads, C::kSmemBytes, stream>>>(tm, p);
+  return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+}
+
+}  // namespace
+
+sp_status launch_attn_bwd(const BwdParams& p_in, const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, cudaStream_t stream) {
+  BwdParams p = p_in;
+  BwdMaps tm;
+  if (!encode_bshd_tmap(&tm.q, q, p.B, p.S, p.H, p.D) || !encode_bshd_tmap(&tm.k, k, p.B, p.S, p.H, p.D) ||
+      !encode_bshd_tmap(&tm.v, v, p.B, p.S, p.H, p.D) || !encode_bshd_tmap(&tm.dout, dout, p.B, p.S, p.H, p.D))
+    return SP_ERR_CUDA;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SP_ERR_CUDA;
+  const long long rows = (long long)p.B * p.S * p.H;
+  const int rows_per_block = 8 * (32 / (p.D / 8));
+  long long blocks = (rows + rows_per_block - 1) / rows_per_block;
+  const long long cap = (long long)num_sms(dev) * 8;
+  if (blocks > cap) blocks = cap;
+  if (p.D == 128)
+    bwd_delta_kernel<128><<<(int)blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                            static_cast<const __nv_bfloat16*>(dout), p.delta, p.B, p.S, p.H);
+  else
+    bwd_delta_kernel<64><<<(int)blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
+                                                           static_cast<const __nv_bfloat16*>(dout), p.delta, p.B, p.S, p.H);
+  if (cudaGetLastError() != cudaSuccess) return SP_ERR_CUDA;
+  const long long items = (long long)p.B * p.H * p.T;
+  if (items > 0x7fffffffLL) return SP_ERR_INVALID_ARG;
+  sp_status s = p.D == 128 ? launch_bwd_one<128, false>(tm, p, (int)items, stream)
+                           : launch_bwd_one<64, false>(tm, p, (int)items, stream);
+  if (s != SP_OK) return s;
+  return p.D == 128 ? launch_bwd_one<128, true>(tm, p, (int)items, stream)
+                    : launch_bwd_one<64, true>(tm, p, (int)items, stream);
+}
+
+}  // namespace spattn

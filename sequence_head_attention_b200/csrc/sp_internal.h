@@ -52,6 +52,22 @@ struct AttnParams {
   void* o_shard[kMaxShards];
 };
 
+// Parameters of the backward launches (all heads, all S queries and keys, optionally causal).
+struct BwdParams {
+  int B, S, H, D;
+  int T;              // ceil(S / 128)
+  int causal;
+  float scale_log2;   // log2(e) / sqrt(D)
+  float scale;        // 1 / sqrt(D)
+  const float* lse;   // forward lse [B, H, S], natural log
+  float* delta;       // [B, H, S] fp32 scratch: rowsum(dO * O)
+  void* dq;           // bf16 BSHD outputs
+  void* dk;
+  void* dv;
+  unsigned long long timeout_ns;
+  unsigned int* err;
+};
+
 // Device properties and driver entry points (cached per device).
 int num_sms(int device);
 bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, int D);
@@ -64,6 +80,8 @@ sp_status launch_attn(const AttnParams& p, const void* q, const void* k, const v
                       cudaStream_t stream);
 // As launch_attn, with Q, K, V (and O) given as the sequence shards in p (n_shards, shard_rows, *_shard).
 sp_status launch_attn_sharded(const AttnParams& p, cudaStream_t stream);
+sp_status launch_attn_bwd(const BwdParams& p, const void* q, const void* k, const void* v, const void* o,
+                          const void* dout, cudaStream_t stream);
 sp_status launch_merge(const float* const* o_parts, const float* const* lse_parts, int n, void* o,
                        float* lse, int o_f32, int B, int S, int H, int D, cudaStream_t stream);
 sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,

@@ -54,6 +54,8 @@ def lib() -> ctypes.CDLL:
                 "sp_head_to_seq_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_attn_fwd_seq_sharded": (I, [P, P, P, P, P, I, I, I, I, I, I, I, P, I, I, P]),
                 "sp_attn_fwd_items": (I, [P, P, P, P, P, I, I, I, I, P, I, I, P, P, Z, P]),
+                "sp_attn_bwd_workspace_bytes": (Z, [I, I, I, I]),
+                "sp_attn_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, P, Z, P]),
                 "sp_dbsp_unit_costs": (I, [P, I, I, I, P]),
                 "sp_dbsp_plan": (I, [P, I, I, I, P, P, P]),
                 "sp_dbsp_rank_items": (I, [P, P, I, I, I, I, P, I, P]),
@@ -319,6 +321,24 @@ def sp_attn_fwd_items(q, k, v, o, lse, items, causal=False, block_mask=None, wor
                                  _stream(stream))
     _check("sp_attn_fwd_items", st)
     return o, lse
+
+
+def sp_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal=False, workspace=None, stream=None):
+    """Gradients dq, dk, dv (bf16 [B,S,H,D]) of the attention for the upstream gradient dout, from the
+    forward's o and lse.  The fp32 delta workspace is allocated here with torch when none is given."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _bshd(t, n)
+    B, S, H, D = q.shape
+    _need(lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, S),
+          "lse must be contiguous fp32 [B, H, S]")
+    ws_bytes = lib().sp_attn_bwd_workspace_bytes(B, S, H, D)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    st = lib().sp_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq), _ptr(dk),
+                           _ptr(dv), B, S, H, D, int(bool(causal)), _ptr(workspace),
+                           workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("sp_attn_bwd", st)
+    return dq, dk, dv
 
 
 def sp_attn_fwd_sparse_noalloc(q, k, v, o, lse, block_mask, causal=False, stream=None):
