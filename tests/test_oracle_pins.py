@@ -388,6 +388,11 @@ MUTANTS = {
                             "const int src_rank = s % P, src_s = s / P, src_h = r * Hl + hh;"),
     "mask_tile_transposed": ("(size_t)(i / r->tile)) * r->n_tiles + (size_t)(j / r->tile)",
                              "(size_t)(j / r->tile)) * r->n_tiles + (size_t)(i / r->tile)"),
+    "bwd_drops_delta": ("const double ds = p[j] * (dp - delta);", "const double ds = p[j] * dp;"),
+    "bwd_dk_unscaled": ("J->dk[IDX(k, j, d)] += ds * J->q[IDX(q, i, d)] * scale;",
+                        "J->dk[IDX(k, j, d)] += ds * J->q[IDX(q, i, d)];"),
+    "bwd_dv_wrong_row": ("J->dv[IDX(v, j, d)] += p[j] * J->dout[IDX(dout, i, d)];",
+                         "J->dv[IDX(v, j, d)] += p[j] * J->dout[IDX(dout, j, d)];"),
 }
 
 
@@ -418,6 +423,22 @@ def _pins_pass(lib):
     outs = oracle.seq_to_head([x[:, :4].copy(), x[:, 4:].copy()], 4, lib=lib)
     if not (np.array_equal(outs[0], x[:, :, :2]) and np.array_equal(outs[1], x[:, :, 2:])):
         return False
+    # backward: gradients against central differences of the forward (through the same library)
+    qs, ks, vs, dos = (g.standard_normal((1, 4, 1, 3)) for _ in range(4))
+    for causal in (False, True):
+        grads = oracle.attention_bwd(qs, ks, vs, dos, causal=causal, lib=lib)
+        for which in range(3):
+            base = [qs, ks, vs]
+            num = np.zeros_like(base[which])
+            for idx in np.ndindex(num.shape):
+                hi, lo = [t.copy() for t in base], [t.copy() for t in base]
+                hi[which][idx] += 1e-6
+                lo[which][idx] -= 1e-6
+                lh = (dos * oracle.attention(*hi, causal=causal, lib=lib)[0]).sum()
+                ll = (dos * oracle.attention(*lo, causal=causal, lib=lib)[0]).sum()
+                num[idx] = (lh - ll) / 2e-6
+            if np.max(np.abs(num - grads[which])) > 1e-6:
+                return False
     return True
 
 
