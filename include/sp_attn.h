@@ -154,6 +154,23 @@ SP_API sp_status sp_attn_bwd(const void* q, const void* k, const void* v, const 
                              void* workspace, size_t workspace_bytes, sp_stream stream);
 
 /*
+ * The backward of one KV block [kv_begin, kv_end) of a ring ("CHARM+ ...", abstract: the backward of the
+ * Ring-Attention scheme; "CHARM+: How Cross-Hardware Attention ...", Ring-Attention paragraph: one KV block
+ * per round).  With o and lse the merged result over all blocks (sp_merge_partials), the gradients split
+ * by block: this call writes dk and dv for the block's keys (rows [kv_begin, kv_end), other rows untouched)
+ * and ADDS the block's contribution to dq into dq_acc (device fp32 [B,S,H,D], zeroed by the caller before
+ * the first block); after every block, dq_acc holds dq (convert with sp_convert_f32_to_bf16).
+ * kv_begin must be a multiple of 128; 0 <= kv_begin < kv_end <= S.  Other arguments as sp_attn_bwd.
+ */
+SP_API sp_status sp_attn_bwd_partial(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                                     const float* lse, float* dq_acc, void* dk, void* dv, int B, int S, int H,
+                                     int D, int kv_begin, int kv_end, int causal, void* workspace,
+                                     size_t workspace_bytes, sp_stream stream);
+
+/* out[i] = in[i] rounded to bf16 (nearest even), n a multiple of 4; in 16-byte and out 8-byte aligned. */
+SP_API sp_status sp_convert_f32_to_bf16(const float* in, void* out, long long n, sp_stream stream);
+
+/*
  * Ulysses relayout, sequence shards -> head shards, between P buffers of one GPU:
  *   in_ranks[r]  device [B, S/P, H, D]   (rank r's slice of the sequence, all heads)
  *   out_ranks[r] device [B, S, H/P, D]   (all positions of heads [r*H/P, (r+1)*H/P))

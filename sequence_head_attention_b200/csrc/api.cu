@@ -511,10 +511,75 @@ sp_status sp_attn_bwd(const void* q, const void* k, const void* v, const void* o
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
+  p.dq_acc = nullptr;
+  p.kv_begin = 0;
+  p.kv_end = S;
+  p.kt0 = 0;
+  p.n_kt = p.T;
   p.timeout_ns = g_timeout_ns;
   p.err = device_error_word();
   if (!p.err) return SP_ERR_CUDA;
   return launch_attn_bwd(p, q, k, v, o, dout, as_stream(stream));
+}
+
+sp_status sp_attn_bwd_partial(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                              const float* lse, float* dq_acc, void* dk, void* dv, int B, int S, int H, int D,
+                              int kv_begin, int kv_end, int causal, void* workspace, size_t workspace_bytes,
+                              sp_stream stream) {
+  if (!sizes_ok(B, S, H, D)) return SP_ERR_INVALID_ARG;
+  if (kv_begin < 0 || kv_end <= kv_begin || kv_end > S || kv_begin % SP_TILE != 0) return SP_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o || !dout || !lse || !dq_acc || !dk || !dv || !workspace) return SP_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, dout, (const void*)lse, (const void*)dq_acc, (const void*)dk,
+                          (const void*)dv, (const void*)workspace})
+    if (!aligned16(ptr)) return SP_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SP_ERR_INVALID_ARG;
+  if (workspace_bytes < sp_attn_bwd_workspace_bytes(B, S, H, D)) return SP_ERR_INVALID_ARG;
+  const size_t tb = (size_t)B * S * H * D * 2;
+  const size_t lb = (size_t)B * H * S * 4;
+  struct Span { const void* p; size_t n; };
+  const Span ins[] = {{q, tb}, {k, tb}, {v, tb}, {o, tb}, {dout, tb}, {lse, lb}, {workspace, lb}};
+  const Span outs[] = {{dq_acc, 2 * tb}, {dk, tb}, {dv, tb}};
+  auto overlap = [](const Span& x, const Span& y) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(x.p), b0 = reinterpret_cast<uintptr_t>(y.p);
+    return a0 < b0 + y.n && b0 < a0 + x.n;
+  };
+  for (int i = 0; i < 3; ++i) {
+    for (const Span& in : ins)
+      if (overlap(outs[i], in)) return SP_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlap(outs[i], outs[j])) return SP_ERR_INVALID_ARG;
+  }
+  BwdParams p{};
+  p.B = B;
+  p.S = S;
+  p.H = H;
+  p.D = D;
+  p.T = (S + SP_TILE - 1) / SP_TILE;
+  p.causal = causal;
+  p.scale_log2 = (float)(1.4426950408889634 / std::sqrt((double)D));
+  p.scale = (float)(1.0 / std::sqrt((double)D));
+  p.lse = lse;
+  p.delta = static_cast<float*>(workspace);
+  p.dq = nullptr;
+  p.dk = dk;
+  p.dv = dv;
+  p.dq_acc = dq_acc;
+  p.kv_begin = kv_begin;
+  p.kv_end = kv_end;
+  p.kt0 = kv_begin / SP_TILE;
+  p.n_kt = (kv_end - kv_begin + SP_TILE - 1) / SP_TILE;
+  p.timeout_ns = g_timeout_ns;
+  p.err = device_error_word();
+  if (!p.err) return SP_ERR_CUDA;
+  return launch_attn_bwd(p, q, k, v, o, dout, as_stream(stream));
+}
+
+sp_status sp_convert_f32_to_bf16(const float* in, void* out, long long n, sp_stream stream) {
+  if (n < 0 || (n > 0 && (!in || !out)) || n % 4 != 0) return SP_ERR_INVALID_ARG;
+  if (!aligned16(in) || ((reinterpret_cast<uintptr_t>(out) & 7u) != 0)) return SP_ERR_INVALID_ARG;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(in), b0 = reinterpret_cast<uintptr_t>(out);
+  if (n > 0 && a0 < b0 + (size_t)n * 2 && b0 < a0 + (size_t)n * 4) return SP_ERR_INVALID_ARG;
+  return launch_f32_to_bf16(in, out, n, as_stream(stream));
 }
 
 sp_status sp_seq_to_head_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,

@@ -77,13 +77,17 @@ template <bool kDQ>
 __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p) {
   BwdItem it;
   const int w = blockIdx.x;
-  it.b = w / (p.H * p.T);
-  it.h = (w / p.T) % p.H;
-  it.tile = w % p.T;
-  if (kDQ) {  // key tiles 0 .. (causal: the query tile's own)
-    it.first = 0;
-    it.n_steps = p.causal ? it.tile + 1 : p.T;
-  } else {    // query tiles (causal: from the key tile's own) .. T-1
+  if (kDQ) {  // every query tile; key tiles of the range, up to (causal) the query tile's own
+    it.b = w / (p.H * p.T);
+    it.h = (w / p.T) % p.H;
+    it.tile = w % p.T;
+    it.first = p.kt0;
+    const int last = p.causal ? min(p.kt0 + p.n_kt, it.tile + 1) : p.kt0 + p.n_kt;  // exclusive
+    it.n_steps = max(0, last - it.first);
+  } else {    // the range's key tiles; query tiles (causal: from the key tile's own) .. T-1
+    it.b = w / (p.H * p.n_kt);
+    it.h = (w / p.n_kt) % p.H;
+    it.tile = p.kt0 + w % p.n_kt;
     it.first = p.causal ? it.tile : 0;
     it.n_steps = p.T - it.first;
   }
@@ -238,6 +242,9 @@ __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, u
   const uint64_t tmo = p.timeout_ns;
   const float sl2 = p.scale_log2;
   const int row = it.tile * kBT + r;                             // global position of this thread's row
+  const int kv_lim = min(p.kv_end, p.S);
+  // rows this CTA writes: queries < S (dQ); keys of the range (dK, dV)
+  const bool row_out = kDQ ? row < p.S : row < kv_lim;
   float lse2_row = 0.f, dlt_row = 0.f;
   if (kDQ && row < p.S) {
     const size_t i = ((size_t)it.b * p.H + it.h) * p.S + row;
@@ -282,7 +289,7 @@ __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, u
           float pv;
           if (kDQ) {
             pv = ex2_approx(sv * sl2 - lse2_row);
-            if (p.causal && t * kBT + c > row) pv = 0.f;  // key after the query
+            if ((p.causal && t * kBT + c > row) || t * kBT + c >= kv_lim) pv = 0.f;  // key after the query, or outside the range
             ds[u] = pv * (dv - dlt_row);
           } else {
             pv = ex2_approx(sv * sl2 - lse2[c]);
@@ -306,6 +313,7 @@ __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, u
   if (!ok) return;
   ok = __all_sync(0xffffffffu, mbar_wait(bars.acc_full, 0, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err));
   if (!ok) return;
+  if (it.n_steps == 0) return;  // (dQ of a key range before this query tile) nothing accumulated
   tc_fence_after();
   const float scale = p.scale;
   const size_t out = (((size_t)it.b * p.S + row) * p.H + it.h) * D;
@@ -320,7 +328,20 @@ __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, u
       uint32_t a[32];
       tmem_ld32(tacc + c * 32, a);
       tmem_wait_ld();
-      if (row < p.S) {
+      if (kDQ && p.dq_acc) {  // add this key range's contribution to the fp32 accumulator
+        if (row_out) {
+          float4* d4 = reinterpret_cast<float4*>(p.dq_acc + out + c * 32);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            float4 x = d4[e];
+            x.x += __uint_as_float(a[4 * e]) * f;
+            x.y += __uint_as_float(a[4 * e + 1]) * f;
+            x.z += __uint_as_float(a[4 * e + 2]) * f;
+            x.w += __uint_as_float(a[4 * e + 3]) * f;
+            d4[e] = x;
+          }
+        }
+      } else if (row_out) {
         uint4* d4 = reinterpret_cast<uint4*>(dst + out + c * 32);
 #pragma unroll
         for (int e = 0; e < 4; ++e)
@@ -431,6 +452,14 @@ __global__ void __launch_bounds__(256) bwd_delta_kernel(const __nv_bfloat16* __r
   }
 }
 
+__global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restrict__ in, uint2* __restrict__ out,
+                                                          long long n4) {
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4; i += (long long)gridDim.x * blockDim.x) {
+    const float4 x = __ldcs(in + i);
+    out[i] = make_uint2(pack_bf16x2(x.x, x.y), pack_bf16x2(x.z, x.w));
+  }
+}
+
 template <int D, bool kDQ>
 sp_status launch_bwd_one(const BwdMaps& tm, const BwdParams& p, int grid, cudaStream_t stream) {
   using C = BCfg<D>;
@@ -470,13 +499,29 @@ sp_status launch_attn_bwd(const BwdParams& p_in, const void* q, const void* k, c
     bwd_delta_kernel<64><<<(int)blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(o),
                                                            static_cast<const __nv_bfloat16*>(dout), p.delta, p.B, p.S, p.H);
   if (cudaGetLastError() != cudaSuccess) return SP_ERR_CUDA;
-  const long long items = (long long)p.B * p.H * p.T;
-  if (items > 0x7fffffffLL) return SP_ERR_INVALID_ARG;
-  sp_status s = p.D == 128 ? launch_bwd_one<128, false>(tm, p, (int)items, stream)
-                           : launch_bwd_one<64, false>(tm, p, (int)items, stream);
-  if (s != SP_OK) return s;
-  return p.D == 128 ? launch_bwd_one<128, true>(tm, p, (int)items, stream)
-                    : launch_bwd_one<64, true>(tm, p, (int)items, stream);
+  const long long items_kv = (long long)p.B * p.H * p.n_kt;  // dK/dV: the range's key tiles
+  const long long items_q = (long long)p.B * p.H * p.T;      // dQ: every query tile
+  if (items_q > 0x7fffffffLL) return SP_ERR_INVALID_ARG;
+  if (items_kv > 0) {
+    sp_status s = p.D == 128 ? launch_bwd_one<128, false>(tm, p, (int)items_kv, stream)
+                             : launch_bwd_one<64, false>(tm, p, (int)items_kv, stream);
+    if (s != SP_OK) return s;
+  }
+  return p.D == 128 ? launch_bwd_one<128, true>(tm, p, (int)items_q, stream)
+                    : launch_bwd_one<64, true>(tm, p, (int)items_q, stream);
+}
+
+sp_status launch_f32_to_bf16(const float* in, void* out, long long n, cudaStream_t stream) {
+  if (n <= 0) return SP_OK;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SP_ERR_CUDA;
+  const long long n4 = n / 4;
+  long long blocks = (n4 + 255) / 256;
+  const long long cap = (long long)num_sms(dev) * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  f32_to_bf16_kernel<<<(int)blocks, 256, 0, stream>>>(reinterpret_cast<const float4*>(in), static_cast<uint2*>(out), n4);
+  return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
 }
 
 }  // namespace spattn

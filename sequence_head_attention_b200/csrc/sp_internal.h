@@ -64,6 +64,10 @@ struct BwdParams {
   void* dq;           // bf16 BSHD outputs
   void* dk;
   void* dv;
+  float* dq_acc;      // non-null: dq is not written; this launch's dQ contribution is added here (fp32 BSHD)
+  int kv_begin;       // keys [kv_begin, kv_end) only (one KV block of a ring); kv_begin a multiple of 128
+  int kv_end;
+  int kt0, n_kt;      // their key tiles: kt0 .. kt0 + n_kt - 1
   unsigned long long timeout_ns;
   unsigned int* err;
 };
@@ -82,6 +86,7 @@ sp_status launch_attn(const AttnParams& p, const void* q, const void* k, const v
 sp_status launch_attn_sharded(const AttnParams& p, cudaStream_t stream);
 sp_status launch_attn_bwd(const BwdParams& p, const void* q, const void* k, const void* v, const void* o,
                           const void* dout, cudaStream_t stream);
+sp_status launch_f32_to_bf16(const float* in, void* out, long long n, cudaStream_t stream);  // n % 4 == 0
 sp_status launch_merge(const float* const* o_parts, const float* const* lse_parts, int n, void* o,
                        float* lse, int o_f32, int B, int S, int H, int D, cudaStream_t stream);
 sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,

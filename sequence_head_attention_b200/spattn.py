@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
                 "sp_attn_fwd_items": (I, [P, P, P, P, P, I, I, I, I, P, I, I, P, P, Z, P]),
                 "sp_attn_bwd_workspace_bytes": (Z, [I, I, I, I]),
                 "sp_attn_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, P, Z, P]),
+                "sp_attn_bwd_partial": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, P, Z, P]),
+                "sp_convert_f32_to_bf16": (I, [P, P, ctypes.c_longlong, P]),
                 "sp_dbsp_unit_costs": (I, [P, I, I, I, P]),
                 "sp_dbsp_plan": (I, [P, I, I, I, P, P, P]),
                 "sp_dbsp_rank_items": (I, [P, P, I, I, I, I, P, I, P]),
@@ -339,6 +341,34 @@ def sp_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, causal=False, workspace=None,
                            workspace.numel() * workspace.element_size(), _stream(stream))
     _check("sp_attn_bwd", st)
     return dq, dk, dv
+
+
+def sp_attn_bwd_partial(q, k, v, o, dout, lse, dq_acc, dk, dv, kv_begin, kv_end, causal=False, workspace=None,
+                        stream=None):
+    """Backward of one KV block [kv_begin, kv_end) (o, lse: the merged forward result): writes dk, dv rows
+    of the block and adds its dq contribution into dq_acc (fp32 [B,S,H,D])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dk, "dk"), (dv, "dv")):
+        _bshd(t, n)
+    _bshd(dq_acc, "dq_acc", torch.float32)
+    B, S, H, D = q.shape
+    _need(lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, S),
+          "lse must be contiguous fp32 [B, H, S]")
+    ws_bytes = lib().sp_attn_bwd_workspace_bytes(B, S, H, D)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 1), dtype=torch.uint8, device=q.device)
+    st = lib().sp_attn_bwd_partial(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(dout), _ptr(lse), _ptr(dq_acc), _ptr(dk),
+                                   _ptr(dv), B, S, H, D, int(kv_begin), int(kv_end), int(bool(causal)),
+                                   _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream))
+    _check("sp_attn_bwd_partial", st)
+    return dq_acc, dk, dv
+
+
+def sp_convert_f32_to_bf16(x, out, stream=None):
+    """out (bf16) = x (fp32) rounded to nearest even; same number of elements, a multiple of 4."""
+    _need(x.dtype == torch.float32 and out.dtype == torch.bfloat16 and x.numel() == out.numel(), "f32 in, bf16 out")
+    _need(x.is_contiguous() and out.is_contiguous(), "contiguous tensors")
+    _check("sp_convert_f32_to_bf16", lib().sp_convert_f32_to_bf16(_ptr(x), _ptr(out), x.numel(), _stream(stream)))
+    return out
 
 
 def sp_attn_fwd_sparse_noalloc(q, k, v, o, lse, block_mask, causal=False, stream=None):

@@ -65,3 +65,41 @@ def test_bwd_deterministic():
     b = run_bwd(q, k, v, do, True)
     for x, y in zip(a, b):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_ring_block_backward_sums_to_full(causal):
+    """KV blocks [0,256), [256,512), [512,768), [768,1000) with the merged forward result: each block's dk and
+    dv rows equal the full backward's bit for bit (same per-key-tile arithmetic), and the fp32 sum of the
+    blocks' dq contributions matches the oracle and the full backward's dq."""
+    B, S, H, D = 1, 1000, 2, 128
+    q, k, v = synth.qkv(B, S, H, D, seed=41, scale=0.5)
+    do = torch.randn((B, S, H, D), generator=torch.Generator().manual_seed(42)).to(torch.bfloat16)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, H, S), device="cuda")
+    spattn.sp_attn_fwd(qd, kd, vd, o, lse, n_kv_blocks=4, causal=causal)  # KV blocks + merge, as in a ring
+    full = [torch.empty_like(qd) for _ in range(3)]
+    spattn.sp_attn_bwd(qd, kd, vd, o, dod, lse, *full, causal=causal)
+    dq_acc = torch.zeros((B, S, H, D), dtype=torch.float32, device="cuda")
+    dk = torch.full_like(qd, float("nan"))
+    dv = torch.full_like(qd, float("nan"))
+    for a, e in ((0, 256), (256, 512), (512, 768), (768, 1000)):
+        spattn.sp_attn_bwd_partial(qd, kd, vd, o, dod, lse, dq_acc, dk, dv, a, e, causal=causal)
+    dq = spattn.sp_convert_f32_to_bf16(dq_acc, torch.empty_like(qd))
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    assert torch.equal(dk, full[1]) and torch.equal(dv, full[2])
+    rq, rk, rv = oracle.attention_bwd(to64(q), to64(k), to64(v), to64(do), causal=causal)
+    close(dq, rq, "dq")
+    close(dk, rk, "dk")
+    close(dv, rv, "dv")
+    close(dq, to64(full[0]), "dq vs full")
+
+
+def test_partial_backward_rejects_unaligned_block():
+    q = torch.zeros((1, 512, 1, 64), dtype=torch.bfloat16, device="cuda")
+    lse = torch.zeros((1, 1, 512), device="cuda")
+    acc = torch.zeros((1, 512, 1, 64), device="cuda")
+    with pytest.raises(spattn.SpError):
+        spattn.sp_attn_bwd_partial(q, q, q, q, q, lse, acc, torch.empty_like(q), torch.empty_like(q), 100, 300)
