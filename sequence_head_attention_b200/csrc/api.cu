@@ -129,7 +129,7 @@ unsigned int* device_error_word() {
   return g_err_addr[dev];
 }
 
-bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, int D) {
+bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, int D, int box_rows) {
   {
     std::lock_guard<std::mutex> lk(g_mu);
     if (!g_encode) {
@@ -142,10 +142,11 @@ bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, i
     }
   }
   // Dimensions innermost first: d, h, s, b.  Box: 64 head-dim elements (128 bytes, the swizzle span)
-  // of one head, 128 positions, one batch.  Rows past S read as zero.
+  // of one head, box_rows positions (128, or 64 for a CTA pair's half of a key tile), one batch.  Rows
+  // past S read as zero.
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)S, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)S * H * D * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box,
                         estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

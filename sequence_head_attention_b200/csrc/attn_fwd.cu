@@ -30,6 +30,7 @@
 #include <atomic>
 #include <climits>
 #include <cstdint>
+#include <cstdlib>
 
 #include "sp_internal.h"
 #include "sp_ptx.cuh"
@@ -61,22 +62,28 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and l are rescaled w
 #endif
 constexpr int kPolyPairs = SP_EXP2_POLY_PAIRS;
 
-template <int D>
+template <int D, bool kPair = false>
 struct Cfg {
   static constexpr int kSub = D / 64;                   // 64-column (128-byte) sub-tiles per row
   static constexpr int kTileBytes = kTile * D * 2;      // one 128 x D bf16 tile
-  static constexpr int kStages = D == 128 ? 4 : 8;      // K/V ring slots
+  // A K or V slot: a whole tile, or for a CTA pair this CTA's half (K: 64 of the 128 keys; V: 64 of the D
+  // columns), the MMA's B operand being split by N between the two SMs.
+  static constexpr int kKVBytes = kPair ? kTileBytes / 2 : kTileBytes;
+  static constexpr int kKSubBytes = kPair ? 8192 : 16384;  // between the 64-column sub-tiles of a K slot
+  static constexpr int kStages = kPair ? 8 : (D == 128 ? 4 : 8);  // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
-  static constexpr int kBarOff = kKVOff + kStages * kTileBytes;
+  static constexpr int kBarOff = kKVOff + kStages * kKVBytes;
   // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2], drain, and
   // 8-byte slots for the o_done[2] counters
   static constexpr int kNumBars = 2 + 2 * kStages + 9;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // misc: TMEM base, abort flag, published-item count, per-warp item-read counts, the item ring
   static constexpr int kSmemBytes = kMiscOff + 96 + 1024;  // + alignment slack
-  static constexpr uint32_t kIdescS = idesc_bf16_f32(128, 128, false, false);
-  static constexpr uint32_t kIdescPV = idesc_bf16_f32(128, D, false, true);
+  static constexpr int kM = kPair ? 256 : 128;  // MMA rows: a pair computes both CTAs' 128 rows at once
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(kM, 128, false, false);
+  static constexpr uint32_t kIdescPV = idesc_bf16_f32(kM, D, false, true);
+  static constexpr uint32_t kRowWarps = kPair ? 8u : 4u;  // softmax warps per lane over the (pair of) CTAs
   static constexpr uint32_t kColS = 0;
   static constexpr uint32_t kColO = 256;
 };
@@ -100,8 +107,13 @@ struct Item {
   int q_end;       // one past the last row of the shard (rows from here on belong to the next shard)
   bool valid[2];
   bool id_ok;      // false: the item list named an item that does not exist
+  // What the MMAs walk: for a CTA pair, lane t covers this CTA's tile and the other CTA's tile t; the key
+  // tiles are those either needs (equal to the fields above for a single CTA).
+  int q_last_u[2];
+  bool valid_u[2];
 };
 
+template <bool kPair = false>
 __device__ __forceinline__ Item decode_item(const AttnParams& p, int w) {
   bool id_ok = true;
   if (p.item_list) {  // an explicit list: ids of the one-chunk layout, query-tile pair as given
@@ -124,19 +136,35 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p, int w) {
   const int qq = r2 % p.n_qpairs;
   it.qp = (p.causal && !p.item_list) ? (p.n_qpairs - 1 - qq) : qq;
   // Query tiles are laid on each shard's own 128-row grid (one shard: the global grid); a shard's last
-  // tile may be short, and pairs never cross shards.
+  // tile may be short, and items never cross shards.  An item is a pair of tiles, or for a CTA pair four:
+  // rank r of the pair takes tiles 4u + 2r and 4u + 2r + 1 of its unit u.
   it.shard = it.qp / p.pairs_per_shard;
   const int lp = it.qp - it.shard * p.pairs_per_shard;
   it.q_end = min(p.S, (it.shard + 1) * p.shard_rows);
+  const int rk = kPair ? (int)cluster_rank() : 0;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const int lt = 2 * lp + t;
-    it.q_start[t] = it.shard * p.shard_rows + lt * kTile;
-    it.valid[t] = lt < p.tiles_per_shard && it.q_start[t] < it.q_end;
-    it.q_last[t] = min(it.q_end, it.q_start[t] + kTile) - 1;
+    it.valid_u[t] = false;
+    it.q_last_u[t] = -1;
+#pragma unroll
+    for (int rr = 0; rr < (kPair ? 2 : 1); ++rr) {
+      const int lt = kPair ? 4 * lp + 2 * rr + t : 2 * lp + t;
+      const int start = it.shard * p.shard_rows + lt * kTile;
+      const bool valid = lt < p.tiles_per_shard && start < it.q_end;
+      const int last = min(it.q_end, start + kTile) - 1;
+      if (rr == rk) {
+        it.q_start[t] = start;
+        it.valid[t] = valid;
+        it.q_last[t] = last;
+      }
+      if (valid) {
+        it.valid_u[t] = true;
+        it.q_last_u[t] = max(it.q_last_u[t], last);
+      }
+    }
   }
   it.id_ok = id_ok;
-  if (!id_ok) it.valid[0] = it.valid[1] = false;  // nothing computed, nothing written
+  if (!id_ok) it.valid[0] = it.valid[1] = it.valid_u[0] = it.valid_u[1] = false;  // nothing computed or written
   return it;
 }
 
@@ -167,10 +195,10 @@ struct StepIter {
   __device__ __forceinline__ void init(const AttnParams& p, const Item& it) {
     causal = p.causal != 0;
     kv_begin = p.kv_begin;
-    q_last0 = it.q_last[0];
-    q_last1 = it.q_last[1];
-    v0 = it.valid[0];
-    v1 = it.valid[1];
+    q_last0 = it.q_last_u[0];
+    q_last1 = it.q_last_u[1];
+    v0 = it.valid_u[0];
+    v1 = it.valid_u[1];
     sparse = p.row_ptr != nullptr;
     sharded = p.n_shards > 1;
     shard_rows = p.shard_rows;
@@ -282,46 +310,58 @@ struct TMaps {
   CUtensorMap q[kMaxShards];
   CUtensorMap k[kMaxShards];
   CUtensorMap v[kMaxShards];
+  CUtensorMap k64[kMaxShards];  // K with 64-row boxes: a CTA pair's halves of a key tile
 };
 
 // ------------------------------------------------------------------------------------------------
 // Producer: one warp walks the work in lockstep (all values warp-uniform); one elected lane issues the
 // TMA loads.
 // ------------------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool kPair>
 __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem, const Bars& bars,
                              const ItemRing& ir, volatile int* abort_flag) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kPair>;
   const uint32_t sbase = smem_u32(smem);
   const uint64_t tmo = p.timeout_ns;
+  // A CTA pair: each CTA loads its own query tiles and its half of every K/V tile, and the bytes complete
+  // on rank 0's barriers (whose MMA consumes both halves); only rank 0 arms them.
+  const uint32_t rk = kPair ? cluster_rank() : 0u;
+  const uint32_t q_full_bar = kPair ? map_shared(bars.q_full, 0) : bars.q_full;
   uint32_t q_empty_ph = 0;
   int ring = 0;
   int n_item = 0;
   int last_q_item = -1;
   bool ok = true;
-  int w = blockIdx.x;
+  int w = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   for (;; ++n_item) {
-    if (n_item > 0) {  // claim the next item
-      int claimed = 0;
-      if (elect_one_sync()) claimed = (int)gridDim.x + (int)atomicAdd(p.sched, 1u);
-      w = __shfl_sync(0xffffffffu, claimed, __ffs(__ballot_sync(0xffffffffu, claimed != 0)) - 1);
-    }
-    const bool done = w >= p.n_items;
-    // publish it (the slot's previous item must have been read by every softmax warp)
-    if (n_item >= kItemRing) {
-      const uint32_t need = (uint32_t)(n_item - kItemRing + 1);
+    bool done;
+    if constexpr (kPair) {  // a pair walks its units in a fixed stride
+      if (n_item > 0) w += (int)(gridDim.x >> 1);
+      done = w >= p.n_items;
+      if (done) break;
+    } else {
+      if (n_item > 0) {  // claim the next item
+        int claimed = 0;
+        if (elect_one_sync()) claimed = (int)gridDim.x + (int)atomicAdd(p.sched, 1u);
+        w = __shfl_sync(0xffffffffu, claimed, __ffs(__ballot_sync(0xffffffffu, claimed != 0)) - 1);
+      }
+      done = w >= p.n_items;
+      // publish it (the slot's previous item must have been read by every softmax warp)
+      if (n_item >= kItemRing) {
+        const uint32_t need = (uint32_t)(n_item - kItemRing + 1);
 #pragma unroll 1
-      for (int k = 0; k < 8 && ok; ++k)
-        ok = warp_counter_wait(ir.used0 + 4u * k, need, tmo, ERR_TIMEOUT_ITEM_FREE, abort_flag, p.err);
-      if (!ok) break;
+        for (int k = 0; k < 8 && ok; ++k)
+          ok = warp_counter_wait(ir.used0 + 4u * k, need, tmo, ERR_TIMEOUT_ITEM_FREE, abort_flag, p.err);
+        if (!ok) break;
+      }
+      if (elect_one_sync()) {
+        ir.ids[n_item % kItemRing] = done ? -1 : w;
+        smem_counter_add_release(ir.pub, 1u);
+      }
+      __syncwarp();
+      if (done) break;
     }
-    if (elect_one_sync()) {
-      ir.ids[n_item % kItemRing] = done ? -1 : w;
-      smem_counter_add_release(ir.pub, 1u);
-    }
-    __syncwarp();
-    if (done) break;
-    const Item it = decode_item(p, w);
+    const Item it = decode_item<kPair>(p, w);
     if (!it.id_ok && elect_one_sync()) atomicOr(p.err, ERR_BAD_ITEM);
     if (n_item > 0) {
       ok = warp_mbar_wait(bars.q_empty, q_empty_ph, tmo, ERR_TIMEOUT_Q_EMPTY, abort_flag, p.err);
@@ -329,14 +369,18 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
       if (!ok) break;
     }
     if (elect_one_sync()) {
-      const int y0 = it.shard * p.shard_rows;  // the pair's shard starts at this global row
-      mbar_arrive_expect_tx(bars.q_full, 2 * C::kTileBytes);
+      const int y0 = it.shard * p.shard_rows;  // the item's shard starts at this global row
+      if (rk == 0) mbar_arrive_expect_tx(bars.q_full, (kPair ? 4 : 2) * C::kTileBytes);
 #pragma unroll
       for (int t = 0; t < 2; ++t)
 #pragma unroll
-        for (int c = 0; c < C::kSub; ++c)
-          tma_load_4d(sbase + C::kQOff + t * C::kTileBytes + c * 16384, &tm.q[it.shard], bars.q_full, 64 * c, it.h,
-                      it.q_start[t] - y0, it.b);
+        for (int c = 0; c < C::kSub; ++c) {
+          const uint32_t dst = sbase + C::kQOff + t * C::kTileBytes + c * 16384;
+          if constexpr (kPair)
+            tma_load_4d_pair(dst, &tm.q[it.shard], q_full_bar, 64 * c, it.h, it.q_start[t] - y0, it.b);
+          else
+            tma_load_4d(dst, &tm.q[it.shard], bars.q_full, 64 * c, it.h, it.q_start[t] - y0, it.b);
+        }
     }
     __syncwarp();
     last_q_item = n_item;
@@ -354,12 +398,25 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
           if (!ok) break;
         }
         if (elect_one_sync()) {
-          mbar_arrive_expect_tx(bars.kv_full(slot), C::kTileBytes);
-          const CUtensorMap* map = kv == 0 ? &tm.k[st.shard] : &tm.v[st.shard];
+          const uint32_t dst = sbase + C::kKVOff + slot * C::kKVBytes;
+          const int y = kv_start - st.shard * p.shard_rows;
+          if constexpr (kPair) {
+            const uint32_t bar = map_shared(bars.kv_full(slot), 0);
+            if (rk == 0) mbar_arrive_expect_tx(bars.kv_full(slot), 2 * C::kKVBytes);
+            if (kv == 0) {  // keys [64 rk, 64 rk + 64) of the tile, all D columns
 #pragma unroll
-          for (int c = 0; c < C::kSub; ++c)
-            tma_load_4d(sbase + C::kKVOff + slot * C::kTileBytes + c * 16384, map, bars.kv_full(slot), 64 * c,
-                        it.h, kv_start - st.shard * p.shard_rows, it.b);
+              for (int c = 0; c < C::kSub; ++c)
+                tma_load_4d_pair(dst + c * C::kKSubBytes, &tm.k64[st.shard], bar, 64 * c, it.h, y + 64 * (int)rk, it.b);
+            } else {        // all 128 keys, columns [64 rk, 64 rk + 64)
+              tma_load_4d_pair(dst, &tm.v[st.shard], bar, 64 * (int)rk, it.h, y, it.b);
+            }
+          } else {
+            mbar_arrive_expect_tx(bars.kv_full(slot), C::kKVBytes);
+            const CUtensorMap* map = kv == 0 ? &tm.k[st.shard] : &tm.v[st.shard];
+#pragma unroll
+            for (int c = 0; c < C::kSub; ++c)
+              tma_load_4d(dst + c * 16384, map, bars.kv_full(slot), 64 * c, it.h, y, it.b);
+          }
         }
         __syncwarp();
         ++ring;
@@ -368,10 +425,18 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
   }
   if (*abort_flag) {
     // Do not leave copies in flight into shared memory: wait (bounded) for the most recent load of
-    // every slot and for the last Q load.
-    for (int pos = max(0, ring - C::kStages); pos < ring; ++pos)
-      warp_mbar_wait(bars.kv_full(pos % C::kStages), (pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, nullptr, p.err);
-    if (last_q_item >= 0) warp_mbar_wait(bars.q_full, last_q_item & 1, tmo, ERR_TIMEOUT_Q_FULL, nullptr, p.err);
+    // every slot and for the last Q load.  A pair's rank 1 cannot observe its own loads (their bytes
+    // complete on rank 0's barriers): it waits out a fixed interval far longer than a load.
+    if (kPair && rk != 0) {
+      const uint64_t t0 = global_timer_ns();
+      while (global_timer_ns() - t0 < 200000ull) {
+      }
+    } else {
+      for (int pos = max(0, ring - C::kStages); pos < ring; ++pos)
+        warp_mbar_wait(bars.kv_full(pos % C::kStages), (pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, nullptr,
+                       p.err);
+      if (last_q_item >= 0) warp_mbar_wait(bars.q_full, last_q_item & 1, tmo, ERR_TIMEOUT_Q_FULL, nullptr, p.err);
+    }
   }
 }
 
@@ -382,14 +447,15 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
 // core interleaves the two lanes.  Shared K/V slots and the Q buffer are released when both lanes are
 // done with them (the "empty" barriers count two arrivals; a lane that skips a tile arrives directly).
 // ------------------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool kPair>
 __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, const ItemRing& ir, uint32_t tmem_in,
                         int t, volatile int* abort_flag) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kPair>;
   const uint32_t sbase = smem_u32(smem);
   const uint64_t tmo = p.timeout_ns;
   const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_in, 0);  // provably warp-uniform
-  // Descriptors of K-step 0; later K-steps add their byte offset / 16 to the start-address field.
+  // Descriptors of K-step 0; later K-steps add their byte offset / 16 to the start-address field.  For a
+  // pair the same shared-memory offsets name both CTAs' halves of each operand.
   const uint64_t q_desc = smem_desc_sw128(sbase + C::kQOff + t * C::kTileBytes, 16, 1024);
   const uint64_t kv_desc0 = smem_desc_sw128(sbase + C::kKVOff, 16, 1024);
   const uint64_t v_desc0 = smem_desc_sw128(sbase + C::kKVOff, 16384, 1024);
@@ -400,17 +466,30 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
   int ring = 0;
   int n_item = 0;
   bool ok = true;
+  int w = kPair ? (int)(blockIdx.x >> 1) : 0;
+  auto commit = [](uint32_t bar) {
+    if constexpr (kPair) mma_commit_pair(bar); else mma_commit(bar);
+  };
+  // A lane that skips a key tile still releases its slot: in both CTAs of a pair.
+  auto release = [&](uint32_t bar) {
+    mbar_arrive(bar);
+    if constexpr (kPair) mbar_arrive_cluster(map_shared(bar, 1));
+  };
   for (;; ++n_item) {
-    int w;
-    ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err);
-    if (!ok || w < 0) break;
-    const Item it = decode_item(p, w);
+    if constexpr (kPair) {
+      if (n_item > 0) w += (int)(gridDim.x >> 1);
+      if (w >= p.n_items) break;
+    } else {
+      ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err);
+      if (!ok || w < 0) break;
+    }
+    const Item it = decode_item<kPair>(p, w);
     ok = warp_mbar_wait(bars.q_full, q_full_ph, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
     q_full_ph ^= 1;
     if (!ok) break;
     tc_fence_after();
-    // O_t may be overwritten by this item's first P V only after the 4 softmax warps of lane t have
-    // read out the previous item's O: o_done[t] counts 4 per finished item.
+    // O_t may be overwritten by this item's first P V only after the softmax warps of lane t (4, or 8 over
+    // a pair) have read out the previous item's O: o_done[t] counts one per warp and finished item.
     bool need_odone = n_item > 0;
     bool first_pv = true;
     StepIter st;
@@ -430,7 +509,9 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
           ok = warp_mbar_wait(bars.kv_full(vs), (prev_v_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
                               abort_flag, p.err);
           if (ok && need_odone) {
-            ok = warp_counter_wait(bars.o_done(t), 4u * (uint32_t)n_item, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err);
+            const uint32_t target = C::kRowWarps * (uint32_t)n_item;
+            ok = kPair ? warp_counter_wait_cluster(bars.o_done(t), target, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err)
+                       : warp_counter_wait(bars.o_done(t), target, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err);
             need_odone = false;
           }
           if (ok) {
@@ -439,14 +520,18 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
           }
           if (!ok) break;
           tc_fence_after();
-          const uint64_t v_desc = v_desc0 + (uint64_t)((vs * C::kTileBytes) >> 4);
+          const uint64_t v_desc = v_desc0 + (uint64_t)((vs * C::kKVBytes) >> 4);
           const uint32_t acc0 = first_pv ? 0u : 1u;
           if (elect_one_sync()) {
 #pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk)
-              mma_ts(o_tmem, s_tmem + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
-            mma_commit(pv_done);
-            mma_commit(bars.kv_empty(vs));
+            for (int kk = 0; kk < kTile / 16; ++kk) {
+              if constexpr (kPair)
+                mma_ts_pair(o_tmem, s_tmem + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
+              else
+                mma_ts(o_tmem, s_tmem + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
+            }
+            commit(pv_done);
+            commit(bars.kv_empty(vs));
           }
           __syncwarp();
           first_pv = false;
@@ -456,7 +541,7 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
           ok = warp_mbar_wait(bars.kv_full(vs), (prev_v_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
                               abort_flag, p.err);
           if (!ok) break;
-          if (elect_one_sync()) mbar_arrive(bars.kv_empty(vs));
+          if (elect_one_sync()) release(bars.kv_empty(vs));
           __syncwarp();
         }
       }
@@ -470,21 +555,25 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
         ok = warp_mbar_wait(bars.kv_full(ks), (k_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
         if (!ok) break;
         tc_fence_after();
-        const uint64_t k_desc = kv_desc0 + (uint64_t)((ks * C::kTileBytes) >> 4);
+        const uint64_t k_desc = kv_desc0 + (uint64_t)((ks * C::kKVBytes) >> 4);
         if (elect_one_sync()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
-            mma_ss(s_tmem, q_desc + off, k_desc + off, C::kIdescS, kk > 0 ? 1u : 0u);
+            const uint64_t qo = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+            const uint64_t ko = (uint64_t)(((kk / 4) * C::kKSubBytes + (kk % 4) * 32) >> 4);
+            if constexpr (kPair)
+              mma_ss_pair(s_tmem, q_desc + qo, k_desc + ko, C::kIdescS, kk > 0 ? 1u : 0u);
+            else
+              mma_ss(s_tmem, q_desc + qo, k_desc + ko, C::kIdescS, kk > 0 ? 1u : 0u);
           }
-          mma_commit(s_full);
-          mma_commit(bars.kv_empty(ks));
+          commit(s_full);
+          commit(bars.kv_empty(ks));
         }
         __syncwarp();
       } else {
         ok = warp_mbar_wait(bars.kv_full(ks), (k_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
         if (!ok) break;
-        if (elect_one_sync()) mbar_arrive(bars.kv_empty(ks));
+        if (elect_one_sync()) release(bars.kv_empty(ks));
         __syncwarp();
       }
       ring += 2;
@@ -493,11 +582,11 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
       prev_v_pos = k_pos + 1;
     }
     if (!ok) break;
-    if (elect_one_sync()) mma_commit(bars.q_empty);  // this lane's S MMAs of the item are all issued
+    if (elect_one_sync()) commit(bars.q_empty);  // this lane's S MMAs of the item are all issued
     __syncwarp();
   }
   // Drain: nothing of ours may still run on the tensor cores when TMEM is released.
-  if (elect_one_sync()) mma_commit(bars.drain);
+  if (elect_one_sync()) commit(bars.drain);
   __syncwarp();
   warp_mbar_wait(bars.drain, 0, tmo, ERR_TIMEOUT_DRAIN, nullptr, p.err);
 }
@@ -505,10 +594,15 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
 // ------------------------------------------------------------------------------------------------
 // Softmax + epilogue: 4 warps per lane, one query row per thread.
 // ------------------------------------------------------------------------------------------------
-template <int D>
+template <int D, bool kPair>
 __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRing& ir, uint32_t tmem, int lane_t,
                             volatile int* abort_flag) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kPair>;
+  // A pair's rank 1 hands its P and its O read-outs to rank 0's barriers and counters.
+  const bool remote = kPair && cluster_rank() != 0;
+  const uint32_t p_full_bar = remote ? map_shared(bars.p_full(lane_t), 0) : bars.p_full(lane_t);
+  const uint32_t o_done_ctr = remote ? map_shared(bars.o_done(lane_t), 0) : bars.o_done(lane_t);
+  int w_pair = kPair ? (int)(blockIdx.x >> 1) : 0;
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int row = (warp & 3) * 32 + lane;                            // row within the 128-row tile
@@ -523,11 +617,17 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
 
   for (int n_item = 0;; ++n_item) {
     int w;
-    ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err);
-    if (!ok || w < 0) break;
-    __syncwarp();
-    if (lane == 0) smem_counter_add_release(ir.used0 + 4u * warp, 1u);  // this warp is done with the slot
-    const Item it = decode_item(p, w);
+    if constexpr (kPair) {
+      if (n_item > 0) w_pair += (int)(gridDim.x >> 1);
+      w = w_pair;
+      if (w >= p.n_items) break;
+    } else {
+      ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err);
+      if (!ok || w < 0) break;
+      __syncwarp();
+      if (lane == 0) smem_counter_add_release(ir.used0 + 4u * warp, 1u);  // this warp is done with the slot
+    }
+    const Item it = decode_item<kPair>(p, w);
     StepIter st;
     st.init(p, it);
     const int q_row = (lane_t ? it.q_start[1] : it.q_start[0]) + row;
@@ -627,7 +727,12 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bars.p_full(lane_t));
+      if (lane == 0) {
+        if (remote)
+          mbar_arrive_cluster(p_full_bar);
+        else
+          mbar_arrive(p_full_bar);
+      }
       ++n_kept;
       ++total_pv;
     }
@@ -690,14 +795,19 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
     }
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) smem_counter_add_release(bars.o_done(lane_t), 1u);
+    if (lane == 0) {
+      if (remote)
+        counter_add_cluster(o_done_ctr, 1u);
+      else
+        smem_counter_add_release(o_done_ctr, 1u);
+    }
   }
 }
 
-template <int D>
+template <int D, bool kPair>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ AttnParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kPair>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t bar0 = smem_u32(smem + C::kBarOff);
@@ -729,7 +839,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bars.s_full(t), 1);
-      mbar_init(bars.p_full(t), 4);   // one arrival per softmax warp
+      mbar_init(bars.p_full(t), C::kRowWarps);  // one arrival per softmax warp of the lane (pair: both CTAs)
       mbar_init(bars.pv_done(t), 1);
     }
     for (int k = 0; k < 2; ++k)  // o_done[0..1] counters
@@ -744,40 +854,52 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kWarpProducer && lane == 0) {
     for (int r = 0; r < p.n_shards; ++r) {
       tma_prefetch_desc(&tm.q[r]);
-      tma_prefetch_desc(&tm.k[r]);
+      if (kPair) {
+        tma_prefetch_desc(&tm.k64[r]);
+      } else {
+        tma_prefetch_desc(&tm.k[r]);
+      }
       tma_prefetch_desc(&tm.v[r]);
     }
   }
-  if (warp == kWarpMma) {
-    tmem_alloc(smem_u32(tmem_holder), 512);
-    tmem_relinquish();
+  if (warp == kWarpMma) {  // a pair allocates the same 512 columns in both CTAs, from the same warp
+    if constexpr (kPair) {
+      tmem_alloc_pair(smem_u32(tmem_holder), 512);
+      tmem_relinquish_pair();
+    } else {
+      tmem_alloc(smem_u32(tmem_holder), 512);
+      tmem_relinquish();
+    }
   }
   tc_fence_before();
-  __syncthreads();
+  // a pair: both CTAs' barriers are initialised before either CTA arrives on the other's
+  if constexpr (kPair) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
 
   if (warp < 8) {
     regs_inc<kRegsSoftmax>();
-    run_softmax<D>(p, bars, ir, tmem, warp >> 2, abort_flag);
+    run_softmax<D, kPair>(p, bars, ir, tmem, warp >> 2, abort_flag);
   } else {
     regs_dec<kRegsControl>();
     if (warp == kWarpProducer) {
-      run_producer<D>(p, tm, smem, bars, ir, abort_flag);
-    } else if (warp == kWarpMma || warp == kWarpMma + 1) {
-      run_mma<D>(p, smem, bars, ir, tmem, warp - kWarpMma, abort_flag);
+      run_producer<D, kPair>(p, tm, smem, bars, ir, abort_flag);
+    } else if ((warp == kWarpMma || warp == kWarpMma + 1) && (!kPair || cluster_rank() == 0)) {
+      run_mma<D, kPair>(p, smem, bars, ir, tmem, warp - kWarpMma, abort_flag);  // a pair's MMAs: rank 0
     }
     __syncwarp();
   }
   tc_fence_before();
-  __syncthreads();
+  // a pair: neither CTA leaves (or frees TMEM) while the other may still touch its shared memory or the
+  // pair's MMAs may still write its TMEM (rank 0 drained them before arriving here)
+  if constexpr (kPair) cluster_sync(); else __syncthreads();
   if (warp == kWarpMma) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    if constexpr (kPair) tmem_dealloc_pair(tmem, 512); else tmem_dealloc(tmem, 512);
   }
   // The last CTA to finish returns this launch's work counter to zero for the next launch that draws
   // the same slot (every CTA has made its last claim before it gets here).
-  if (threadIdx.x == 0) {
+  if (!kPair && threadIdx.x == 0) {
     __threadfence();
     if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
       atomicExch(p.sched, 0u);
@@ -807,21 +929,92 @@ sp_status launch_attn(const AttnParams& p_in, const void* q, const void* k, cons
   return launch_attn_sharded(p, stream);
 }
 
+// CTA pairs (one cluster of two CTAs per TPC) for D = 128 without a mask or item list; SP_ATTN_PAIR=0 in the
+// environment keeps every launch on single CTAs.
+static bool pair_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = std::getenv("SP_ATTN_PAIR");
+    on = (e && e[0] == '0') ? 0 : 1;
+  }
+  return on == 1;
+}
+
+template <int D, bool kPair>
+static sp_status launch_kernel(const TMaps& tm, const AttnParams& p, int grid, cudaStream_t stream, int dev) {
+  using C = Cfg<D, kPair>;
+  static int regs_ok[kMaxDevices] = {};
+  static bool attr_set[kMaxDevices] = {};
+  // The warpgroups re-divide the registers the CTA was launched with; a kernel built with another
+  // per-thread count would make that division wait forever, so it is never launched.
+  if (regs_ok[dev] == 0) {
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kPair>) != cudaSuccess) return SP_ERR_CUDA;
+    regs_ok[dev] = fa.numRegs == kRegsLaunch ? 1 : -1;
+  }
+  if (regs_ok[dev] < 0) return SP_ERR_UNSUPPORTED;
+  if (!attr_set[dev]) {
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kPair>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+      return SP_ERR_CUDA;
+    attr_set[dev] = true;
+  }
+  if constexpr (kPair) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = C::kSmemBytes;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    if (cudaLaunchKernelEx(&cfg, attn_fwd_kernel<D, kPair>, tm, p) != cudaSuccess) return SP_ERR_CUDA;
+  } else {
+    attn_fwd_kernel<D, kPair><<<grid, kThreads, C::kSmemBytes, stream>>>(tm, p);
+  }
+  return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+}
+
 sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
   AttnParams p = p_in;
   if (p.n_shards < 1 || p.n_shards > kMaxShards || p.shard_rows < 1 || (long long)p.n_shards * p.shard_rows != p.S ||
       p.tiles_per_shard != (p.shard_rows + kTile - 1) / kTile || p.pairs_per_shard != (p.tiles_per_shard + 1) / 2 ||
       p.n_qpairs != p.n_shards * p.pairs_per_shard)
     return SP_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SP_ERR_CUDA;
+  const int sms = num_sms(dev);
+  const bool pair = p.D == 128 && !p.row_ptr && !p.item_list && sms >= 2 && pair_enabled();
   TMaps tm{};  // the kernel argument (copied at launch)
   for (int r = 0; r < p.n_shards; ++r)
     if (!encode_bshd_tmap(&tm.q[r], p.q_shard[r], p.B, p.shard_rows, p.H, p.D) ||
         !encode_bshd_tmap(&tm.k[r], p.k_shard[r], p.B, p.shard_rows, p.H, p.D) ||
-        !encode_bshd_tmap(&tm.v[r], p.v_shard[r], p.B, p.shard_rows, p.H, p.D))
+        !encode_bshd_tmap(&tm.v[r], p.v_shard[r], p.B, p.shard_rows, p.H, p.D) ||
+        (pair && !encode_bshd_tmap(&tm.k64[r], p.k_shard[r], p.B, p.shard_rows, p.H, p.D, 64)))
       return SP_ERR_CUDA;
+  if (pair) {
+    // work units of four query tiles (two per CTA of the pair), per shard
+    p.pairs_per_shard = (p.tiles_per_shard + 3) / 4;
+    p.n_qpairs = p.n_shards * p.pairs_per_shard;
+    long long items = 0;
+    for (int c = 0; c < p.n_chunks; ++c) {
+      p.chunk_item0[c] = (int)items;
+      items += (long long)p.B * (p.chunk_h0[c + 1] - p.chunk_h0[c]) * p.n_qpairs;
+    }
+    p.chunk_item0[p.n_chunks] = (int)items;
+    if (items > 0x7fffffffLL) return SP_ERR_INVALID_ARG;
+    p.n_items = (int)items;
+  }
   if (p.n_items <= 0) return SP_OK;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SP_ERR_CUDA;
+  if (pair) {
+    const long long want = 2LL * p.n_items;
+    const int grid = (int)(want < (sms & ~1) ? want : (sms & ~1));
+    return launch_kernel<128, true>(tm, p, grid, stream, dev);
+  }
   {
     static unsigned int* sched_base[kMaxDevices] = {};
     static std::atomic<unsigned int> launch_seq{0};
@@ -832,40 +1025,9 @@ sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
     }
     p.sched = sched_base[dev] + 2 * (launch_seq.fetch_add(1) % kSchedSlots);
   }
-  const int grid = p.n_items < num_sms(dev) ? p.n_items : num_sms(dev);
-  const int smem = attn_smem_bytes(p.D);
-  cudaError_t e;
-  // The warpgroups re-divide the registers the CTA was launched with; a kernel built with another
-  // per-thread count would make that division wait forever, so it is never launched.
-  {
-    static int regs_ok[kMaxDevices][2] = {};
-    int& ok = regs_ok[dev][p.D == 128 ? 1 : 0];
-    if (ok == 0) {
-      cudaFuncAttributes fa;
-      e = p.D == 128 ? cudaFuncGetAttributes(&fa, attn_fwd_kernel<128>) : cudaFuncGetAttributes(&fa, attn_fwd_kernel<64>);
-      if (e != cudaSuccess) return SP_ERR_CUDA;
-      ok = fa.numRegs == kRegsLaunch ? 1 : -1;
-    }
-    if (ok < 0) return SP_ERR_UNSUPPORTED;
-  }
-  if (p.D == 128) {
-    static bool attr_set[kMaxDevices] = {};
-    if (!attr_set[dev]) {
-      e = cudaFuncSetAttribute(attn_fwd_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return SP_ERR_CUDA;
-      attr_set[dev] = true;
-    }
-    attn_fwd_kernel<128><<<grid, kThreads, smem, stream>>>(tm, p);
-  } else {
-    static bool attr_set[kMaxDevices] = {};
-    if (!attr_set[dev]) {
-      e = cudaFuncSetAttribute(attn_fwd_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-      if (e != cudaSuccess) return SP_ERR_CUDA;
-      attr_set[dev] = true;
-    }
-    attn_fwd_kernel<64><<<grid, kThreads, smem, stream>>>(tm, p);
-  }
-  return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+  const int grid = p.n_items < sms ? p.n_items : sms;
+  return p.D == 128 ? launch_kernel<128, false>(tm, p, grid, stream, dev)
+                    : launch_kernel<64, false>(tm, p, grid, stream, dev);
 }
 
 }  // namespace spattn

@@ -74,7 +74,7 @@ struct BwdParams {
 
 // Device properties and driver entry points (cached per device).
 int num_sms(int device);
-bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, int D);
+bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, int D, int box_rows = 128);
 unsigned long long wait_timeout_ns();
 unsigned int* device_error_word();  // address of the current device's error word, or nullptr
 

@@ -268,6 +268,110 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
 }
 
 // ------------------------------------------------------------------------------------------------
+// CTA pairs (a cluster of two CTAs on the two SMs of a TPC): the pair's MMAs are issued by rank 0 and
+// run on both SMs, each SM holding its half of A (rows) and of B (N columns) in its own shared memory
+// at the same offsets, and its half of D (rows) in its own TMEM.
+// ------------------------------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// The shared::cluster address of this CTA's shared address `a` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t map_shared(uint32_t a, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// Arrive on an mbarrier given by its shared::cluster address (possibly in the other CTA of the pair).
+// Default (CTA-scope) release semantics: the data this hands over lives in TMEM and is ordered by the
+// tcgen05 fences around the arrive and the wait; a cluster-scope release here made every step of the
+// pair's chain about 40% longer.
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+__device__ __forceinline__ void counter_add_cluster(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("red.release.cluster.shared::cluster.add.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t smem_load_acquire_cluster(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.acquire.cluster.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+// Waits as counter_wait, acquiring at cluster scope: for a counter the other CTA of a pair also adds to.
+__device__ __forceinline__ bool warp_counter_wait_cluster(uint32_t addr, uint32_t target, uint64_t timeout_ns,
+                                                          unsigned int code, volatile int* abort_flag,
+                                                          unsigned int* err) {
+  bool ok = smem_load_acquire_cluster(addr) >= target;
+  if (!ok) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (smem_load_acquire_cluster(addr) >= target) {
+        ok = true;
+        break;
+      }
+      if ((it & 63u) == 0) {
+        if (abort_flag && *abort_flag) break;
+        if (global_timer_ns() - t0 > timeout_ns) {
+          atomicOr(err, code);
+          if (abort_flag) *abort_flag = 1;
+          break;
+        }
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
+// A tile load of this CTA's half of a pair operand: the data lands in this CTA's shared memory at dst,
+// the byte count completes on the mbarrier at the shared::cluster address bar (rank 0's barrier).
+__device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1, int c2,
+                                                 int c3) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(tmap), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t dst_smem, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(dst_smem), "r"(ncols)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish_pair() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+// D[tmem] (+)= A[smem] * B[smem] over the pair (M = 256: 128 rows per CTA; B split by N).
+__device__ __forceinline__ void mma_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u));
+}
+// D[tmem] (+)= A[tmem] * B[smem] over the pair.
+__device__ __forceinline__ void mma_ts_pair(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], [%1], %2, %3, {%5, %5, %5, %5, %5, %5, %5, %5}, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(0u));
+}
+// Arrive once on the mbarrier at shared offset `bar` in both CTAs of the pair when every tcgen05 operation
+// this thread issued before has completed.
+__device__ __forceinline__ void mma_commit_pair(uint32_t bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"((uint16_t)3));
+}
+
+// ------------------------------------------------------------------------------------------------
 // Descriptors
 // ------------------------------------------------------------------------------------------------
 // Shared-memory matrix descriptor, 128-byte swizzle: start address, leading and stride byte offsets
