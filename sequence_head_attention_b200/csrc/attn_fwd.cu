@@ -294,9 +294,12 @@ struct ItemRing {
   volatile int* ids;
 };
 
+// cluster_acquire: the ring is written by the other CTA of a pair (rank 1 reads what rank 0 publishes).
 __device__ __forceinline__ bool ring_read(const ItemRing& r, int n, int& w, uint64_t tmo, volatile int* abort_flag,
-                                          unsigned int* err) {
-  if (!warp_counter_wait(r.pub, (uint32_t)(n + 1), tmo, ERR_TIMEOUT_ITEM, abort_flag, err)) return false;
+                                          unsigned int* err, bool cluster_acquire = false) {
+  const bool ok = cluster_acquire ? warp_counter_wait_cluster(r.pub, (uint32_t)(n + 1), tmo, ERR_TIMEOUT_ITEM, abort_flag, err)
+                                  : warp_counter_wait(r.pub, (uint32_t)(n + 1), tmo, ERR_TIMEOUT_ITEM, abort_flag, err);
+  if (!ok) return false;
   w = r.ids[n % kItemRing];
   return true;
 }
@@ -332,31 +335,46 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
   int n_item = 0;
   int last_q_item = -1;
   bool ok = true;
+  // The work units a CTA (or a pair, whose rank 0 claims for both) takes: its first by its index, then by
+  // claiming from the launch's counter; ids go into the item ring of the CTA (or of both CTAs of the pair).
+  const int n_workers = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   int w = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
   for (;; ++n_item) {
     bool done;
-    if constexpr (kPair) {  // a pair walks its units in a fixed stride
-      if (n_item > 0) w += (int)(gridDim.x >> 1);
-      done = w >= p.n_items;
+    if (kPair && rk != 0) {  // rank 1 reads what rank 0 published into its ring
+      ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err, true);
+      if (!ok) break;
+      done = w < 0;
       if (done) break;
     } else {
       if (n_item > 0) {  // claim the next item
         int claimed = 0;
-        if (elect_one_sync()) claimed = (int)gridDim.x + (int)atomicAdd(p.sched, 1u);
+        if (elect_one_sync()) claimed = n_workers + (int)atomicAdd(p.sched, 1u);
         w = __shfl_sync(0xffffffffu, claimed, __ffs(__ballot_sync(0xffffffffu, claimed != 0)) - 1);
       }
       done = w >= p.n_items;
-      // publish it (the slot's previous item must have been read by every softmax warp)
+      // publish it (the slot's previous item must have been read by every softmax warp, of both CTAs)
       if (n_item >= kItemRing) {
         const uint32_t need = (uint32_t)(n_item - kItemRing + 1);
 #pragma unroll 1
         for (int k = 0; k < 8 && ok; ++k)
           ok = warp_counter_wait(ir.used0 + 4u * k, need, tmo, ERR_TIMEOUT_ITEM_FREE, abort_flag, p.err);
+        if constexpr (kPair) {
+#pragma unroll 1
+          for (int k = 0; k < 8 && ok; ++k)
+            ok = warp_remote_counter_wait(map_shared(ir.used0 + 4u * k, 1), need, tmo, ERR_TIMEOUT_ITEM_FREE,
+                                          abort_flag, p.err);
+        }
         if (!ok) break;
       }
       if (elect_one_sync()) {
-        ir.ids[n_item % kItemRing] = done ? -1 : w;
+        const int id = done ? -1 : w;
+        ir.ids[n_item % kItemRing] = id;
         smem_counter_add_release(ir.pub, 1u);
+        if constexpr (kPair) {
+          remote_store(map_shared(smem_u32((const void*)(ir.ids + n_item % kItemRing)), 1), (uint32_t)id);
+          counter_add_cluster(map_shared(ir.pub, 1), 1u);
+        }
       }
       __syncwarp();
       if (done) break;
@@ -466,7 +484,7 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
   int ring = 0;
   int n_item = 0;
   bool ok = true;
-  int w = kPair ? (int)(blockIdx.x >> 1) : 0;
+  int w = 0;
   auto commit = [](uint32_t bar) {
     if constexpr (kPair) mma_commit_pair(bar); else mma_commit(bar);
   };
@@ -476,13 +494,8 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
     if constexpr (kPair) mbar_arrive_cluster(map_shared(bar, 1));
   };
   for (;; ++n_item) {
-    if constexpr (kPair) {
-      if (n_item > 0) w += (int)(gridDim.x >> 1);
-      if (w >= p.n_items) break;
-    } else {
-      ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err);
-      if (!ok || w < 0) break;
-    }
+    ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err);
+    if (!ok || w < 0) break;
     const Item it = decode_item<kPair>(p, w);
     ok = warp_mbar_wait(bars.q_full, q_full_ph, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
     q_full_ph ^= 1;
@@ -602,7 +615,7 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
   const bool remote = kPair && cluster_rank() != 0;
   const uint32_t p_full_bar = remote ? map_shared(bars.p_full(lane_t), 0) : bars.p_full(lane_t);
   const uint32_t o_done_ctr = remote ? map_shared(bars.o_done(lane_t), 0) : bars.o_done(lane_t);
-  int w_pair = kPair ? (int)(blockIdx.x >> 1) : 0;
+
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int row = (warp & 3) * 32 + lane;                            // row within the 128-row tile
@@ -617,16 +630,10 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
 
   for (int n_item = 0;; ++n_item) {
     int w;
-    if constexpr (kPair) {
-      if (n_item > 0) w_pair += (int)(gridDim.x >> 1);
-      w = w_pair;
-      if (w >= p.n_items) break;
-    } else {
-      ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err);
-      if (!ok || w < 0) break;
-      __syncwarp();
-      if (lane == 0) smem_counter_add_release(ir.used0 + 4u * warp, 1u);  // this warp is done with the slot
-    }
+    ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err, remote);
+    if (!ok || w < 0) break;
+    __syncwarp();
+    if (lane == 0) smem_counter_add_release(ir.used0 + 4u * warp, 1u);  // this warp is done with the slot
     const Item it = decode_item<kPair>(p, w);
     StepIter st;
     st.init(p, it);
@@ -899,7 +906,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // The last CTA to finish returns this launch's work counter to zero for the next launch that draws
   // the same slot (every CTA has made its last claim before it gets here).
-  if (!kPair && threadIdx.x == 0) {
+  if (threadIdx.x == 0) {
     __threadfence();
     if (atomicAdd(p.sched + 1, 1u) == gridDim.x - 1) {
       atomicExch(p.sched, 0u);
@@ -1010,11 +1017,6 @@ sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
     p.n_items = (int)items;
   }
   if (p.n_items <= 0) return SP_OK;
-  if (pair) {
-    const long long want = 2LL * p.n_items;
-    const int grid = (int)(want < (sms & ~1) ? want : (sms & ~1));
-    return launch_kernel<128, true>(tm, p, grid, stream, dev);
-  }
   {
     static unsigned int* sched_base[kMaxDevices] = {};
     static std::atomic<unsigned int> launch_seq{0};
@@ -1024,6 +1026,11 @@ sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
       sched_base[dev] = static_cast<unsigned int*>(ptr);
     }
     p.sched = sched_base[dev] + 2 * (launch_seq.fetch_add(1) % kSchedSlots);
+  }
+  if (pair) {
+    const long long want = 2LL * p.n_items;
+    const int grid = (int)(want < (sms & ~1) ? want : (sms & ~1));
+    return launch_kernel<128, true>(tm, p, grid, stream, dev);
   }
   const int grid = p.n_items < sms ? p.n_items : sms;
   return p.D == 128 ? launch_kernel<128, false>(tm, p, grid, stream, dev)

@@ -325,6 +325,39 @@ __device__ __forceinline__ bool warp_counter_wait_cluster(uint32_t addr, uint32_
   }
   return __all_sync(0xffffffffu, ok);
 }
+// Loads and stores of another CTA's shared memory (shared::cluster addresses).
+__device__ __forceinline__ uint32_t remote_load_acquire(uint32_t cluster_addr) {
+  uint32_t v;
+  asm volatile("ld.acquire.cluster.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void remote_store(uint32_t cluster_addr, uint32_t v) {
+  asm volatile("st.relaxed.cluster.shared::cluster.u32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+// Waits until the counter at a shared::cluster address reaches `target` (bounded like counter_wait).
+__device__ __forceinline__ bool warp_remote_counter_wait(uint32_t cluster_addr, uint32_t target, uint64_t timeout_ns,
+                                                         unsigned int code, volatile int* abort_flag,
+                                                         unsigned int* err) {
+  bool ok = remote_load_acquire(cluster_addr) >= target;
+  if (!ok) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 1;; ++it) {
+      if (remote_load_acquire(cluster_addr) >= target) {
+        ok = true;
+        break;
+      }
+      if ((it & 63u) == 0) {
+        if (abort_flag && *abort_flag) break;
+        if (global_timer_ns() - t0 > timeout_ns) {
+          atomicOr(err, code);
+          if (abort_flag) *abort_flag = 1;
+          break;
+        }
+      }
+    }
+  }
+  return __all_sync(0xffffffffu, ok);
+}
 // A tile load of this CTA's half of a pair operand: the data lands in this CTA's shared memory at dst,
 // the byte count completes on the mbarrier at the shared::cluster address bar (rank 0's barrier).
 __device__ __forceinline__ void tma_load_4d_pair(uint32_t dst, const void* tmap, uint32_t bar, int c0, int c1, int c2,
