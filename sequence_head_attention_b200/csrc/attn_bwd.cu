@@ -48,12 +48,13 @@ struct BCfg {
   static constexpr int kStageOff = 2 * kTileBytes;
   static constexpr int kStageBytes = 2 * kTileBytes + 1024;
   static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
-  static constexpr int kNumBars = 1 + 2 * kStages + 4;  // res_full, full[S], empty[S], st_full, p_full, acc_full, drain
+  // res_full, full[S], empty[S], st_full[2], p_full[2], acc_full, drain
+  static constexpr int kNumBars = 1 + 2 * kStages + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // one CTA per SM: its TMEM allocation takes all 512 columns
   static constexpr int kRaw = kMiscOff + 16 + 1024;
   static constexpr int kSmemBytes = kRaw > 120 * 1024 ? kRaw : 120 * 1024;
-  static constexpr uint32_t kIdescSq = idesc_bf16_f32(128, 128, false, false);  // both operands K-major
+  static constexpr uint32_t kIdescSq = idesc_bf16_f32(128, 64, false, false);  // S, dP of a 64-row half; K-major
   static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);    // B operand MN-major
 };
 
@@ -62,10 +63,17 @@ struct BwdMaps {
 };
 
 struct BwdBars {
-  uint32_t res_full, full0, empty0, st_full, p_full, acc_full, drain;
+  uint32_t res_full, full0, empty0, st_full0, p_full0, acc_full, drain;
   __device__ uint32_t full(int s) const { return full0 + 8u * s; }
   __device__ uint32_t empty(int s) const { return empty0 + 8u * s; }
+  __device__ uint32_t st_full(int b) const { return st_full0 + 8u * b; }  // per TMEM buffer
+  __device__ uint32_t p_full(int b) const { return p_full0 + 8u * b; }
 };
+
+// TMEM: two buffers of a 64-row half of a streamed tile, each S (64 columns) then dP (64 columns): buffer b
+// at columns [128 b, 128 b + 128); accumulators from 256.
+__device__ __forceinline__ uint32_t tS_of(uint32_t t, int b) { return t + 128u * b; }
+__device__ __forceinline__ uint32_t tdP_of(uint32_t t, int b) { return t + 128u * b + 64u; }
 
 // The CTA's tile and the range of streamed tiles it walks.
 struct BwdItem {
@@ -165,60 +173,80 @@ __device__ void bwd_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase,
   using C = BCfg<D>;
   const uint64_t tmo = p.timeout_ns;
   const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_in, 0);
-  const uint32_t tS = tmem, tdP = tmem + 128, tAcc0 = tmem + 256, tAcc1 = tmem + 256 + D;
+  const uint32_t tAcc0 = tmem + 256, tAcc1 = tmem + 256 + D;
   // K-major descriptors of K-step 0 (the row-major tiles as the MMAs' K-major operands), and MN-major ones
-  // of the streamed tiles as the right operand of the accumulating MMAs.
+  // of the streamed tiles as the right operand of the accumulating MMAs.  Streamed tiles are taken in two
+  // halves of 64 rows (sub-step m = 2 n + h, TMEM buffer h): half h starts 8192 bytes into each 64-column
+  // sub-tile.  The S and dP of half m are issued before the accumulating MMAs of half m - 1, so the tensor
+  // cores run one half while the row warps work on the other.
   const uint64_t res0_k = smem_desc_sw128(sbase + C::kResOff, 16, 1024);
   const uint64_t res1_k = smem_desc_sw128(sbase + C::kResOff + C::kTileBytes, 16, 1024);
   bool ok = warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
-  for (int n = 0; n < it.n_steps && ok; ++n) {
-    const int s = n % C::kStages;
-    const uint32_t stage = sbase + C::kStageOff + s * C::kStageBytes;
-    ok = warp_mbar_wait(bars.full(s), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
-    if (!ok) break;
-    tc_fence_after();
-    const uint64_t str0_k = smem_desc_sw128(stage, 16, 1024);
-    const uint64_t str1_k = smem_desc_sw128(stage + C::kTileBytes, 16, 1024);
+  // accumulating MMAs of half hh of streamed tile nn (rows 64 hh .. 64 hh + 63), from TMEM buffer hh
+  auto accumulate = [&](int nn, int hh) {
+    const uint32_t stage = sbase + C::kStageOff + (nn % C::kStages) * C::kStageBytes;
+    const uint64_t str0_mn = smem_desc_sw128(stage, 16384, 1024) + (uint64_t)((8192 * hh) >> 4);
+    const uint64_t str1_mn = smem_desc_sw128(stage + C::kTileBytes, 16384, 1024) + (uint64_t)((8192 * hh) >> 4);
+    const bool first = nn == 0 && hh == 0;
+    if (kDQ) {
+      // dQ += dS K
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts(tAcc0, tdP_of(tmem, hh) + kk * 8, str0_mn + (uint64_t)(kk * 128), C::kIdescAcc, (first && kk == 0) ? 0u : 1u);
+    } else {
+      // dV += P^T dO, dK += dS^T Q
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts(tAcc0, tS_of(tmem, hh) + kk * 8, str1_mn + (uint64_t)(kk * 128), C::kIdescAcc, (first && kk == 0) ? 0u : 1u);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts(tAcc1, tdP_of(tmem, hh) + kk * 8, str0_mn + (uint64_t)(kk * 128), C::kIdescAcc, (first && kk == 0) ? 0u : 1u);
+    }
+    if (hh == 1) mma_commit(bars.empty(nn % C::kStages));  // both halves of the tile consumed
+  };
+  const int n_sub = 2 * it.n_steps;
+  for (int m = 0; m < n_sub && ok; ++m) {
+    const int n = m >> 1, h = m & 1;
+    if (h == 0) {
+      ok = warp_mbar_wait(bars.full(n % C::kStages), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+      if (!ok) break;
+      tc_fence_after();
+    }
+    const uint32_t stage = sbase + C::kStageOff + (n % C::kStages) * C::kStageBytes;
+    const uint64_t str0_k = smem_desc_sw128(stage, 16, 1024) + (uint64_t)((8192 * h) >> 4);
+    const uint64_t str1_k = smem_desc_sw128(stage + C::kTileBytes, 16, 1024) + (uint64_t)((8192 * h) >> 4);
     if (elect_one_sync()) {
-      // dK/dV: S^T = K Q^T, dP^T = V dO^T.   dQ: S = Q K^T, dP = dO V^T.
+      // dK/dV: S^T = K Q_h^T, dP^T = V dO_h^T.   dQ: S = Q K_h^T, dP = dO V_h^T.
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
-        mma_ss(tS, res0_k + off, str0_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
+        mma_ss(tS_of(tmem, h), res0_k + off, str0_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
-        mma_ss(tdP, res1_k + off, str1_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
+        mma_ss(tdP_of(tmem, h), res1_k + off, str1_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
       }
-      mma_commit(bars.st_full);
+      mma_commit(bars.st_full(h));
     }
     __syncwarp();
-    ok = warp_mbar_wait(bars.p_full, n & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
-    if (!ok) break;
-    tc_fence_after();
-    const uint32_t acc = n > 0 ? 1u : 0u;
-    if (elect_one_sync()) {
-      // K-steps of 16 rows of the streamed tiles: 8 packed bf16 columns of P / dS, 16 rows of the tile
-      const uint64_t str0_mn = smem_desc_sw128(stage, 16384, 1024);
-      const uint64_t str1_mn = smem_desc_sw128(stage + C::kTileBytes, 16384, 1024);
-      if (kDQ) {
-        // dQ += dS K
-#pragma unroll
-        for (int kk = 0; kk < kBT / 16; ++kk)
-          mma_ts(tAcc0, tdP + kk * 8, str0_mn + (uint64_t)(kk * 128), C::kIdescAcc, kk > 0 ? 1u : acc);
-      } else {
-        // dV += P^T dO, dK += dS^T Q
-#pragma unroll
-        for (int kk = 0; kk < kBT / 16; ++kk)
-          mma_ts(tAcc0, tS + kk * 8, str1_mn + (uint64_t)(kk * 128), C::kIdescAcc, kk > 0 ? 1u : acc);
-#pragma unroll
-        for (int kk = 0; kk < kBT / 16; ++kk)
-          mma_ts(tAcc1, tdP + kk * 8, str0_mn + (uint64_t)(kk * 128), C::kIdescAcc, kk > 0 ? 1u : acc);
-      }
-      mma_commit(bars.empty(s));
+    if (m > 0) {  // the previous half: once its P and dS are in TMEM
+      const int mp = m - 1, hp = mp & 1;
+      ok = warp_mbar_wait(bars.p_full(hp), (mp >> 1) & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one_sync()) accumulate(mp >> 1, hp);
+      __syncwarp();
     }
-    __syncwarp();
+  }
+  if (ok && n_sub > 0) {  // the last half
+    const int mp = n_sub - 1, hp = mp & 1;
+    ok = warp_mbar_wait(bars.p_full(hp), (mp >> 1) & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
+    if (ok) {
+      tc_fence_after();
+      if (elect_one_sync()) accumulate(mp >> 1, hp);
+      __syncwarp();
+    }
   }
   if (ok && elect_one_sync()) mma_commit(bars.acc_full);
   __syncwarp();
@@ -238,7 +266,7 @@ __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, u
   const int quad = warp & 3;
   const int r = quad * 32 + lane;                                // row of the resident tile
   const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
-  const uint32_t tS = trow, tdP = trow + 128, tAcc0 = trow + 256, tAcc1 = trow + 256 + D;
+  const uint32_t tAcc0 = trow + 256, tAcc1 = trow + 256 + D;
   const uint64_t tmo = p.timeout_ns;
   const float sl2 = p.scale_log2;
   const int row = it.tile * kBT + r;                             // global position of this thread's row
@@ -252,63 +280,63 @@ __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, u
     dlt_row = __ldg(p.delta + i);
   }
   bool ok = true;
-  for (int n = 0; n < it.n_steps; ++n) {
+  // sub-step m = 2 n + h: the 64 rows 64 h .. 64 h + 63 of streamed tile n, in TMEM buffer h
+  for (int m = 0; m < 2 * it.n_steps; ++m) {
+    const int n = m >> 1, h = m & 1;
     const int t = it.first + n;
     const float* lse2 = reinterpret_cast<const float*>(smem + C::kStageOff + (n % C::kStages) * C::kStageBytes +
                                                        2 * C::kTileBytes);
     const float* dlt = lse2 + kBT;
-    if (!kDQ) {
+    if (!kDQ && h == 0) {
       // lse and delta of the streamed tile were stored by the producer before it released the slot's
-      // full barrier: acquire them from that barrier (the slot is refilled only after this step's
-      // P arrives, so the phase cannot have moved on)
+      // full barrier: acquire them from that barrier (the slot is refilled only after both halves' P
+      // arrive, so the phase cannot have moved on)
       ok = mbar_wait(bars.full(n % C::kStages), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
     }
-    ok = mbar_wait(bars.st_full, n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err);
+    ok = mbar_wait(bars.st_full(h), n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     tc_fence_after();
+    const uint32_t tS = trow + 128u * h, tdP = tS + 64;
+    uint32_t s[2][32], dp[2][32];
+    tmem_ld32(tS, s[0]);
+    tmem_ld32(tS + 32, s[1]);
+    tmem_ld32(tdP, dp[0]);
+    tmem_ld32(tdP + 32, dp[1]);
+    tmem_wait_ld();
+    uint32_t pk_p[32], pk_ds[32];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t s[2][32], dp[2][32];
-      tmem_ld32(tS + 64 * half, s[0]);
-      tmem_ld32(tS + 64 * half + 32, s[1]);
-      tmem_ld32(tdP + 64 * half, dp[0]);
-      tmem_ld32(tdP + 64 * half + 32, dp[1]);
-      tmem_wait_ld();
-      uint32_t pk_p[32], pk_ds[32];
+    for (int e = 0; e < 64; e += 2) {
+      float pr[2], ds[2];
 #pragma unroll
-      for (int e = 0; e < 64; e += 2) {
-        float pr[2], ds[2];
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          const int c = 64 * half + e + u;  // column: the streamed tile's row
-          const float sv = __uint_as_float(s[(e + u) >> 5][(e + u) & 31]);
-          const float dv = __uint_as_float(dp[(e + u) >> 5][(e + u) & 31]);
-          float pv;
-          if (kDQ) {
-            pv = ex2_approx(sv * sl2 - lse2_row);
-            if ((p.causal && t * kBT + c > row) || t * kBT + c >= kv_lim) pv = 0.f;  // key after the query, or outside the range
-            ds[u] = pv * (dv - dlt_row);
-          } else {
-            pv = ex2_approx(sv * sl2 - lse2[c]);
-            if (p.causal && t * kBT + c < row) pv = 0.f;  // query before the key
-            ds[u] = pv * (dv - dlt[c]);
-          }
-          pr[u] = pv;
+      for (int u = 0; u < 2; ++u) {
+        const int c = 64 * h + e + u;  // column: the streamed tile's row
+        const float sv = __uint_as_float(s[(e + u) >> 5][(e + u) & 31]);
+        const float dv = __uint_as_float(dp[(e + u) >> 5][(e + u) & 31]);
+        float pv;
+        if (kDQ) {
+          pv = ex2_approx(sv * sl2 - lse2_row);
+          if ((p.causal && t * kBT + c > row) || t * kBT + c >= kv_lim) pv = 0.f;  // key after the query, or outside the range
+          ds[u] = pv * (dv - dlt_row);
+        } else {
+          pv = ex2_approx(sv * sl2 - lse2[c]);
+          if (p.causal && t * kBT + c < row) pv = 0.f;  // query before the key
+          ds[u] = pv * (dv - dlt[c]);
         }
-        pk_p[e >> 1] = pack_bf16x2(pr[0], pr[1]);
-        pk_ds[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+        pr[u] = pv;
       }
-      // packed columns [32 half, 32 half + 32) of S and dP: this thread has already read them
-      if (!kDQ) tmem_st32(tS + 32 * half, pk_p);
-      tmem_st32(tdP + 32 * half, pk_ds);
+      pk_p[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+      pk_ds[e >> 1] = pack_bf16x2(ds[0], ds[1]);
     }
+    // packed into the first 32 columns of S and dP: this thread has already read them
+    if (!kDQ) tmem_st32(tS, pk_p);
+    tmem_st32(tdP, pk_ds);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(bars.p_full);
+    if (lane == 0) mbar_arrive(bars.p_full(h));
   }
   if (!ok) return;
   ok = __all_sync(0xffffffffu, mbar_wait(bars.acc_full, 0, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err));
@@ -366,9 +394,9 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   bars.res_full = bar0;
   bars.full0 = bar0 + 8;
   bars.empty0 = bars.full0 + 8 * C::kStages;
-  bars.st_full = bars.empty0 + 8 * C::kStages;
-  bars.p_full = bars.st_full + 8;
-  bars.acc_full = bars.p_full + 8;
+  bars.st_full0 = bars.empty0 + 8 * C::kStages;
+  bars.p_full0 = bars.st_full0 + 16;
+  bars.acc_full = bars.p_full0 + 16;
   bars.drain = bars.acc_full + 8;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
@@ -379,8 +407,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bars.full(s), 1);
       mbar_init(bars.empty(s), 1);
     }
-    mbar_init(bars.st_full, 1);
-    mbar_init(bars.p_full, 4);  // one arrival per row warp
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bars.st_full(b), 1);
+      mbar_init(bars.p_full(b), 4);  // one arrival per row warp
+    }
     mbar_init(bars.acc_full, 1);
     mbar_init(bars.drain, 1);
     *abort_flag = 0;
