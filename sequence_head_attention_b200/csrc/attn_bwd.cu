@@ -13,14 +13,17 @@
 //   bwd_kernel<D, false>  one CTA per (b, h, key tile of 128): K and V stay in shared memory while the
 //                      query tiles stream through a two-slot ring.  Per query tile, on the tensor cores:
 //                      S^T = K Q^T and dP^T = V dO^T (both operands in shared memory, fp32 in TMEM); the
-//                      four row warps turn them into P^T and dS^T (bf16, written back over S^T and dP^T in
+//                      eight row warps turn them into P^T and dS^T (bf16, written back over S^T and dP^T in
 //                      TMEM); then dV += P^T dO and dK += dS^T Q with the left operand read from TMEM.
 //   bwd_kernel<D, true>   one CTA per (b, h, query tile): Q and dO stay, key tiles stream; S = Q K^T and
 //                      dP = dO V^T, then dS, then dQ += dS K.
-//   Warps: 0 TMA producer, 1 MMA issuer (one elected lane), 2-3 idle, 4-7 the 128 tile rows (one row per
-//   thread: the TMEM lane quadrant of warp w is w % 4).  TMEM: S [0,128), dP [128,256), accumulators
-//   from 256 (dV then dK, or dQ).  The MMA issuer queues the next tile's S and dP right behind the
-//   previous tile's accumulating MMAs: tcgen05 MMAs from one thread execute in order, so the new S cannot
+//   Streamed tiles are taken in halves of 64 rows, alternating between two TMEM buffers, so the tensor
+//   cores compute one half while the row warps work on the other.
+//   Warps: 0 TMA producer, 1 MMA issuer (one elected lane), 2-3 idle, 4-11 the 128 tile rows (one row per
+//   thread; the TMEM lane quadrant of warp w is w % 4, and warps w and w + 4 take 32 columns each of a
+//   half).  TMEM: buffer b holds S at [128 b, 128 b + 64) and dP at [128 b + 64, 128 b + 128);
+//   accumulators from 256 (dV then dK, or dQ).  The MMA issuer queues a half's S and dP right behind the
+//   previous half's accumulating MMAs: tcgen05 MMAs from one thread execute in order, so a new S cannot
 //   overwrite P before it has been read.
 // Every barrier wait is bounded in time; on expiry the kernel records an error and returns cleanly.
 #include <cuda_bf16.h>
@@ -35,8 +38,9 @@ namespace spattn {
 namespace {
 
 constexpr int kBT = 128;           // tile edge
-constexpr int kBwdThreads = 256;   // 8 warps
+constexpr int kBwdThreads = 384;   // 12 warps
 constexpr int kWarpLoad = 0, kWarpIssue = 1, kWarpRow0 = 4;
+constexpr int kRowWarps = 8;       // two per TMEM lane quadrant, 32 columns of a 64-row half each
 
 template <int D>
 struct BCfg {
@@ -74,6 +78,10 @@ struct BwdBars {
 // at columns [128 b, 128 b + 128); accumulators from 256.
 __device__ __forceinline__ uint32_t tS_of(uint32_t t, int b) { return t + 128u * b; }
 __device__ __forceinline__ uint32_t tdP_of(uint32_t t, int b) { return t + 128u * b + 64u; }
+// The row warp of columns [32 j, 32 j + 32) of a half packs their bf16 P (dS) into the 16 columns at 32 j of
+// the S (dP) region, columns it has itself just read.  K-step kk (16 rows of the half) of an accumulating
+// MMA therefore starts at packed column 32 (kk / 2) + 8 (kk % 2).
+__device__ __forceinline__ uint32_t packed_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
 
 // The CTA's tile and the range of streamed tiles it walks.
 struct BwdItem {
@@ -128,22 +136,32 @@ __device__ void bwd_load(const BwdParams& p, const BwdMaps& tm, const BwdItem& i
   for (int n = 0; n < it.n_steps && ok; ++n) {
     const int s = n % C::kStages;
     const int lap = n / C::kStages;
+    const int t = it.first + n;
+    // the streamed query tile's lse (in log2 units) and delta, one per column of S^T, read before the
+    // wait for the slot so that their latency hides behind it; rows past S get lse = +inf, so their
+    // probabilities are exactly 0
+    float l2v[kBT / 32], dlv[kBT / 32];
+    if (!kDQ) {
+      const size_t base = ((size_t)it.b * p.H + it.h) * p.S;
+#pragma unroll
+      for (int j = 0; j < kBT / 32; ++j) {
+        const int row = t * kBT + lane + 32 * j;
+        l2v[j] = row < p.S ? __ldg(p.lse + base + row) * 1.4426950408889634f : INFINITY;
+        dlv[j] = row < p.S ? __ldg(p.delta + base + row) : 0.f;
+      }
+    }
     if (lap > 0) {
       ok = warp_mbar_wait(bars.empty(s), (lap - 1) & 1, tmo, ERR_TIMEOUT_KV_EMPTY, abort_flag, p.err);
       if (!ok) break;
     }
-    const int t = it.first + n;
     const uint32_t stage = sbase + C::kStageOff + s * C::kStageBytes;
     if (!kDQ) {
-      // the streamed query tile's lse (in log2 units) and delta, one per column of S^T; rows past S get
-      // lse = +inf, so their probabilities are exactly 0
       float* lse2 = reinterpret_cast<float*>(smem + C::kStageOff + s * C::kStageBytes + 2 * C::kTileBytes);
       float* dlt = lse2 + kBT;
-      const size_t base = ((size_t)it.b * p.H + it.h) * p.S;
-      for (int r = lane; r < kBT; r += 32) {
-        const int row = t * kBT + r;
-        lse2[r] = row < p.S ? __ldg(p.lse + base + row) * 1.4426950408889634f : INFINITY;
-        dlt[r] = row < p.S ? __ldg(p.delta + base + row) : 0.f;
+#pragma unroll
+      for (int j = 0; j < kBT / 32; ++j) {
+        lse2[lane + 32 * j] = l2v[j];
+        dlt[lane + 32 * j] = dlv[j];
       }
       __threadfence_block();
       __syncwarp();
@@ -192,15 +210,18 @@ __device__ void bwd_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase,
       // dQ += dS K
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_ts(tAcc0, tdP_of(tmem, hh) + kk * 8, str0_mn + (uint64_t)(kk * 128), C::kIdescAcc, (first && kk == 0) ? 0u : 1u);
+        mma_ts(tAcc0, tdP_of(tmem, hh) + packed_col(kk), str0_mn + (uint64_t)(kk * 128), C::kIdescAcc,
+               (first && kk == 0) ? 0u : 1u);
     } else {
       // dV += P^T dO, dK += dS^T Q
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_ts(tAcc0, tS_of(tmem, hh) + kk * 8, str1_mn + (uint64_t)(kk * 128), C::kIdescAcc, (first && kk == 0) ? 0u : 1u);
+        mma_ts(tAcc0, tS_of(tmem, hh) + packed_col(kk), str1_mn + (uint64_t)(kk * 128), C::kIdescAcc,
+               (first && kk == 0) ? 0u : 1u);
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk)
-        mma_ts(tAcc1, tdP_of(tmem, hh) + kk * 8, str0_mn + (uint64_t)(kk * 128), C::kIdescAcc, (first && kk == 0) ? 0u : 1u);
+        mma_ts(tAcc1, tdP_of(tmem, hh) + packed_col(kk), str0_mn + (uint64_t)(kk * 128), C::kIdescAcc,
+               (first && kk == 0) ? 0u : 1u);
     }
     if (hh == 1) mma_commit(bars.empty(nn % C::kStages));  // both halves of the tile consumed
   };
@@ -257,6 +278,43 @@ __device__ void bwd_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase,
 }
 
 // ------------------------------------------------------------------------------------------------
+// P and dS of 32 columns (streamed-tile rows c0 .. c0 + 31) of this thread's row, packed to bf16 pairs.
+// dK/dV: per-column lse (log2 units) and delta from shared memory; column c is kept when c >= lo.
+// dQ: the row's lse and delta; column c is kept when c < hi.  kMask false: every column is kept.
+template <bool kDQ, bool kMask>
+__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float sl2,
+                                          float lse2_row, float dlt_row, const float* lse2, const float* dlt,
+                                          int c0, int lo, int hi, uint32_t (&pk_p)[16], uint32_t (&pk_ds)[16]) {
+#pragma unroll
+  for (int e = 0; e < 32; e += 4) {
+    float l4[4], d4[4];
+    if (kDQ) {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) { l4[u] = lse2_row; d4[u] = dlt_row; }
+    } else {
+      const float4 lv = *reinterpret_cast<const float4*>(lse2 + c0 + e);
+      const float4 dv = *reinterpret_cast<const float4*>(dlt + c0 + e);
+      l4[0] = lv.x; l4[1] = lv.y; l4[2] = lv.z; l4[3] = lv.w;
+      d4[0] = dv.x; d4[1] = dv.y; d4[2] = dv.z; d4[3] = dv.w;
+    }
+    float pr[4], ds[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float pv = ex2_approx(__uint_as_float(s[e + u]) * sl2 - l4[u]);
+      if (kMask) {
+        const int c = c0 + e + u;
+        if (kDQ ? c >= hi : c < lo) pv = 0.f;
+      }
+      pr[u] = pv;
+      ds[u] = pv * (__uint_as_float(dp[e + u]) - d4[u]);
+    }
+    pk_p[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+    pk_p[(e >> 1) + 1] = pack_bf16x2(pr[2], pr[3]);
+    pk_ds[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+    pk_ds[(e >> 1) + 1] = pack_bf16x2(ds[2], ds[3]);
+  }
+}
+
 template <int D, bool kDQ>
 __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, uint32_t tmem, const BwdBars& bars,
                          volatile int* abort_flag) {
@@ -264,6 +322,7 @@ __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, u
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int quad = warp & 3;
+  const int j = (warp - kWarpRow0) >> 2;                         // this warp's 32 columns of each half
   const int r = quad * 32 + lane;                                // row of the resident tile
   const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
   const uint32_t tAcc0 = trow + 256, tAcc1 = trow + 256 + D;
@@ -299,40 +358,25 @@ __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, u
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     tc_fence_after();
-    const uint32_t tS = trow + 128u * h, tdP = tS + 64;
-    uint32_t s[2][32], dp[2][32];
-    tmem_ld32(tS, s[0]);
-    tmem_ld32(tS + 32, s[1]);
-    tmem_ld32(tdP, dp[0]);
-    tmem_ld32(tdP + 32, dp[1]);
+    const uint32_t tS = trow + 128u * h + 32u * j, tdP = tS + 64;
+    uint32_t s[32], dp[32];
+    tmem_ld32(tS, s);
+    tmem_ld32(tdP, dp);
+    const int c0 = 64 * h + 32 * j;  // first column: the streamed tile's row
+    // kept columns: dK/dV, queries t kBT + c not before the key (causal); dQ, keys t kBT + c not after the
+    // query (causal) and inside the key range
+    const int lo = (!kDQ && p.causal) ? row - t * kBT : INT_MIN;
+    const int hi = kDQ ? min(p.causal ? row - t * kBT + 1 : INT_MAX, kv_lim - t * kBT) : INT_MAX;
+    const bool edge = kDQ ? hi < c0 + 32 : lo > c0;
+    uint32_t pk_p[16], pk_ds[16];
     tmem_wait_ld();
-    uint32_t pk_p[32], pk_ds[32];
-#pragma unroll
-    for (int e = 0; e < 64; e += 2) {
-      float pr[2], ds[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int c = 64 * h + e + u;  // column: the streamed tile's row
-        const float sv = __uint_as_float(s[(e + u) >> 5][(e + u) & 31]);
-        const float dv = __uint_as_float(dp[(e + u) >> 5][(e + u) & 31]);
-        float pv;
-        if (kDQ) {
-          pv = ex2_approx(sv * sl2 - lse2_row);
-          if ((p.causal && t * kBT + c > row) || t * kBT + c >= kv_lim) pv = 0.f;  // key after the query, or outside the range
-          ds[u] = pv * (dv - dlt_row);
-        } else {
-          pv = ex2_approx(sv * sl2 - lse2[c]);
-          if (p.causal && t * kBT + c < row) pv = 0.f;  // query before the key
-          ds[u] = pv * (dv - dlt[c]);
-        }
-        pr[u] = pv;
-      }
-      pk_p[e >> 1] = pack_bf16x2(pr[0], pr[1]);
-      pk_ds[e >> 1] = pack_bf16x2(ds[0], ds[1]);
-    }
-    // packed into the first 32 columns of S and dP: this thread has already read them
-    if (!kDQ) tmem_st32(tS, pk_p);
-    tmem_st32(tdP, pk_ds);
+    if (edge)
+      bwd_chunk<kDQ, true>(s, dp, sl2, lse2_row, dlt_row, lse2, dlt, c0, lo, hi, pk_p, pk_ds);
+    else
+      bwd_chunk<kDQ, false>(s, dp, sl2, lse2_row, dlt_row, lse2, dlt, c0, lo, hi, pk_p, pk_ds);
+    // packed into the first 16 of the 32 columns of S and dP this warp has just read
+    if (!kDQ) tmem_st16(tS, pk_p);
+    tmem_st16(tdP, pk_ds);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
@@ -352,7 +396,7 @@ __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, u
     const float f = (kDQ || which == 1) ? scale : 1.f;
     __nv_bfloat16* dst = static_cast<__nv_bfloat16*>(kDQ ? p.dq : (which == 0 ? p.dv : p.dk));
 #pragma unroll 1
-    for (int c = 0; c < D / 32; ++c) {
+    for (int c = j * (D / 64); c < (j + 1) * (D / 64); ++c) {  // this warp's half of the D columns
       uint32_t a[32];
       tmem_ld32(tacc + c * 32, a);
       tmem_wait_ld();
@@ -409,7 +453,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bars.st_full(b), 1);
-      mbar_init(bars.p_full(b), 4);  // one arrival per row warp
+      mbar_init(bars.p_full(b), kRowWarps);  // one arrival per row warp
     }
     mbar_init(bars.acc_full, 1);
     mbar_init(bars.drain, 1);
