@@ -12,19 +12,24 @@
 //   bwd_delta_kernel   delta = rowsum(dO * O), fp32 [B, H, S] (HBM-bound, 16-byte loads).
 //   bwd_kernel<D, false>  one CTA per (b, h, key tile of 128): K and V stay in shared memory while the
 //                      query tiles stream through a two-slot ring.  Per query tile, on the tensor cores:
-//                      S^T = K Q^T and dP^T = V dO^T (both operands in shared memory, fp32 in TMEM); the
-//                      eight row warps turn them into P^T and dS^T (bf16, written back over S^T and dP^T in
-//                      TMEM); then dV += P^T dO and dK += dS^T Q with the left operand read from TMEM.
-//   bwd_kernel<D, true>   one CTA per (b, h, query tile): Q and dO stay, key tiles stream; S = Q K^T and
-//                      dP = dO V^T, then dS, then dQ += dS K.
-//   Streamed tiles are taken in halves of 64 rows, alternating between two TMEM buffers, so the tensor
-//   cores compute one half while the row warps work on the other.
+//                      S'^T = K Q^T - lse / scale and dP'^T = V dO^T - delta (both operands in shared
+//                      memory, fp32 in TMEM).  The per-query terms enter as one extra K-step of 16: a
+//                      constant left operand with ones in its first three columns times a right operand
+//                      holding each query's value split into three bf16 parts (hi + mid + lo carries the
+//                      fp32 value to about 2^-24 of it), so the row warps need no per-column loads.
+//                      The eight row warps read S' into registers (which frees it for the next tile's
+//                      S', computed meanwhile), turn it into P^T = 2^(S' scale log2 e) and, once dP' is
+//                      in, dS^T = P^T dP'; both go back as bf16 into the dP' region of TMEM, where
+//                      dK += dS^T Q and dV += P^T dO read their left operand.  Q and dO of a ring slot
+//                      are released separately (dK runs first), so the next Q copy starts early.
+//   bwd_kernel<D, true>   one CTA per (b, h, query tile): Q and dO stay, key tiles stream in halves of 64
+//                      rows alternating between two TMEM buffers, so the tensor cores compute one half
+//                      while the row warps work on the other; S = Q K^T and dP = dO V^T, then dS, then
+//                      dQ += dS K.
 //   Warps: 0 TMA producer, 1 MMA issuer (one elected lane), 2-3 idle, 4-11 the 128 tile rows (one row per
-//   thread; the TMEM lane quadrant of warp w is w % 4, and warps w and w + 4 take 32 columns each of a
-//   half).  TMEM: buffer b holds S at [128 b, 128 b + 64) and dP at [128 b + 64, 128 b + 128);
-//   accumulators from 256 (dV then dK, or dQ).  The MMA issuer queues a half's S and dP right behind the
-//   previous half's accumulating MMAs: tcgen05 MMAs from one thread execute in order, so a new S cannot
-//   overwrite P before it has been read.
+//   thread; the TMEM lane quadrant of warp w is w % 4, and warps w and w + 4 take half of the columns
+//   each).  TMEM: dK/dV, S' at [0,128), dP' at [128,256); dQ, buffer b holds S at [128 b, 128 b + 64) and
+//   dP at [128 b + 64, 128 b + 128); accumulators from 256 (dV then dK, or dQ).
 // Every barrier wait is bounded in time; on expiry the kernel records an error and returns cleanly.
 #include <cuda_bf16.h>
 
@@ -41,25 +46,35 @@ constexpr int kBT = 128;           // tile edge
 constexpr int kBwdThreads = 384;   // 12 warps
 constexpr int kWarpLoad = 0, kWarpIssue = 1, kWarpRow0 = 4;
 constexpr int kRowWarps = 8;       // two per TMEM lane quadrant, 32 columns of a 64-row half each
+#ifndef SP_BWD_POLY_PAIRS
+#define SP_BWD_POLY_PAIRS 0            // of every 4 pairs of exponentials, this many run on the FMA pipe
+#endif
+constexpr int kBwdPolyPairs = SP_BWD_POLY_PAIRS;
 
-template <int D>
+template <int D, bool kDQ>
 struct BCfg {
   static constexpr int kSub = D / 64;
   static constexpr int kTileBytes = kBT * D * 2;
   static constexpr int kStages = 2;
-  // resident tiles (K, V or Q, dO) at [0, 2 tiles); then per slot: two streamed tiles and 2 x 128 floats
+  // dK/dV: the per-query terms of S' and dP' as the right operand of one K-step (128 rows x 16 bf16,
+  // 32-byte swizzle), and the constant left operand of that step
+  static constexpr int kAugBytes = kBT * 32;
+  // resident tiles (K, V or Q, dO) at [0, 2 tiles); dK/dV: the constant operand; then per slot the two
+  // streamed tiles, and (dK/dV) the lse and delta operands
   static constexpr int kResOff = 0;
-  static constexpr int kStageOff = 2 * kTileBytes;
-  static constexpr int kStageBytes = 2 * kTileBytes + 1024;
+  static constexpr int kOnesOff = 2 * kTileBytes;
+  static constexpr int kStageOff = 2 * kTileBytes + (kDQ ? 0 : 1024 * ((kAugBytes + 1023) / 1024));
+  static constexpr int kStageBytes = 2 * kTileBytes + (kDQ ? 0 : 2 * kAugBytes);
   static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
-  // res_full, full[S], empty[S], st_full[2], p_full[2], acc_full, drain
-  static constexpr int kNumBars = 1 + 2 * kStages + 6;
+  // res_full, full[S], empty[S], st_full[2], p_full[2], acc_full, drain, full_o[S], empty_o[S]
+  static constexpr int kNumBars = 1 + 4 * kStages + 6;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // one CTA per SM: its TMEM allocation takes all 512 columns
   static constexpr int kRaw = kMiscOff + 16 + 1024;
   static constexpr int kSmemBytes = kRaw > 120 * 1024 ? kRaw : 120 * 1024;
-  static constexpr uint32_t kIdescSq = idesc_bf16_f32(128, 64, false, false);  // S, dP of a 64-row half; K-major
-  static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);    // B operand MN-major
+  // S, dP: a 64-row half of a key tile (dQ) or a whole query tile (dK/dV); K-major operands
+  static constexpr uint32_t kIdescSq = idesc_bf16_f32(128, kDQ ? 64 : 128, false, false);
+  static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);  // B operand MN-major
 };
 
 struct BwdMaps {
@@ -67,21 +82,48 @@ struct BwdMaps {
 };
 
 struct BwdBars {
-  uint32_t res_full, full0, empty0, st_full0, p_full0, acc_full, drain;
+  uint32_t res_full, full0, empty0, st_full0, p_full0, acc_full, drain, full_o0, empty_o0;
+  // slot s of the streamed ring: dQ, its K and V; dK/dV, its Q and lse operand
   __device__ uint32_t full(int s) const { return full0 + 8u * s; }
   __device__ uint32_t empty(int s) const { return empty0 + 8u * s; }
-  __device__ uint32_t st_full(int b) const { return st_full0 + 8u * b; }  // per TMEM buffer
+  // dK/dV: the dO and delta operand of slot s, loaded and released on their own
+  __device__ uint32_t full_o(int s) const { return full_o0 + 8u * s; }
+  __device__ uint32_t empty_o(int s) const { return empty_o0 + 8u * s; }
+  // dQ: per TMEM buffer, S and dP computed / dS stored
+  __device__ uint32_t st_full(int b) const { return st_full0 + 8u * b; }
   __device__ uint32_t p_full(int b) const { return p_full0 + 8u * b; }
+  // dK/dV: S' computed, dP' computed, S' read by every row warp, P and dS stored
+  __device__ uint32_t s_ready() const { return st_full0; }
+  __device__ uint32_t dp_ready() const { return st_full0 + 8u; }
+  __device__ uint32_t s_free() const { return p_full0; }
+  __device__ uint32_t pds_stored() const { return p_full0 + 8u; }
 };
 
 // TMEM: two buffers of a 64-row half of a streamed tile, each S (64 columns) then dP (64 columns): buffer b
 // at columns [128 b, 128 b + 128); accumulators from 256.
 __device__ __forceinline__ uint32_t tS_of(uint32_t t, int b) { return t + 128u * b; }
 __device__ __forceinline__ uint32_t tdP_of(uint32_t t, int b) { return t + 128u * b + 64u; }
-// The row warp of columns [32 j, 32 j + 32) of a half packs their bf16 P (dS) into the 16 columns at 32 j of
-// the S (dP) region, columns it has itself just read.  K-step kk (16 rows of the half) of an accumulating
-// MMA therefore starts at packed column 32 (kk / 2) + 8 (kk % 2).
+// dQ: the row warp of columns [32 j, 32 j + 32) of a half packs their bf16 P (dS) into the 16 columns at
+// 32 j of the S (dP) region, columns it has itself just read.  K-step kk (16 rows of the half) of an
+// accumulating MMA therefore starts at packed column 32 (kk / 2) + 8 (kk % 2).
 __device__ __forceinline__ uint32_t packed_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
+// dK/dV: the row warp of queries [64 j, 64 j + 64) of a tile packs their dS into the 32 columns at 64 j of
+// the dP' region and their P into the 32 after them; K-step kk (16 queries) of dK starts at packed column
+// 64 (kk / 4) + 8 (kk % 4) there, and of dV 32 columns further.
+__device__ __forceinline__ uint32_t packed_col_full(int kk) { return 64u * (kk >> 2) + 8u * (kk & 3); }
+
+// Row r of a 32-byte-swizzled K-major operand of 16 bf16 columns: its 16-byte half holding columns 0-7.
+__device__ __forceinline__ uint32_t sw32_first_half(int r) { return 32u * r + 16u * ((r >> 2) & 1); }
+
+// x as hi + mid + lo, each rounded to bf16, packed as the first three bf16 of a 16-byte row half.
+__device__ __forceinline__ uint4 bf16_split3(float x) {
+  const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+  const float r1 = x - __bfloat162float(hi);
+  const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+  const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+  return make_uint4((uint32_t)__bfloat16_as_ushort(hi) | ((uint32_t)__bfloat16_as_ushort(mid) << 16),
+                    (uint32_t)__bfloat16_as_ushort(lo), 0u, 0u);
+}
 
 // The CTA's tile and the range of streamed tiles it walks.
 struct BwdItem {
@@ -114,7 +156,7 @@ __device__ __forceinline__ BwdItem bwd_item(const BwdParams& p) {
 template <int D, bool kDQ>
 __device__ void bwd_load(const BwdParams& p, const BwdMaps& tm, const BwdItem& it, uint32_t sbase, uint8_t* smem,
                          const BwdBars& bars, volatile int* abort_flag) {
-  using C = BCfg<D>;
+  using C = BCfg<D, kDQ>;
   const int lane = threadIdx.x & 31;
   const uint64_t tmo = p.timeout_ns;
   const CUtensorMap* res0 = kDQ ? &tm.q : &tm.k;     // resident pair
@@ -131,98 +173,107 @@ __device__ void bwd_load(const BwdParams& p, const BwdMaps& tm, const BwdItem& i
     }
   }
   __syncwarp();
-  int issued = 0;
+  int issued = 0, issued_o = 0;  // slots whose (Q / K and V) and (dO) copies were started
   bool ok = true;
   for (int n = 0; n < it.n_steps && ok; ++n) {
     const int s = n % C::kStages;
     const int lap = n / C::kStages;
     const int t = it.first + n;
-    // the streamed query tile's lse (in log2 units) and delta, one per column of S^T, read before the
-    // wait for the slot so that their latency hides behind it; rows past S get lse = +inf, so their
-    // probabilities are exactly 0
-    float l2v[kBT / 32], dlv[kBT / 32];
+    // dK/dV: the streamed query tile's -lse / scale and -delta (the per-query terms of S' and dP'), read
+    // before the wait for the slot so that their latency hides behind it.  Query rows past S (zero-filled
+    // Q and dO) get -1e30, so their probabilities are exactly 0, and delta 0.
+    float lq[kBT / 32], dq[kBT / 32];
     if (!kDQ) {
       const size_t base = ((size_t)it.b * p.H + it.h) * p.S;
+      const float inv_scale = 1.f / p.scale;
 #pragma unroll
       for (int j = 0; j < kBT / 32; ++j) {
         const int row = t * kBT + lane + 32 * j;
-        l2v[j] = row < p.S ? __ldg(p.lse + base + row) * 1.4426950408889634f : INFINITY;
-        dlv[j] = row < p.S ? __ldg(p.delta + base + row) : 0.f;
+        lq[j] = row < p.S ? -__ldg(p.lse + base + row) * inv_scale : -1e30f;
+        dq[j] = row < p.S ? -__ldg(p.delta + base + row) : 0.f;
       }
-    }
-    if (lap > 0) {
-      ok = warp_mbar_wait(bars.empty(s), (lap - 1) & 1, tmo, ERR_TIMEOUT_KV_EMPTY, abort_flag, p.err);
-      if (!ok) break;
     }
     const uint32_t stage = sbase + C::kStageOff + s * C::kStageBytes;
-    if (!kDQ) {
-      float* lse2 = reinterpret_cast<float*>(smem + C::kStageOff + s * C::kStageBytes + 2 * C::kTileBytes);
-      float* dlt = lse2 + kBT;
-#pragma unroll
-      for (int j = 0; j < kBT / 32; ++j) {
-        lse2[lane + 32 * j] = l2v[j];
-        dlt[lane + 32 * j] = dlv[j];
+    if (kDQ) {
+      if (lap > 0) {
+        ok = warp_mbar_wait(bars.empty(s), (lap - 1) & 1, tmo, ERR_TIMEOUT_KV_EMPTY, abort_flag, p.err);
+        if (!ok) break;
       }
-      __threadfence_block();
+      if (elect_one_sync()) {
+        mbar_arrive_expect_tx(bars.full(s), 2 * C::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < C::kSub; ++c) {
+          tma_load_4d(stage + c * 16384, str0, bars.full(s), 64 * c, it.h, t * kBT, it.b);
+          tma_load_4d(stage + C::kTileBytes + c * 16384, str1, bars.full(s), 64 * c, it.h, t * kBT, it.b);
+        }
+      }
       __syncwarp();
-    }
-    if (elect_one_sync()) {
-      mbar_arrive_expect_tx(bars.full(s), 2 * C::kTileBytes);
+      issued = n + 1;
+    } else {
+      // Q with its lse operand, then dO with its delta operand, each once its part of the slot is free
+      // (dK, the last reader of Q, runs before dV, the last reader of dO).  Operand row q: (hi, mid, lo,
+      // 0 ...) in its first 16 bytes; the rest stays zero.
+      uint8_t* aug = smem + C::kStageOff + s * C::kStageBytes + 2 * C::kTileBytes;
 #pragma unroll
-      for (int c = 0; c < C::kSub; ++c) {
-        tma_load_4d(stage + c * 16384, str0, bars.full(s), 64 * c, it.h, t * kBT, it.b);
-        tma_load_4d(stage + C::kTileBytes + c * 16384, str1, bars.full(s), 64 * c, it.h, t * kBT, it.b);
+      for (int part = 0; part < 2; ++part) {
+        const uint32_t full_b = part == 0 ? bars.full(s) : bars.full_o(s);
+        if (lap > 0) {
+          ok = warp_mbar_wait(part == 0 ? bars.empty(s) : bars.empty_o(s), (lap - 1) & 1, tmo, ERR_TIMEOUT_KV_EMPTY,
+                              abort_flag, p.err);
+          if (!ok) break;
+        }
+#pragma unroll
+        for (int j = 0; j < kBT / 32; ++j)
+          *reinterpret_cast<uint4*>(aug + part * C::kAugBytes + sw32_first_half(lane + 32 * j)) =
+              bf16_split3(part == 0 ? lq[j] : dq[j]);
+        fence_proxy_async_smem();  // the tensor cores read them once the full barrier passes them on
+        __syncwarp();
+        if (elect_one_sync()) {
+          mbar_arrive_expect_tx(full_b, C::kTileBytes);
+#pragma unroll
+          for (int c = 0; c < C::kSub; ++c)
+            tma_load_4d(stage + part * C::kTileBytes + c * 16384, part == 0 ? str0 : str1, full_b, 64 * c, it.h,
+                        t * kBT, it.b);
+        }
+        __syncwarp();
+        if (part == 0) issued = n + 1; else issued_o = n + 1;
       }
     }
-    __syncwarp();
-    issued = n + 1;
   }
   if (*abort_flag) {  // no copy may still be landing when the CTA exits: wait (bounded) for the last ones
     warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, nullptr, p.err);
     for (int n = issued > C::kStages ? issued - C::kStages : 0; n < issued; ++n)
       warp_mbar_wait(bars.full(n % C::kStages), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, nullptr, p.err);
+    for (int n = issued_o > C::kStages ? issued_o - C::kStages : 0; n < issued_o; ++n)
+      warp_mbar_wait(bars.full_o(n % C::kStages), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, nullptr, p.err);
   }
 }
 
 // ------------------------------------------------------------------------------------------------
-template <int D, bool kDQ>
-__device__ void bwd_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase, uint32_t tmem_in, const BwdBars& bars,
-                          volatile int* abort_flag) {
-  using C = BCfg<D>;
+// dQ issuer.  Key tiles stream in two halves of 64 rows (sub-step m = 2 n + h, TMEM buffer h): half h
+// starts 8192 bytes into each 64-column sub-tile.  The S and dP of half m are issued before the
+// accumulating MMAs of half m - 1, so the tensor cores run one half while the row warps work on the other.
+template <int D>
+__device__ void dq_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase, uint32_t tmem_in, const BwdBars& bars,
+                         volatile int* abort_flag) {
+  using C = BCfg<D, true>;
   const uint64_t tmo = p.timeout_ns;
   const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_in, 0);
-  const uint32_t tAcc0 = tmem + 256, tAcc1 = tmem + 256 + D;
+  const uint32_t tAcc = tmem + 256;
   // K-major descriptors of K-step 0 (the row-major tiles as the MMAs' K-major operands), and MN-major ones
-  // of the streamed tiles as the right operand of the accumulating MMAs.  Streamed tiles are taken in two
-  // halves of 64 rows (sub-step m = 2 n + h, TMEM buffer h): half h starts 8192 bytes into each 64-column
-  // sub-tile.  The S and dP of half m are issued before the accumulating MMAs of half m - 1, so the tensor
-  // cores run one half while the row warps work on the other.
+  // of the streamed tiles as the right operand of the accumulating MMAs
   const uint64_t res0_k = smem_desc_sw128(sbase + C::kResOff, 16, 1024);
   const uint64_t res1_k = smem_desc_sw128(sbase + C::kResOff + C::kTileBytes, 16, 1024);
   bool ok = warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
-  // accumulating MMAs of half hh of streamed tile nn (rows 64 hh .. 64 hh + 63), from TMEM buffer hh
+  // dQ += dS K over half hh of streamed tile nn (rows 64 hh .. 64 hh + 63), from TMEM buffer hh
   auto accumulate = [&](int nn, int hh) {
     const uint32_t stage = sbase + C::kStageOff + (nn % C::kStages) * C::kStageBytes;
-    const uint64_t str0_mn = smem_desc_sw128(stage, 16384, 1024) + (uint64_t)((8192 * hh) >> 4);
-    const uint64_t str1_mn = smem_desc_sw128(stage + C::kTileBytes, 16384, 1024) + (uint64_t)((8192 * hh) >> 4);
+    const uint64_t k_mn = smem_desc_sw128(stage, 16384, 1024) + (uint64_t)((8192 * hh) >> 4);
     const bool first = nn == 0 && hh == 0;
-    if (kDQ) {
-      // dQ += dS K
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_ts(tAcc0, tdP_of(tmem, hh) + packed_col(kk), str0_mn + (uint64_t)(kk * 128), C::kIdescAcc,
-               (first && kk == 0) ? 0u : 1u);
-    } else {
-      // dV += P^T dO, dK += dS^T Q
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_ts(tAcc0, tS_of(tmem, hh) + packed_col(kk), str1_mn + (uint64_t)(kk * 128), C::kIdescAcc,
-               (first && kk == 0) ? 0u : 1u);
-#pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_ts(tAcc1, tdP_of(tmem, hh) + packed_col(kk), str0_mn + (uint64_t)(kk * 128), C::kIdescAcc,
-               (first && kk == 0) ? 0u : 1u);
-    }
+    for (int kk = 0; kk < 4; ++kk)
+      mma_ts(tAcc, tdP_of(tmem, hh) + packed_col(kk), k_mn + (uint64_t)(kk * 128), C::kIdescAcc,
+             (first && kk == 0) ? 0u : 1u);
     if (hh == 1) mma_commit(bars.empty(nn % C::kStages));  // both halves of the tile consumed
   };
   const int n_sub = 2 * it.n_steps;
@@ -237,7 +288,7 @@ __device__ void bwd_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase,
     const uint64_t str0_k = smem_desc_sw128(stage, 16, 1024) + (uint64_t)((8192 * h) >> 4);
     const uint64_t str1_k = smem_desc_sw128(stage + C::kTileBytes, 16, 1024) + (uint64_t)((8192 * h) >> 4);
     if (elect_one_sync()) {
-      // dK/dV: S^T = K Q_h^T, dP^T = V dO_h^T.   dQ: S = Q K_h^T, dP = dO V_h^T.
+      // S = Q K_h^T, dP = dO V_h^T
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
@@ -251,7 +302,7 @@ __device__ void bwd_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase,
       mma_commit(bars.st_full(h));
     }
     __syncwarp();
-    if (m > 0) {  // the previous half: once its P and dS are in TMEM
+    if (m > 0) {  // the previous half: once its dS is in TMEM
       const int mp = m - 1, hp = mp & 1;
       ok = warp_mbar_wait(bars.p_full(hp), (mp >> 1) & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
       if (!ok) break;
@@ -277,116 +328,143 @@ __device__ void bwd_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase,
   warp_mbar_wait(bars.drain, 0, tmo, ERR_TIMEOUT_DRAIN, nullptr, p.err);
 }
 
-// ------------------------------------------------------------------------------------------------
-// P and dS of 32 columns (streamed-tile rows c0 .. c0 + 31) of this thread's row, packed to bf16 pairs.
-// dK/dV: per-column lse (log2 units) and delta from shared memory; column c is kept when c >= lo.
-// dQ: the row's lse and delta; column c is kept when c < hi.  kMask false: every column is kept.
-template <bool kDQ, bool kMask>
-__device__ __forceinline__ void bwd_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float sl2,
-                                          float lse2_row, float dlt_row, const float* lse2, const float* dlt,
-                                          int c0, int lo, int hi, uint32_t (&pk_p)[16], uint32_t (&pk_ds)[16]) {
+// dK/dV issuer.  Order on the tensor cores: S'(0) dP'(0) | S'(1) dK(0) dV(0) dP'(1) | S'(2) dK(1) ...
+// S'(n+1) is issued as soon as every row warp has read S'(n) into registers, so it runs while they
+// compute P(n); dK(n) and dV(n) wait for P(n) and dS(n), which the row warps pack into the dP' region;
+// dP'(n+1) overwrites them only behind dV(n) (tcgen05 MMAs of one thread run in order).  dK(n) frees
+// the slot's Q, then dV(n) its dO.
+template <int D>
+__device__ void dkdv_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase, uint32_t tmem_in,
+                           const BwdBars& bars, volatile int* abort_flag) {
+  using C = BCfg<D, false>;
+  const uint64_t tmo = p.timeout_ns;
+  const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_in, 0);
+  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 256 + D;
+  const uint64_t k_k = smem_desc_sw128(sbase + C::kResOff, 16, 1024);
+  const uint64_t v_k = smem_desc_sw128(sbase + C::kResOff + C::kTileBytes, 16, 1024);
+  const uint64_t ones = smem_desc_sw32(sbase + C::kOnesOff, 256);
+  auto stage_of = [&](int n) { return sbase + C::kStageOff + (n % C::kStages) * C::kStageBytes; };
+  // S'^T = K Q^T + ones lq^T (lq: -lse / scale in three parts), into TMEM [0, 128)
+  auto issue_s = [&](int n) {
+    const uint32_t st = stage_of(n);
+    const uint64_t q_k = smem_desc_sw128(st, 16, 1024);
+    mma_ss(tS, ones, smem_desc_sw32(st + 2 * C::kTileBytes, 256), C::kIdescSq, 0u);
 #pragma unroll
-  for (int e = 0; e < 32; e += 4) {
-    float l4[4], d4[4];
-    if (kDQ) {
-#pragma unroll
-      for (int u = 0; u < 4; ++u) { l4[u] = lse2_row; d4[u] = dlt_row; }
-    } else {
-      const float4 lv = *reinterpret_cast<const float4*>(lse2 + c0 + e);
-      const float4 dv = *reinterpret_cast<const float4*>(dlt + c0 + e);
-      l4[0] = lv.x; l4[1] = lv.y; l4[2] = lv.z; l4[3] = lv.w;
-      d4[0] = dv.x; d4[1] = dv.y; d4[2] = dv.z; d4[3] = dv.w;
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+      mma_ss(tS, k_k + off, q_k + off, C::kIdescSq, 1u);
     }
-    float pr[4], ds[4];
+    mma_commit(bars.s_ready());
+  };
+  // dP'^T = V dO^T + ones dl^T (dl: -delta in three parts), into TMEM [128, 256)
+  auto issue_dp = [&](int n) {
+    const uint32_t st = stage_of(n);
+    const uint64_t do_k = smem_desc_sw128(st + C::kTileBytes, 16, 1024);
+    mma_ss(tdP, ones, smem_desc_sw32(st + 2 * C::kTileBytes + C::kAugBytes, 256), C::kIdescSq, 0u);
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      float pv = ex2_approx(__uint_as_float(s[e + u]) * sl2 - l4[u]);
-      if (kMask) {
-        const int c = c0 + e + u;
-        if (kDQ ? c >= hi : c < lo) pv = 0.f;
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+      mma_ss(tdP, v_k + off, do_k + off, C::kIdescSq, 1u);
+    }
+    mma_commit(bars.dp_ready());
+  };
+  bool ok = warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
+  const int N = it.n_steps;
+  if (ok && N > 0) {
+    ok = warp_mbar_wait(bars.full(0), 0, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+    if (ok) ok = warp_mbar_wait(bars.full_o(0), 0, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+    if (ok) {
+      tc_fence_after();
+      if (elect_one_sync()) {
+        issue_s(0);
+        issue_dp(0);
       }
-      pr[u] = pv;
-      ds[u] = pv * (__uint_as_float(dp[e + u]) - d4[u]);
+      __syncwarp();
     }
-    pk_p[e >> 1] = pack_bf16x2(pr[0], pr[1]);
-    pk_p[(e >> 1) + 1] = pack_bf16x2(pr[2], pr[3]);
-    pk_ds[e >> 1] = pack_bf16x2(ds[0], ds[1]);
-    pk_ds[(e >> 1) + 1] = pack_bf16x2(ds[2], ds[3]);
+  }
+  for (int n = 0; n < N && ok; ++n) {
+    const uint32_t st = stage_of(n);
+    // K-steps of 16 queries: MN-major right operands, 2048 bytes apart
+    const uint64_t q_mn = smem_desc_sw128(st, 16384, 1024);
+    const uint64_t do_mn = smem_desc_sw128(st + C::kTileBytes, 16384, 1024);
+    if (n + 1 < N) {
+      ok = warp_mbar_wait(bars.s_free(), n & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
+      if (ok)
+        ok = warp_mbar_wait(bars.full((n + 1) % C::kStages), ((n + 1) / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
+                            abort_flag, p.err);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one_sync()) issue_s(n + 1);
+      __syncwarp();
+    }
+    ok = warp_mbar_wait(bars.pds_stored(), n & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
+    if (!ok) break;
+    tc_fence_after();
+    if (elect_one_sync()) {
+      // dK += dS^T Q, then the slot's Q is free; dV += P^T dO, then its dO
+#pragma unroll
+      for (int kk = 0; kk < kBT / 16; ++kk)
+        mma_ts(tdK, tdP + packed_col_full(kk), q_mn + (uint64_t)(kk * 128), C::kIdescAcc, (n == 0 && kk == 0) ? 0u : 1u);
+      mma_commit(bars.empty(n % C::kStages));
+#pragma unroll
+      for (int kk = 0; kk < kBT / 16; ++kk)
+        mma_ts(tdV, tdP + 32 + packed_col_full(kk), do_mn + (uint64_t)(kk * 128), C::kIdescAcc,
+               (n == 0 && kk == 0) ? 0u : 1u);
+      mma_commit(bars.empty_o(n % C::kStages));
+    }
+    __syncwarp();
+    if (n + 1 < N) {
+      ok = warp_mbar_wait(bars.full_o((n + 1) % C::kStages), ((n + 1) / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
+                          abort_flag, p.err);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one_sync()) issue_dp(n + 1);
+      __syncwarp();
+    }
+  }
+  if (ok && elect_one_sync()) mma_commit(bars.acc_full);
+  __syncwarp();
+  // nothing of ours may still run on the tensor cores when TMEM is released
+  if (elect_one_sync()) mma_commit(bars.drain);
+  __syncwarp();
+  warp_mbar_wait(bars.drain, 0, tmo, ERR_TIMEOUT_DRAIN, nullptr, p.err);
+}
+
+// ------------------------------------------------------------------------------------------------
+// dQ rows: P and dS of 32 columns (key-tile rows c0 .. c0 + 31) of this thread's query row, packed to bf16
+// pairs, in the paired (.f32x2) FMA-pipe arithmetic, from the row's -lse (log2 units) and -delta; column
+// c is kept when c < hi (kMask false: every column is kept).  Of every 4 pairs of exponentials,
+// kBwdPolyPairs run through the FMA-pipe polynomial, the rest through ex2.approx.
+template <bool kMask>
+__device__ __forceinline__ void dq_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float sl2,
+                                         float nlse2_row, float ndlt_row, int c0, int hi, uint32_t (&pk_ds)[16]) {
+  const f2 sc = {sl2, sl2};
+  const f2 nl = {nlse2_row, nlse2_row}, nd = {ndlt_row, ndlt_row};
+#pragma unroll
+  for (int i = 0; i < 32; i += 2) {
+    const f2 x = ffma2(f2{__uint_as_float(s[i]), __uint_as_float(s[i + 1])}, sc, nl);
+    f2 pv;
+    if (((i >> 1) & 3) >= 4 - kBwdPolyPairs) {
+      pv = exp2_poly2(x);
+    } else {
+      pv.x = ex2_approx(x.x);
+      pv.y = ex2_approx(x.y);
+    }
+    if (kMask) {
+      if (c0 + i >= hi) pv.x = 0.f;
+      if (c0 + i + 1 >= hi) pv.y = 0.f;
+    }
+    const f2 ds = fmul2(pv, fadd2(f2{__uint_as_float(dp[i]), __uint_as_float(dp[i + 1])}, nd));
+    pk_ds[i >> 1] = pack_bf16x2(ds.x, ds.y);
   }
 }
 
+// Epilogue of the accumulators: this warp's half of the D columns of each, scaled, to bf16 (or added into
+// the fp32 dQ accumulator).
 template <int D, bool kDQ>
-__device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, uint32_t tmem, const BwdBars& bars,
-                         volatile int* abort_flag) {
-  using C = BCfg<D>;
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int quad = warp & 3;
-  const int j = (warp - kWarpRow0) >> 2;                         // this warp's 32 columns of each half
-  const int r = quad * 32 + lane;                                // row of the resident tile
-  const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+__device__ __forceinline__ void bwd_epilogue(const BwdParams& p, const BwdItem& it, uint32_t trow, int j, int row,
+                                             bool row_out) {
   const uint32_t tAcc0 = trow + 256, tAcc1 = trow + 256 + D;
-  const uint64_t tmo = p.timeout_ns;
-  const float sl2 = p.scale_log2;
-  const int row = it.tile * kBT + r;                             // global position of this thread's row
-  const int kv_lim = min(p.kv_end, p.S);
-  // rows this CTA writes: queries < S (dQ); keys of the range (dK, dV)
-  const bool row_out = kDQ ? row < p.S : row < kv_lim;
-  float lse2_row = 0.f, dlt_row = 0.f;
-  if (kDQ && row < p.S) {
-    const size_t i = ((size_t)it.b * p.H + it.h) * p.S + row;
-    lse2_row = __ldg(p.lse + i) * 1.4426950408889634f;
-    dlt_row = __ldg(p.delta + i);
-  }
-  bool ok = true;
-  // sub-step m = 2 n + h: the 64 rows 64 h .. 64 h + 63 of streamed tile n, in TMEM buffer h
-  for (int m = 0; m < 2 * it.n_steps; ++m) {
-    const int n = m >> 1, h = m & 1;
-    const int t = it.first + n;
-    const float* lse2 = reinterpret_cast<const float*>(smem + C::kStageOff + (n % C::kStages) * C::kStageBytes +
-                                                       2 * C::kTileBytes);
-    const float* dlt = lse2 + kBT;
-    if (!kDQ && h == 0) {
-      // lse and delta of the streamed tile were stored by the producer before it released the slot's
-      // full barrier: acquire them from that barrier (the slot is refilled only after both halves' P
-      // arrive, so the phase cannot have moved on)
-      ok = mbar_wait(bars.full(n % C::kStages), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-    }
-    ok = mbar_wait(bars.st_full(h), n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err);
-    ok = __all_sync(0xffffffffu, ok);
-    if (!ok) break;
-    tc_fence_after();
-    const uint32_t tS = trow + 128u * h + 32u * j, tdP = tS + 64;
-    uint32_t s[32], dp[32];
-    tmem_ld32(tS, s);
-    tmem_ld32(tdP, dp);
-    const int c0 = 64 * h + 32 * j;  // first column: the streamed tile's row
-    // kept columns: dK/dV, queries t kBT + c not before the key (causal); dQ, keys t kBT + c not after the
-    // query (causal) and inside the key range
-    const int lo = (!kDQ && p.causal) ? row - t * kBT : INT_MIN;
-    const int hi = kDQ ? min(p.causal ? row - t * kBT + 1 : INT_MAX, kv_lim - t * kBT) : INT_MAX;
-    const bool edge = kDQ ? hi < c0 + 32 : lo > c0;
-    uint32_t pk_p[16], pk_ds[16];
-    tmem_wait_ld();
-    if (edge)
-      bwd_chunk<kDQ, true>(s, dp, sl2, lse2_row, dlt_row, lse2, dlt, c0, lo, hi, pk_p, pk_ds);
-    else
-      bwd_chunk<kDQ, false>(s, dp, sl2, lse2_row, dlt_row, lse2, dlt, c0, lo, hi, pk_p, pk_ds);
-    // packed into the first 16 of the 32 columns of S and dP this warp has just read
-    if (!kDQ) tmem_st16(tS, pk_p);
-    tmem_st16(tdP, pk_ds);
-    tmem_wait_st();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) mbar_arrive(bars.p_full(h));
-  }
-  if (!ok) return;
-  ok = __all_sync(0xffffffffu, mbar_wait(bars.acc_full, 0, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err));
-  if (!ok) return;
-  if (it.n_steps == 0) return;  // (dQ of a key range before this query tile) nothing accumulated
-  tc_fence_after();
   const float scale = p.scale;
   const size_t out = (((size_t)it.b * p.S + row) * p.H + it.h) * D;
 #pragma unroll
@@ -426,10 +504,153 @@ __device__ void bwd_rows(const BwdParams& p, const BwdItem& it, uint8_t* smem, u
   }
 }
 
+template <int D>
+__device__ void dq_rows(const BwdParams& p, const BwdItem& it, uint32_t tmem, const BwdBars& bars,
+                        volatile int* abort_flag) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int quad = warp & 3;
+  const int j = (warp - kWarpRow0) >> 2;                         // this warp's 32 columns of each half
+  const int r = quad * 32 + lane;                                // row of the resident tile
+  const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+  const uint64_t tmo = p.timeout_ns;
+  const float sl2 = p.scale_log2;
+  const int row = it.tile * kBT + r;                             // this thread's query
+  const int kv_lim = min(p.kv_end, p.S);
+  const bool row_out = row < p.S;
+  float nlse2_row = 0.f, ndlt_row = 0.f;  // -lse (log2 units) and -delta of this thread's query
+  if (row < p.S) {
+    const size_t i = ((size_t)it.b * p.H + it.h) * p.S + row;
+    nlse2_row = __ldg(p.lse + i) * -1.4426950408889634f;
+    ndlt_row = -__ldg(p.delta + i);
+  }
+  bool ok = true;
+  // sub-step m = 2 n + h: the 64 rows 64 h .. 64 h + 63 of key tile n, in TMEM buffer h
+  for (int m = 0; m < 2 * it.n_steps; ++m) {
+    const int n = m >> 1, h = m & 1;
+    const int t = it.first + n;
+    ok = mbar_wait(bars.st_full(h), n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    tc_fence_after();
+    const uint32_t tS = trow + 128u * h + 32u * j, tdP = tS + 64;
+    uint32_t s[32], dp[32];
+    tmem_ld32(tS, s);
+    tmem_ld32(tdP, dp);
+    const int c0 = 64 * h + 32 * j;  // first column: the key tile's row
+    // kept columns: keys t kBT + c not after the query (causal) and inside the key range
+    const int hi = min(p.causal ? row - t * kBT + 1 : INT_MAX, kv_lim - t * kBT);
+    uint32_t pk_ds[16];
+    tmem_wait_ld();
+    if (hi < c0 + 32)
+      dq_chunk<true>(s, dp, sl2, nlse2_row, ndlt_row, c0, hi, pk_ds);
+    else
+      dq_chunk<false>(s, dp, sl2, nlse2_row, ndlt_row, c0, hi, pk_ds);
+    // packed into the first 16 of the 32 columns of dP this warp has just read
+    tmem_st16(tdP, pk_ds);
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars.p_full(h));
+  }
+  if (!ok) return;
+  ok = __all_sync(0xffffffffu, mbar_wait(bars.acc_full, 0, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err));
+  if (!ok) return;
+  if (it.n_steps == 0) return;  // (a key range before this query tile) nothing accumulated
+  tc_fence_after();
+  bwd_epilogue<D, true>(p, it, trow, j, row, row_out);
+}
+
+// dK/dV rows: this thread is key `row`; warp j takes queries [64 j, 64 j + 64) of each query tile.
+template <int D>
+__device__ void dkdv_rows(const BwdParams& p, const BwdItem& it, uint32_t tmem, const BwdBars& bars,
+                          volatile int* abort_flag) {
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int quad = warp & 3;
+  const int j = (warp - kWarpRow0) >> 2;
+  const int r = quad * 32 + lane;
+  const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+  const uint32_t tS = trow + 64u * j, tdP = trow + 128u + 64u * j;
+  const uint64_t tmo = p.timeout_ns;
+  const f2 sc = {p.scale_log2, p.scale_log2};
+  const int row = it.tile * kBT + r;
+  const bool row_out = row < min(p.kv_end, p.S);
+  bool ok = true;
+  for (int n = 0; n < it.n_steps; ++n) {
+    const int t = it.first + n;
+    ok = __all_sync(0xffffffffu, mbar_wait(bars.s_ready(), n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err));
+    if (!ok) break;
+    tc_fence_after();
+    // P = 2^(S' scale log2 e) over this warp's 64 queries; causal: queries before the key get 0.  S' is
+    // released to the next tile's MMA as soon as it is in registers.
+    float pf[64];
+    {
+      uint32_t s[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.s_free());
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) {
+        const f2 x = fmul2(f2{__uint_as_float(s[i]), __uint_as_float(s[i + 1])}, sc);
+        f2 pv;
+        if (((i >> 1) & 3) >= 4 - kBwdPolyPairs) {
+          pv = exp2_poly2(x);
+        } else {
+          pv.x = ex2_approx(x.x);
+          pv.y = ex2_approx(x.y);
+        }
+        pf[i] = pv.x;
+        pf[i + 1] = pv.y;
+      }
+    }
+    const int lo = p.causal ? row - t * kBT : INT_MIN;  // kept: query column c >= lo
+    if (lo > 64 * j) {
+#pragma unroll
+      for (int i = 0; i < 64; ++i)
+        if (64 * j + i < lo) pf[i] = 0.f;
+    }
+    // dS = P dP' in two chunks of 32 queries, packed over columns already read; then P after them
+    ok = __all_sync(0xffffffffu, mbar_wait(bars.dp_ready(), n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err));
+    if (!ok) break;
+    tc_fence_after();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t d[32], pk[16];
+      tmem_ld32(tdP + 32 * h, d);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const f2 ds = fmul2(f2{pf[32 * h + i], pf[32 * h + i + 1]}, f2{__uint_as_float(d[i]), __uint_as_float(d[i + 1])});
+        pk[i >> 1] = pack_bf16x2(ds.x, ds.y);
+      }
+      tmem_st16(tdP + 16 * h, pk);
+    }
+    {
+      uint32_t pk[32];
+#pragma unroll
+      for (int i = 0; i < 64; i += 2) pk[i >> 1] = pack_bf16x2(pf[i], pf[i + 1]);
+      tmem_st32(tdP + 32, pk);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars.pds_stored());
+  }
+  if (!ok) return;
+  ok = __all_sync(0xffffffffu, mbar_wait(bars.acc_full, 0, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err));
+  if (!ok) return;
+  tc_fence_after();
+  bwd_epilogue<D, false>(p, it, trow, j, row, row_out);
+}
+
 template <int D, bool kDQ>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     bwd_kernel(const __grid_constant__ BwdMaps tm, const __grid_constant__ BwdParams p) {
-  using C = BCfg<D>;
+  using C = BCfg<D, kDQ>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -442,6 +663,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   bars.p_full0 = bars.st_full0 + 16;
   bars.acc_full = bars.p_full0 + 16;
   bars.drain = bars.acc_full + 8;
+  bars.full_o0 = bars.drain + 8;
+  bars.empty_o0 = bars.full_o0 + 8 * C::kStages;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   const int warp = threadIdx.x >> 5;
@@ -450,6 +673,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bars.full(s), 1);
       mbar_init(bars.empty(s), 1);
+      mbar_init(bars.full_o(s), 1);
+      mbar_init(bars.empty_o(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bars.st_full(b), 1);
@@ -470,6 +695,22 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     tmem_alloc(smem_u32(tmem_holder), 512);
     tmem_relinquish();
   }
+  if (!kDQ) {
+    // the constant operand (rows 1, 1, 1, 0 ...), and zeros in the per-query operands of both slots (the
+    // producer rewrites only the first three columns of each row)
+    for (int i = threadIdx.x; i < kBT * 2; i += kBwdThreads) {
+      const int r = i >> 1, half = i & 1;
+      const uint32_t at = sw32_first_half(r) ^ (half ? 16u : 0u);
+      *reinterpret_cast<uint4*>(smem + C::kOnesOff + at) =
+          half ? make_uint4(0u, 0u, 0u, 0u) : make_uint4(0x3F803F80u, 0x00003F80u, 0u, 0u);
+    }
+    for (int i = threadIdx.x; i < C::kStages * 2 * C::kAugBytes / 16; i += kBwdThreads) {
+      const int s = i / (2 * C::kAugBytes / 16), rem = i % (2 * C::kAugBytes / 16);
+      *reinterpret_cast<uint4*>(smem + C::kStageOff + s * C::kStageBytes + 2 * C::kTileBytes + 16 * rem) =
+          make_uint4(0u, 0u, 0u, 0u);
+    }
+    fence_proxy_async_smem();
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -478,9 +719,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   if (warp == kWarpLoad) {
     bwd_load<D, kDQ>(p, tm, it, sbase, smem, bars, abort_flag);
   } else if (warp == kWarpIssue) {
-    bwd_issue<D, kDQ>(p, it, sbase, tmem, bars, abort_flag);
+    if (kDQ)
+      dq_issue<D>(p, it, sbase, tmem, bars, abort_flag);
+    else
+      dkdv_issue<D>(p, it, sbase, tmem, bars, abort_flag);
   } else if (warp >= kWarpRow0) {
-    bwd_rows<D, kDQ>(p, it, smem, tmem, bars, abort_flag);
+    if (kDQ)
+      dq_rows<D>(p, it, tmem, bars, abort_flag);
+    else
+      dkdv_rows<D>(p, it, tmem, bars, abort_flag);
   }
   tc_fence_before();
   __syncthreads();
@@ -536,7 +783,7 @@ __global__ void __launch_bounds__(256) f32_to_bf16_kernel(const float4* __restri
 
 template <int D, bool kDQ>
 sp_status launch_bwd_one(const BwdMaps& tm, const BwdParams& p, int grid, cudaStream_t stream) {
-  using C = BCfg<D>;
+  using C = BCfg<D, kDQ>;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SP_ERR_CUDA;
   static bool attr_set[kMaxDevices] = {};
