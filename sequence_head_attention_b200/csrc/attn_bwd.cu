@@ -55,15 +55,17 @@ template <int D, bool kDQ>
 struct BCfg {
   static constexpr int kSub = D / 64;
   static constexpr int kTileBytes = kBT * D * 2;
-  static constexpr int kStages = 2;
+  // dQ keeps its resident Q and dO in TMEM, so its shared memory holds three slots of the K/V ring
+  static constexpr int kStages = kDQ ? 3 : 2;
   // dK/dV: the per-query terms of S' and dP' as the right operand of one K-step (128 rows x 16 bf16,
   // 32-byte swizzle), and the constant left operand of that step
   static constexpr int kAugBytes = kBT * 32;
-  // resident tiles (K, V or Q, dO) at [0, 2 tiles); dK/dV: the constant operand; then per slot the two
-  // streamed tiles, and (dK/dV) the lse and delta operands
+  // dK/dV: resident K and V at [0, 2 tiles), then the constant operand; then per slot the two streamed
+  // tiles, and (dK/dV) the lse and delta operands
   static constexpr int kResOff = 0;
-  static constexpr int kOnesOff = 2 * kTileBytes;
-  static constexpr int kStageOff = 2 * kTileBytes + (kDQ ? 0 : 1024 * ((kAugBytes + 1023) / 1024));
+  static constexpr int kResBytes = kDQ ? 0 : 2 * kTileBytes;
+  static constexpr int kOnesOff = kResBytes;
+  static constexpr int kStageOff = kResBytes + (kDQ ? 0 : 1024 * ((kAugBytes + 1023) / 1024));
   static constexpr int kStageBytes = 2 * kTileBytes + (kDQ ? 0 : 2 * kAugBytes);
   static constexpr int kBarOff = kStageOff + kStages * kStageBytes;
   // res_full, full[S], empty[S], st_full[2], p_full[2], acc_full, drain, full_o[S], empty_o[S]
@@ -163,7 +165,7 @@ __device__ void bwd_load(const BwdParams& p, const BwdMaps& tm, const BwdItem& i
   const CUtensorMap* res1 = kDQ ? &tm.dout : &tm.v;
   const CUtensorMap* str0 = kDQ ? &tm.k : &tm.q;     // streamed pair
   const CUtensorMap* str1 = kDQ ? &tm.v : &tm.dout;
-  if (elect_one_sync()) {
+  if (!kDQ && elect_one_sync()) {
     mbar_arrive_expect_tx(bars.res_full, 2 * C::kTileBytes);
 #pragma unroll
     for (int c = 0; c < C::kSub; ++c) {
@@ -241,7 +243,7 @@ __device__ void bwd_load(const BwdParams& p, const BwdMaps& tm, const BwdItem& i
     }
   }
   if (*abort_flag) {  // no copy may still be landing when the CTA exits: wait (bounded) for the last ones
-    warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, nullptr, p.err);
+    if (!kDQ) warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, nullptr, p.err);
     for (int n = issued > C::kStages ? issued - C::kStages : 0; n < issued; ++n)
       warp_mbar_wait(bars.full(n % C::kStages), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, nullptr, p.err);
     for (int n = issued_o > C::kStages ? issued_o - C::kStages : 0; n < issued_o; ++n)
@@ -259,11 +261,8 @@ __device__ void dq_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase, 
   using C = BCfg<D, true>;
   const uint64_t tmo = p.timeout_ns;
   const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_in, 0);
-  const uint32_t tAcc = tmem + 256;
-  // K-major descriptors of K-step 0 (the row-major tiles as the MMAs' K-major operands), and MN-major ones
-  // of the streamed tiles as the right operand of the accumulating MMAs
-  const uint64_t res0_k = smem_desc_sw128(sbase + C::kResOff, 16, 1024);
-  const uint64_t res1_k = smem_desc_sw128(sbase + C::kResOff + C::kTileBytes, 16, 1024);
+  const uint32_t tAcc = tmem + 256, tQ = tmem + 256 + D, tdO = tQ + D / 2;
+  // the row warps have put Q and dO (bf16 pairs) into TMEM: the left operands of S and dP
   bool ok = warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
   // dQ += dS K over half hh of streamed tile nn (rows 64 hh .. 64 hh + 63), from TMEM buffer hh
   auto accumulate = [&](int nn, int hh) {
@@ -288,16 +287,16 @@ __device__ void dq_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase, 
     const uint64_t str0_k = smem_desc_sw128(stage, 16, 1024) + (uint64_t)((8192 * h) >> 4);
     const uint64_t str1_k = smem_desc_sw128(stage + C::kTileBytes, 16, 1024) + (uint64_t)((8192 * h) >> 4);
     if (elect_one_sync()) {
-      // S = Q K_h^T, dP = dO V_h^T
+      // S = Q K_h^T, dP = dO V_h^T: left operand from TMEM (8 columns per K-step of 16)
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
-        mma_ss(tS_of(tmem, h), res0_k + off, str0_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
+        mma_ts(tS_of(tmem, h), tQ + 8 * kk, str0_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
       }
 #pragma unroll
       for (int kk = 0; kk < D / 16; ++kk) {
         const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
-        mma_ss(tdP_of(tmem, h), res1_k + off, str1_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
+        mma_ts(tdP_of(tmem, h), tdO + 8 * kk, str1_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
       }
       mma_commit(bars.st_full(h));
     }
@@ -524,6 +523,30 @@ __device__ void dq_rows(const BwdParams& p, const BwdItem& it, uint32_t tmem, co
     nlse2_row = __ldg(p.lse + i) * -1.4426950408889634f;
     ndlt_row = -__ldg(p.delta + i);
   }
+  {
+    // this thread's query row of Q and dO, half j of the D columns, into TMEM (zeros past S): the left
+    // operands of S and dP for every key tile
+    const uint32_t tQ = trow + 256 + D + (D / 4) * j, tdO = tQ + D / 2;
+    const size_t src = (((size_t)it.b * p.S + row) * p.H + it.h) * D + (D / 2) * j;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const uint4* g = reinterpret_cast<const uint4*>(static_cast<const __nv_bfloat16*>(which ? p.dout : p.q) + src);
+      uint32_t v[D / 4];
+#pragma unroll
+      for (int e = 0; e < D / 16; ++e) {
+        const uint4 x = row < p.S ? __ldg(g + e) : make_uint4(0u, 0u, 0u, 0u);
+        v[4 * e] = x.x; v[4 * e + 1] = x.y; v[4 * e + 2] = x.z; v[4 * e + 3] = x.w;
+      }
+      if (D == 128)
+        tmem_st32(which ? tdO : tQ, *reinterpret_cast<uint32_t(*)[32]>(&v[0]));
+      else
+        tmem_st16(which ? tdO : tQ, *reinterpret_cast<uint32_t(*)[16]>(&v[0]));
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bars.res_full);
+  }
   bool ok = true;
   // sub-step m = 2 n + h: the 64 rows 64 h .. 64 h + 63 of key tile n, in TMEM buffer h
   for (int m = 0; m < 2 * it.n_steps; ++m) {
@@ -561,6 +584,29 @@ __device__ void dq_rows(const BwdParams& p, const BwdItem& it, uint32_t tmem, co
   bwd_epilogue<D, true>(p, it, trow, j, row, row_out);
 }
 
+// P = 2^(S' scale log2 e) of 64 queries; kMask: queries i < lo get 0.  Of every 4 pairs of exponentials,
+// kBwdPolyPairs run through the FMA-pipe polynomial, the rest through ex2.approx.
+template <bool kMask>
+__device__ __forceinline__ void dkdv_p(const uint32_t (&s)[64], float (&pf)[64], f2 sc, int lo) {
+#pragma unroll
+  for (int i = 0; i < 64; i += 2) {
+    const f2 x = fmul2(f2{__uint_as_float(s[i]), __uint_as_float(s[i + 1])}, sc);
+    f2 pv;
+    if (((i >> 1) & 3) >= 4 - kBwdPolyPairs) {
+      pv = exp2_poly2(x);
+    } else {
+      pv.x = ex2_approx(x.x);
+      pv.y = ex2_approx(x.y);
+    }
+    if (kMask) {
+      if (i < lo) pv.x = 0.f;
+      if (i + 1 < lo) pv.y = 0.f;
+    }
+    pf[i] = pv.x;
+    pf[i + 1] = pv.y;
+  }
+}
+
 // dK/dV rows: this thread is key `row`; warp j takes queries [64 j, 64 j + 64) of each query tile.
 template <int D>
 __device__ void dkdv_rows(const BwdParams& p, const BwdItem& it, uint32_t tmem, const BwdBars& bars,
@@ -593,25 +639,11 @@ __device__ void dkdv_rows(const BwdParams& p, const BwdItem& it, uint32_t tmem, 
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bars.s_free());
-#pragma unroll
-      for (int i = 0; i < 64; i += 2) {
-        const f2 x = fmul2(f2{__uint_as_float(s[i]), __uint_as_float(s[i + 1])}, sc);
-        f2 pv;
-        if (((i >> 1) & 3) >= 4 - kBwdPolyPairs) {
-          pv = exp2_poly2(x);
-        } else {
-          pv.x = ex2_approx(x.x);
-          pv.y = ex2_approx(x.y);
-        }
-        pf[i] = pv.x;
-        pf[i + 1] = pv.y;
-      }
-    }
-    const int lo = p.causal ? row - t * kBT : INT_MIN;  // kept: query column c >= lo
-    if (lo > 64 * j) {
-#pragma unroll
-      for (int i = 0; i < 64; ++i)
-        if (64 * j + i < lo) pf[i] = 0.f;
+      const int lo = p.causal ? row - t * kBT - 64 * j : INT_MIN;  // kept: this warp's query i >= lo
+      if (lo > 0)
+        dkdv_p<true>(s, pf, sc, lo);
+      else
+        dkdv_p<false>(s, pf, sc, lo);
     }
     // dS = P dP' in two chunks of 32 queries, packed over columns already read; then P after them
     ok = __all_sync(0xffffffffu, mbar_wait(bars.dp_ready(), n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err));
@@ -669,7 +701,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   const int warp = threadIdx.x >> 5;
   if (threadIdx.x == 0) {
-    mbar_init(bars.res_full, 1);
+    mbar_init(bars.res_full, kDQ ? kRowWarps : 1);  // dQ: every row warp's Q and dO in TMEM
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(bars.full(s), 1);
       mbar_init(bars.empty(s), 1);
@@ -802,6 +834,8 @@ sp_status launch_bwd_one(const BwdMaps& tm, const BwdParams& p, int grid, cudaSt
 sp_status launch_attn_bwd(const BwdParams& p_in, const void* q, const void* k, const void* v, const void* o,
                           const void* dout, cudaStream_t stream) {
   BwdParams p = p_in;
+  p.q = q;
+  p.dout = dout;
   BwdMaps tm;
   if (!encode_bshd_tmap(&tm.q, q, p.B, p.S, p.H, p.D) || !encode_bshd_tmap(&tm.k, k, p.B, p.S, p.H, p.D) ||
       !encode_bshd_tmap(&tm.v, v, p.B, p.S, p.H, p.D) || !encode_bshd_tmap(&tm.dout, dout, p.B, p.S, p.H, p.D))

@@ -65,6 +65,8 @@ struct BwdParams {
   void* dk;
   void* dv;
   float* dq_acc;      // non-null: dq is not written; this launch's dQ contribution is added here (fp32 BSHD)
+  const void* q;      // bf16 BSHD inputs read directly by the dQ kernel (its resident operands)
+  const void* dout;
   int kv_begin;       // keys [kv_begin, kv_end) only (one KV block of a ring); kv_begin a multiple of 128
   int kv_end;
   int kt0, n_kt;      // their key tiles: kt0 .. kt0 + n_kt - 1
