@@ -22,14 +22,14 @@
 //                      in, dS^T = P^T dP'; both go back as bf16 into the dP' region of TMEM, where
 //                      dK += dS^T Q and dV += P^T dO read their left operand.  Q and dO of a ring slot
 //                      are released separately (dK runs first), so the next Q copy starts early.
-//   bwd_kernel<D, true>   one CTA per (b, h, query tile): Q and dO stay, key tiles stream in halves of 64
-//                      rows alternating between two TMEM buffers, so the tensor cores compute one half
-//                      while the row warps work on the other; S = Q K^T and dP = dO V^T, then dS, then
-//                      dQ += dS K.
+//   bwd_kernel<D, true>   one CTA per (b, h, query tile): the row warps copy the tile's Q and dO rows into
+//                      TMEM once, as the left operands of S = Q K^T and dP = dO V^T; key tiles stream
+//                      through a three-slot ring, with the same early release of S as above, and
+//                      dQ += dS K reads dS from TMEM.
 //   Warps: 0 TMA producer, 1 MMA issuer (one elected lane), 2-3 idle, 4-11 the 128 tile rows (one row per
 //   thread; the TMEM lane quadrant of warp w is w % 4, and warps w and w + 4 take half of the columns
-//   each).  TMEM: dK/dV, S' at [0,128), dP' at [128,256); dQ, buffer b holds S at [128 b, 128 b + 64) and
-//   dP at [128 b + 64, 128 b + 128); accumulators from 256 (dV then dK, or dQ).
+//   each).  TMEM: S (S') at [0,128), dP (dP') at [128,256), accumulators from 256 (dV then dK, or dQ),
+//   and, dQ, the resident Q and dO after its accumulator.
 // Every barrier wait is bounded in time; on expiry the kernel records an error and returns cleanly.
 #include <cuda_bf16.h>
 
@@ -45,7 +45,7 @@ namespace {
 constexpr int kBT = 128;           // tile edge
 constexpr int kBwdThreads = 384;   // 12 warps
 constexpr int kWarpLoad = 0, kWarpIssue = 1, kWarpRow0 = 4;
-constexpr int kRowWarps = 8;       // two per TMEM lane quadrant, 32 columns of a 64-row half each
+constexpr int kRowWarps = 8;       // two per TMEM lane quadrant, 64 columns of a streamed tile each
 #ifndef SP_BWD_POLY_PAIRS
 #define SP_BWD_POLY_PAIRS 0            // of every 4 pairs of exponentials, this many run on the FMA pipe
 #endif
@@ -74,8 +74,8 @@ struct BCfg {
   // one CTA per SM: its TMEM allocation takes all 512 columns
   static constexpr int kRaw = kMiscOff + 16 + 1024;
   static constexpr int kSmemBytes = kRaw > 120 * 1024 ? kRaw : 120 * 1024;
-  // S, dP: a 64-row half of a key tile (dQ) or a whole query tile (dK/dV); K-major operands
-  static constexpr uint32_t kIdescSq = idesc_bf16_f32(128, kDQ ? 64 : 128, false, false);
+  // S, dP over a whole streamed tile; K-major operands
+  static constexpr uint32_t kIdescSq = idesc_bf16_f32(128, 128, false, false);
   static constexpr uint32_t kIdescAcc = idesc_bf16_f32(128, D, false, true);  // B operand MN-major
 };
 
@@ -91,27 +91,16 @@ struct BwdBars {
   // dK/dV: the dO and delta operand of slot s, loaded and released on their own
   __device__ uint32_t full_o(int s) const { return full_o0 + 8u * s; }
   __device__ uint32_t empty_o(int s) const { return empty_o0 + 8u * s; }
-  // dQ: per TMEM buffer, S and dP computed / dS stored
-  __device__ uint32_t st_full(int b) const { return st_full0 + 8u * b; }
-  __device__ uint32_t p_full(int b) const { return p_full0 + 8u * b; }
-  // dK/dV: S' computed, dP' computed, S' read by every row warp, P and dS stored
+  // S (S') computed, dP (dP') computed, S read by every row warp, dS (and P) stored
   __device__ uint32_t s_ready() const { return st_full0; }
   __device__ uint32_t dp_ready() const { return st_full0 + 8u; }
   __device__ uint32_t s_free() const { return p_full0; }
   __device__ uint32_t pds_stored() const { return p_full0 + 8u; }
 };
 
-// TMEM: two buffers of a 64-row half of a streamed tile, each S (64 columns) then dP (64 columns): buffer b
-// at columns [128 b, 128 b + 128); accumulators from 256.
-__device__ __forceinline__ uint32_t tS_of(uint32_t t, int b) { return t + 128u * b; }
-__device__ __forceinline__ uint32_t tdP_of(uint32_t t, int b) { return t + 128u * b + 64u; }
-// dQ: the row warp of columns [32 j, 32 j + 32) of a half packs their bf16 P (dS) into the 16 columns at
-// 32 j of the S (dP) region, columns it has itself just read.  K-step kk (16 rows of the half) of an
-// accumulating MMA therefore starts at packed column 32 (kk / 2) + 8 (kk % 2).
-__device__ __forceinline__ uint32_t packed_col(int kk) { return 32u * (kk >> 1) + 8u * (kk & 1); }
-// dK/dV: the row warp of queries [64 j, 64 j + 64) of a tile packs their dS into the 32 columns at 64 j of
-// the dP' region and their P into the 32 after them; K-step kk (16 queries) of dK starts at packed column
-// 64 (kk / 4) + 8 (kk % 4) there, and of dV 32 columns further.
+// The row warp of columns [64 j, 64 j + 64) of a streamed tile packs their dS into the 32 columns at 64 j
+// of the dP region (and, dK/dV, their P into the 32 after them); K-step kk (16 streamed rows) of the
+// accumulating MMA starts at packed column 64 (kk / 4) + 8 (kk % 4) there, or 32 columns further for P.
 __device__ __forceinline__ uint32_t packed_col_full(int kk) { return 64u * (kk >> 2) + 8u * (kk & 3); }
 
 // Row r of a 32-byte-swizzled K-major operand of 16 bf16 columns: its 16-byte half holding columns 0-7.
@@ -196,50 +185,36 @@ __device__ void bwd_load(const BwdParams& p, const BwdMaps& tm, const BwdItem& i
       }
     }
     const uint32_t stage = sbase + C::kStageOff + s * C::kStageBytes;
-    if (kDQ) {
+    // Part 0 of the slot (dK/dV: Q with its lse operand; dQ: K), then part 1 (dK/dV: dO with its delta
+    // operand; dQ: V), each once its own reader has released it: dK (or dQ) is the last reader of part 0,
+    // dV (or dP) of part 1.  dK/dV operand row q: (hi, mid, lo, 0 ...) in its first 16 bytes; the rest
+    // stays zero.
+    uint8_t* aug = smem + C::kStageOff + s * C::kStageBytes + 2 * C::kTileBytes;
+#pragma unroll
+    for (int part = 0; part < 2; ++part) {
+      const uint32_t full_b = part == 0 ? bars.full(s) : bars.full_o(s);
       if (lap > 0) {
-        ok = warp_mbar_wait(bars.empty(s), (lap - 1) & 1, tmo, ERR_TIMEOUT_KV_EMPTY, abort_flag, p.err);
+        ok = warp_mbar_wait(part == 0 ? bars.empty(s) : bars.empty_o(s), (lap - 1) & 1, tmo, ERR_TIMEOUT_KV_EMPTY,
+                            abort_flag, p.err);
         if (!ok) break;
       }
-      if (elect_one_sync()) {
-        mbar_arrive_expect_tx(bars.full(s), 2 * C::kTileBytes);
-#pragma unroll
-        for (int c = 0; c < C::kSub; ++c) {
-          tma_load_4d(stage + c * 16384, str0, bars.full(s), 64 * c, it.h, t * kBT, it.b);
-          tma_load_4d(stage + C::kTileBytes + c * 16384, str1, bars.full(s), 64 * c, it.h, t * kBT, it.b);
-        }
-      }
-      __syncwarp();
-      issued = n + 1;
-    } else {
-      // Q with its lse operand, then dO with its delta operand, each once its part of the slot is free
-      // (dK, the last reader of Q, runs before dV, the last reader of dO).  Operand row q: (hi, mid, lo,
-      // 0 ...) in its first 16 bytes; the rest stays zero.
-      uint8_t* aug = smem + C::kStageOff + s * C::kStageBytes + 2 * C::kTileBytes;
-#pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        const uint32_t full_b = part == 0 ? bars.full(s) : bars.full_o(s);
-        if (lap > 0) {
-          ok = warp_mbar_wait(part == 0 ? bars.empty(s) : bars.empty_o(s), (lap - 1) & 1, tmo, ERR_TIMEOUT_KV_EMPTY,
-                              abort_flag, p.err);
-          if (!ok) break;
-        }
+      if (!kDQ) {
 #pragma unroll
         for (int j = 0; j < kBT / 32; ++j)
           *reinterpret_cast<uint4*>(aug + part * C::kAugBytes + sw32_first_half(lane + 32 * j)) =
               bf16_split3(part == 0 ? lq[j] : dq[j]);
         fence_proxy_async_smem();  // the tensor cores read them once the full barrier passes them on
         __syncwarp();
-        if (elect_one_sync()) {
-          mbar_arrive_expect_tx(full_b, C::kTileBytes);
-#pragma unroll
-          for (int c = 0; c < C::kSub; ++c)
-            tma_load_4d(stage + part * C::kTileBytes + c * 16384, part == 0 ? str0 : str1, full_b, 64 * c, it.h,
-                        t * kBT, it.b);
-        }
-        __syncwarp();
-        if (part == 0) issued = n + 1; else issued_o = n + 1;
       }
+      if (elect_one_sync()) {
+        mbar_arrive_expect_tx(full_b, C::kTileBytes);
+#pragma unroll
+        for (int c = 0; c < C::kSub; ++c)
+          tma_load_4d(stage + part * C::kTileBytes + c * 16384, part == 0 ? str0 : str1, full_b, 64 * c, it.h,
+                      t * kBT, it.b);
+      }
+      __syncwarp();
+      if (part == 0) issued = n + 1; else issued_o = n + 1;
     }
   }
   if (*abort_flag) {  // no copy may still be landing when the CTA exits: wait (bounded) for the last ones
@@ -252,70 +227,81 @@ __device__ void bwd_load(const BwdParams& p, const BwdMaps& tm, const BwdItem& i
 }
 
 // ------------------------------------------------------------------------------------------------
-// dQ issuer.  Key tiles stream in two halves of 64 rows (sub-step m = 2 n + h, TMEM buffer h): half h
-// starts 8192 bytes into each 64-column sub-tile.  The S and dP of half m are issued before the
-// accumulating MMAs of half m - 1, so the tensor cores run one half while the row warps work on the other.
+// dQ issuer.  Order on the tensor cores: S(0) dP(0) | S(1) dQ(0) dP(1) | S(2) dQ(1) dP(2) | ...
+// S = Q K^T and dP = dO V^T take their left operand (Q, dO) from TMEM.  S(n+1) is issued as soon as every
+// row warp has read S(n); dQ(n) += dS(n) K(n) waits for dS(n), which the row warps pack into the dP
+// region, and dP(n+1) overwrites it only behind dQ(n).  dP(n) frees the slot's V, dQ(n) its K.
 template <int D>
 __device__ void dq_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase, uint32_t tmem_in, const BwdBars& bars,
                          volatile int* abort_flag) {
   using C = BCfg<D, true>;
   const uint64_t tmo = p.timeout_ns;
   const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_in, 0);
-  const uint32_t tAcc = tmem + 256, tQ = tmem + 256 + D, tdO = tQ + D / 2;
-  // the row warps have put Q and dO (bf16 pairs) into TMEM: the left operands of S and dP
-  bool ok = warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
-  // dQ += dS K over half hh of streamed tile nn (rows 64 hh .. 64 hh + 63), from TMEM buffer hh
-  auto accumulate = [&](int nn, int hh) {
-    const uint32_t stage = sbase + C::kStageOff + (nn % C::kStages) * C::kStageBytes;
-    const uint64_t k_mn = smem_desc_sw128(stage, 16384, 1024) + (uint64_t)((8192 * hh) >> 4);
-    const bool first = nn == 0 && hh == 0;
+  const uint32_t tS = tmem, tdP = tmem + 128, tAcc = tmem + 256, tQ = tmem + 256 + D, tdO = tQ + D / 2;
+  auto stage_of = [&](int n) { return sbase + C::kStageOff + (n % C::kStages) * C::kStageBytes; };
+  auto issue_s = [&](int n) {  // S = Q K^T, left operand from TMEM (8 columns per K-step of 16)
+    const uint64_t k_k = smem_desc_sw128(stage_of(n), 16, 1024);
 #pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_ts(tAcc, tdP_of(tmem, hh) + packed_col(kk), k_mn + (uint64_t)(kk * 128), C::kIdescAcc,
-             (first && kk == 0) ? 0u : 1u);
-    if (hh == 1) mma_commit(bars.empty(nn % C::kStages));  // both halves of the tile consumed
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+      mma_ts(tS, tQ + 8 * kk, k_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(bars.s_ready());
   };
-  const int n_sub = 2 * it.n_steps;
-  for (int m = 0; m < n_sub && ok; ++m) {
-    const int n = m >> 1, h = m & 1;
-    if (h == 0) {
-      ok = warp_mbar_wait(bars.full(n % C::kStages), (n / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
-      if (!ok) break;
-      tc_fence_after();
-    }
-    const uint32_t stage = sbase + C::kStageOff + (n % C::kStages) * C::kStageBytes;
-    const uint64_t str0_k = smem_desc_sw128(stage, 16, 1024) + (uint64_t)((8192 * h) >> 4);
-    const uint64_t str1_k = smem_desc_sw128(stage + C::kTileBytes, 16, 1024) + (uint64_t)((8192 * h) >> 4);
-    if (elect_one_sync()) {
-      // S = Q K_h^T, dP = dO V_h^T: left operand from TMEM (8 columns per K-step of 16)
+  auto issue_dp = [&](int n) {  // dP = dO V^T; then the slot's V is free
+    const uint64_t v_k = smem_desc_sw128(stage_of(n) + C::kTileBytes, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
-        mma_ts(tS_of(tmem, h), tQ + 8 * kk, str0_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
-      }
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
-        mma_ts(tdP_of(tmem, h), tdO + 8 * kk, str1_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(bars.st_full(h));
+    for (int kk = 0; kk < D / 16; ++kk) {
+      const uint64_t off = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+      mma_ts(tdP, tdO + 8 * kk, v_k + off, C::kIdescSq, kk > 0 ? 1u : 0u);
     }
-    __syncwarp();
-    if (m > 0) {  // the previous half: once its dS is in TMEM
-      const int mp = m - 1, hp = mp & 1;
-      ok = warp_mbar_wait(bars.p_full(hp), (mp >> 1) & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
-      if (!ok) break;
+    mma_commit(bars.dp_ready());
+    mma_commit(bars.empty_o(n % C::kStages));
+  };
+  // the row warps have put Q and dO (bf16 pairs) into TMEM
+  bool ok = warp_mbar_wait(bars.res_full, 0, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
+  const int N = it.n_steps;
+  if (ok && N > 0) {
+    ok = warp_mbar_wait(bars.full(0), 0, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+    if (ok) ok = warp_mbar_wait(bars.full_o(0), 0, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+    if (ok) {
       tc_fence_after();
-      if (elect_one_sync()) accumulate(mp >> 1, hp);
+      if (elect_one_sync()) {
+        issue_s(0);
+        issue_dp(0);
+      }
       __syncwarp();
     }
   }
-  if (ok && n_sub > 0) {  // the last half
-    const int mp = n_sub - 1, hp = mp & 1;
-    ok = warp_mbar_wait(bars.p_full(hp), (mp >> 1) & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
-    if (ok) {
+  for (int n = 0; n < N && ok; ++n) {
+    if (n + 1 < N) {
+      ok = warp_mbar_wait(bars.s_free(), n & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
+      if (ok)
+        ok = warp_mbar_wait(bars.full((n + 1) % C::kStages), ((n + 1) / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
+                            abort_flag, p.err);
+      if (!ok) break;
       tc_fence_after();
-      if (elect_one_sync()) accumulate(mp >> 1, hp);
+      if (elect_one_sync()) issue_s(n + 1);
+      __syncwarp();
+    }
+    ok = warp_mbar_wait(bars.pds_stored(), n & 1, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
+    if (!ok) break;
+    tc_fence_after();
+    if (elect_one_sync()) {  // dQ += dS K (K-steps of 16 keys: MN-major K, 2048 bytes apart)
+      const uint64_t k_mn = smem_desc_sw128(stage_of(n), 16384, 1024);
+#pragma unroll
+      for (int kk = 0; kk < kBT / 16; ++kk)
+        mma_ts(tAcc, tdP + packed_col_full(kk), k_mn + (uint64_t)(kk * 128), C::kIdescAcc,
+               (n == 0 && kk == 0) ? 0u : 1u);
+      mma_commit(bars.empty(n % C::kStages));
+    }
+    __syncwarp();
+    if (n + 1 < N) {
+      ok = warp_mbar_wait(bars.full_o((n + 1) % C::kStages), ((n + 1) / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
+                          abort_flag, p.err);
+      if (!ok) break;
+      tc_fence_after();
+      if (elect_one_sync()) issue_dp(n + 1);
       __syncwarp();
     }
   }
@@ -430,34 +416,6 @@ __device__ void dkdv_issue(const BwdParams& p, const BwdItem& it, uint32_t sbase
 }
 
 // ------------------------------------------------------------------------------------------------
-// dQ rows: P and dS of 32 columns (key-tile rows c0 .. c0 + 31) of this thread's query row, packed to bf16
-// pairs, in the paired (.f32x2) FMA-pipe arithmetic, from the row's -lse (log2 units) and -delta; column
-// c is kept when c < hi (kMask false: every column is kept).  Of every 4 pairs of exponentials,
-// kBwdPolyPairs run through the FMA-pipe polynomial, the rest through ex2.approx.
-template <bool kMask>
-__device__ __forceinline__ void dq_chunk(const uint32_t (&s)[32], const uint32_t (&dp)[32], float sl2,
-                                         float nlse2_row, float ndlt_row, int c0, int hi, uint32_t (&pk_ds)[16]) {
-  const f2 sc = {sl2, sl2};
-  const f2 nl = {nlse2_row, nlse2_row}, nd = {ndlt_row, ndlt_row};
-#pragma unroll
-  for (int i = 0; i < 32; i += 2) {
-    const f2 x = ffma2(f2{__uint_as_float(s[i]), __uint_as_float(s[i + 1])}, sc, nl);
-    f2 pv;
-    if (((i >> 1) & 3) >= 4 - kBwdPolyPairs) {
-      pv = exp2_poly2(x);
-    } else {
-      pv.x = ex2_approx(x.x);
-      pv.y = ex2_approx(x.y);
-    }
-    if (kMask) {
-      if (c0 + i >= hi) pv.x = 0.f;
-      if (c0 + i + 1 >= hi) pv.y = 0.f;
-    }
-    const f2 ds = fmul2(pv, fadd2(f2{__uint_as_float(dp[i]), __uint_as_float(dp[i + 1])}, nd));
-    pk_ds[i >> 1] = pack_bf16x2(ds.x, ds.y);
-  }
-}
-
 // Epilogue of the accumulators: this warp's half of the D columns of each, scaled, to bf16 (or added into
 // the fp32 dQ accumulator).
 template <int D, bool kDQ>
@@ -503,17 +461,43 @@ __device__ __forceinline__ void bwd_epilogue(const BwdParams& p, const BwdItem& 
   }
 }
 
+// dQ rows: P = 2^(S scale log2 e - lse log2 e) of 64 keys from this query row's -lse (log2 units); keys
+// c >= hi get 0 (kMask).  Of every 4 pairs of exponentials, kBwdPolyPairs run through the FMA-pipe
+// polynomial, the rest through ex2.approx.
+template <bool kMask>
+__device__ __forceinline__ void dq_p(const uint32_t (&s)[64], float (&pf)[64], f2 sc, f2 nl, int hi) {
+#pragma unroll
+  for (int i = 0; i < 64; i += 2) {
+    const f2 x = ffma2(f2{__uint_as_float(s[i]), __uint_as_float(s[i + 1])}, sc, nl);
+    f2 pv;
+    if (((i >> 1) & 3) >= 4 - kBwdPolyPairs) {
+      pv = exp2_poly2(x);
+    } else {
+      pv.x = ex2_approx(x.x);
+      pv.y = ex2_approx(x.y);
+    }
+    if (kMask) {
+      if (i >= hi) pv.x = 0.f;
+      if (i + 1 >= hi) pv.y = 0.f;
+    }
+    pf[i] = pv.x;
+    pf[i + 1] = pv.y;
+  }
+}
+
+// dQ rows: this thread is query `row`; warp j takes keys [64 j, 64 j + 64) of each key tile.
 template <int D>
 __device__ void dq_rows(const BwdParams& p, const BwdItem& it, uint32_t tmem, const BwdBars& bars,
                         volatile int* abort_flag) {
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int quad = warp & 3;
-  const int j = (warp - kWarpRow0) >> 2;                         // this warp's 32 columns of each half
-  const int r = quad * 32 + lane;                                // row of the resident tile
+  const int j = (warp - kWarpRow0) >> 2;
+  const int r = quad * 32 + lane;
   const uint32_t trow = tmem + ((uint32_t)(quad * 32) << 16);
+  const uint32_t tS = trow + 64u * j, tdP = trow + 128u + 64u * j;
   const uint64_t tmo = p.timeout_ns;
-  const float sl2 = p.scale_log2;
+  const f2 sc = {p.scale_log2, p.scale_log2};
   const int row = it.tile * kBT + r;                             // this thread's query
   const int kv_lim = min(p.kv_end, p.S);
   const bool row_out = row < p.S;
@@ -547,34 +531,50 @@ __device__ void dq_rows(const BwdParams& p, const BwdItem& it, uint32_t tmem, co
     __syncwarp();
     if (lane == 0) mbar_arrive(bars.res_full);
   }
+  const f2 nl = {nlse2_row, nlse2_row}, nd = {ndlt_row, ndlt_row};
   bool ok = true;
-  // sub-step m = 2 n + h: the 64 rows 64 h .. 64 h + 63 of key tile n, in TMEM buffer h
-  for (int m = 0; m < 2 * it.n_steps; ++m) {
-    const int n = m >> 1, h = m & 1;
+  for (int n = 0; n < it.n_steps; ++n) {
     const int t = it.first + n;
-    ok = mbar_wait(bars.st_full(h), n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err);
-    ok = __all_sync(0xffffffffu, ok);
+    ok = __all_sync(0xffffffffu, mbar_wait(bars.s_ready(), n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err));
     if (!ok) break;
     tc_fence_after();
-    const uint32_t tS = trow + 128u * h + 32u * j, tdP = tS + 64;
-    uint32_t s[32], dp[32];
-    tmem_ld32(tS, s);
-    tmem_ld32(tdP, dp);
-    const int c0 = 64 * h + 32 * j;  // first column: the key tile's row
-    // kept columns: keys t kBT + c not after the query (causal) and inside the key range
-    const int hi = min(p.causal ? row - t * kBT + 1 : INT_MAX, kv_lim - t * kBT);
-    uint32_t pk_ds[16];
-    tmem_wait_ld();
-    if (hi < c0 + 32)
-      dq_chunk<true>(s, dp, sl2, nlse2_row, ndlt_row, c0, hi, pk_ds);
-    else
-      dq_chunk<false>(s, dp, sl2, nlse2_row, ndlt_row, c0, hi, pk_ds);
-    // packed into the first 16 of the 32 columns of dP this warp has just read
-    tmem_st16(tdP, pk_ds);
+    float pf[64];
+    {
+      uint32_t s[64];
+      tmem_ld32(tS, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bars.s_free());
+      // kept: keys t kBT + 64 j + i not after the query (causal) and inside the key range
+      const int hi = min(p.causal ? row - t * kBT + 1 : INT_MAX, kv_lim - t * kBT) - 64 * j;
+      if (hi < 64)
+        dq_p<true>(s, pf, sc, nl, hi);
+      else
+        dq_p<false>(s, pf, sc, nl, hi);
+    }
+    // dS = P (dP - delta) in two chunks of 32 keys, packed over columns already read
+    ok = __all_sync(0xffffffffu, mbar_wait(bars.dp_ready(), n & 1, tmo, ERR_TIMEOUT_S_FULL, abort_flag, p.err));
+    if (!ok) break;
+    tc_fence_after();
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t d[32], pk[16];
+      tmem_ld32(tdP + 32 * h, d);
+      tmem_wait_ld();
+#pragma unroll
+      for (int i = 0; i < 32; i += 2) {
+        const f2 ds = fmul2(f2{pf[32 * h + i], pf[32 * h + i + 1]},
+                            fadd2(f2{__uint_as_float(d[i]), __uint_as_float(d[i + 1])}, nd));
+        pk[i >> 1] = pack_bf16x2(ds.x, ds.y);
+      }
+      tmem_st16(tdP + 16 * h, pk);
+    }
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(bars.p_full(h));
+    if (lane == 0) mbar_arrive(bars.pds_stored());
   }
   if (!ok) return;
   ok = __all_sync(0xffffffffu, mbar_wait(bars.acc_full, 0, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err));
@@ -708,10 +708,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
       mbar_init(bars.full_o(s), 1);
       mbar_init(bars.empty_o(s), 1);
     }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(bars.st_full(b), 1);
-      mbar_init(bars.p_full(b), kRowWarps);  // one arrival per row warp
-    }
+    mbar_init(bars.s_ready(), 1);
+    mbar_init(bars.dp_ready(), 1);
+    mbar_init(bars.s_free(), kRowWarps);  // one arrival per row warp
+    mbar_init(bars.pds_stored(), kRowWarps);
     mbar_init(bars.acc_full, 1);
     mbar_init(bars.drain, 1);
     *abort_flag = 0;
