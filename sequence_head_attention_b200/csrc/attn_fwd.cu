@@ -128,12 +128,14 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p, int w) {
   while (c + 1 < p.n_chunks && w >= p.chunk_item0[c + 1]) ++c;
   const int r = w - p.chunk_item0[c];
   const int hc = p.chunk_h0[c + 1] - p.chunk_h0[c];
-  const int per_b = hc * p.n_qpairs;
+  // (a causal partial launch has no items for the leading p.qp_skip pairs, which no key reaches)
+  const int n_run = p.n_qpairs - p.qp_skip;
+  const int per_b = hc * n_run;
   Item it;
   it.b = r / per_b;
   const int r2 = r - it.b * per_b;
-  it.h = p.chunk_h0[c] + r2 / p.n_qpairs;
-  const int qq = r2 % p.n_qpairs;
+  it.h = p.chunk_h0[c] + r2 / n_run;
+  const int qq = r2 % n_run;
   it.qp = (p.causal && !p.item_list) ? (p.n_qpairs - 1 - qq) : qq;
   // Query tiles are laid on each shard's own 128-row grid (one shard: the global grid); a shard's last
   // tile may be short, and items never cross shards.  An item is a pair of tiles, or for a CTA pair four:
@@ -986,6 +988,31 @@ static sp_status launch_kernel(const TMaps& tm, const AttnParams& p, int grid, c
   return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
 }
 
+// Rows [0, rows) of heads [h0, h1) of every batch: O = 0 (16-byte stores; each head's D values are 128 or
+// 256 bytes) and lse = -inf.  For the query rows of a causal partial launch that no key of its range
+// reaches.
+__global__ void __launch_bounds__(256) fill_empty_rows_kernel(void* __restrict__ o, int o_elem_bytes,
+                                                              float* __restrict__ lse, int B, int S, int H, int D,
+                                                              int h0, int h1, int rows) {
+  const long long per_row = (long long)(h1 - h0) * D * o_elem_bytes / 16;  // 16-byte chunks per (b, s)
+  const long long n_o = (long long)B * rows * per_row;
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_o; i += stride) {
+    const long long bs = i / per_row, c = i % per_row;
+    const long long b = bs / rows, s = bs % rows;
+    uint8_t* row = static_cast<uint8_t*>(o) + (((b * S + s) * H + h0) * (long long)D) * o_elem_bytes;
+    reinterpret_cast<uint4*>(row)[c] = make_uint4(0u, 0u, 0u, 0u);
+  }
+  if (lse) {
+    const long long n_l = (long long)B * (h1 - h0) * rows;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n_l; i += stride) {
+      const long long bh = i / rows, s = i % rows;
+      const long long b = bh / (h1 - h0), h = h0 + bh % (h1 - h0);
+      lse[(b * H + h) * S + s] = -INFINITY;
+    }
+  }
+}
+
 sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
   AttnParams p = p_in;
   if (p.n_shards < 1 || p.n_shards > kMaxShards || p.shard_rows < 1 || (long long)p.n_shards * p.shard_rows != p.S ||
@@ -1014,6 +1041,31 @@ sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
     }
     p.chunk_item0[p.n_chunks] = (int)items;
     if (items > 0x7fffffffLL) return SP_ERR_INVALID_ARG;
+    p.n_items = (int)items;
+  }
+  // A causal launch over keys from kv_begin: queries before kv_begin see none of them.  Whole leading
+  // work units of such rows get no item; their rows are written here (O = 0, lse = -inf) at HBM speed.
+  p.qp_skip = 0;
+  if (p.causal && p.kv_begin > 0 && p.n_shards == 1 && !p.item_list && !p.row_ptr) {
+    const int unit_rows = (pair ? 4 : 2) * kTile;
+    p.qp_skip = p.kv_begin / unit_rows < p.n_qpairs ? p.kv_begin / unit_rows : p.n_qpairs;
+    const int rows = p.qp_skip * unit_rows < p.S ? p.qp_skip * unit_rows : p.S;
+    if (rows > 0) {
+      const int h0 = p.chunk_h0[0], h1 = p.chunk_h0[p.n_chunks];
+      const long long n = (long long)p.B * rows * (h1 - h0) * p.D * (p.o_f32 ? 4 : 2) / 16;
+      long long blocks = (n + 255) / 256;
+      if (blocks > (long long)sms * 8) blocks = (long long)sms * 8;
+      if (blocks < 1) blocks = 1;
+      fill_empty_rows_kernel<<<(int)blocks, 256, 0, stream>>>(p.o, p.o_f32 ? 4 : 2, p.lse, p.B, p.S, p.H, p.D, h0, h1,
+                                                              rows);
+      if (cudaGetLastError() != cudaSuccess) return SP_ERR_CUDA;
+    }
+    long long items = 0;
+    for (int c = 0; c < p.n_chunks; ++c) {
+      p.chunk_item0[c] = (int)items;
+      items += (long long)p.B * (p.chunk_h0[c + 1] - p.chunk_h0[c]) * (p.n_qpairs - p.qp_skip);
+    }
+    p.chunk_item0[p.n_chunks] = (int)items;
     p.n_items = (int)items;
   }
   if (p.n_items <= 0) return SP_OK;

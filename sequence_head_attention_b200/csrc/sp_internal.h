@@ -18,7 +18,9 @@ constexpr int kMaxShards = SP_MAX_SHARDS;  // sequence shards one attention laun
 struct AttnParams {
   int B, S, H, D;
   int n_qpairs;     // ceil(ceil(S/128) / 2): work items per (b, h)
-  int n_items;      // B * H * n_qpairs
+  int n_items;      // B * H * (n_qpairs - qp_skip)
+  int qp_skip;      // causal partial launches: leading query pairs per (b, h) that no key of the range
+                    // reaches; they get no work item (their rows are filled with O = 0, lse = -inf)
   int kv_begin;     // first key position
   int kv_lim;       // one past the last key position (<= S)
   int n_kv_tiles;   // ceil((kv_lim - kv_begin) / 128)
