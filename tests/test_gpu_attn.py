@@ -97,6 +97,23 @@ def test_partial_block(kv, causal):
         assert np.all(oe == 0)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("kv", [(1100, 1500), (512, 1024), (1400, 1401)])
+def test_causal_partial_rows_before_block(D, kv):
+    """A causal block over keys [kv_begin, kv_end): query rows before kv_begin see no key.  Whole work
+    units of them are not run but filled (O = 0, lse = -inf), batch by batch; every other row matches."""
+    B, S, H = 2, 1500, 3
+    q, k, v = synth.qkv(B, S, H, D, seed=kv[0] + D, scale=0.5)
+    ref = ref_attn(q, k, v, causal=True, kv_begin=kv[0], kv_end=kv[1])
+    o = torch.full((B, S, H, D), float("nan"), device="cuda")
+    lse = torch.full((B, H, S), float("nan"), device="cuda")
+    spattn.sp_attn_fwd_partial(q.cuda(), k.cuda(), v.cuda(), o, lse, kv[0], kv[1], causal=True)
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    assert_close(o, ref[0], lse, ref[1])
+    oc, lc = o.cpu().numpy(), lse.cpu().numpy()
+    assert np.all(oc[:, :kv[0]] == 0) and np.all(np.isneginf(lc[:, :, :kv[0]]))
+
+
 @pytest.mark.parametrize("n_kv", [2, 3, 8])
 @pytest.mark.parametrize("causal", [False, True])
 def test_kv_blocks_merge_equals_unsplit(n_kv, causal):
