@@ -7,7 +7,8 @@
 //   seq -> head:  out_r[b, s, h', :] = in_{s / (S/P)}[b, s % (S/P), r H/P + h', :]
 //   head -> seq:  out_r[b, s', h, :] = in_{h / (H/P)}[b, r S/P + s', h % (H/P), :]
 // Both directions move contiguous runs of (H/P) * D elements: one warp copies one run with 16-byte
-// vector loads and stores (streaming cache hints), so both sides are fully coalesced.  Bit-exact.
+// vector loads and stores, up to 4 KB per lane group in flight, so both sides are fully coalesced.
+// Bit-exact.
 #include <cstdint>
 
 #include "sp_internal.h"
@@ -50,17 +51,26 @@ __global__ void __launch_bounds__(256) relayout_kernel(const __grid_constant__ R
       src = rp.in[g] + ((long long)b * S + (long long)r * Sl + sl) * run_bytes;
       dst = rp.out[r] + (((long long)b * Sl + sl) * P + g) * run_bytes;
     }
+    // up to 8 vectors per lane in flight (a run of up to 4 KB in one round), loads before stores
     const uint4* s4 = reinterpret_cast<const uint4*>(src);
     uint4* d4 = reinterpret_cast<uint4*>(dst);
     int v = lane;
-    for (; v + 96 < nvec; v += 128) {
-      const uint4 x0 = __ldcs(s4 + v), x1 = __ldcs(s4 + v + 32), x2 = __ldcs(s4 + v + 64), x3 = __ldcs(s4 + v + 96);
-      __stcs(d4 + v, x0);
-      __stcs(d4 + v + 32, x1);
-      __stcs(d4 + v + 64, x2);
-      __stcs(d4 + v + 96, x3);
+    for (; v + 224 < nvec; v += 256) {
+      uint4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = __ldg(s4 + v + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) d4[v + 32 * u] = x[u];
     }
-    for (; v < nvec; v += 32) __stcs(d4 + v, __ldcs(s4 + v));
+    {
+      uint4 x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (v + 32 * u < nvec) x[u] = __ldg(s4 + v + 32 * u);
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (v + 32 * u < nvec) d4[v + 32 * u] = x[u];
+    }
   }
 }
 
