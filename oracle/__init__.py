@@ -138,6 +138,44 @@ def attention_bwd(q, k, v, dout, *, causal=False, nthreads=None, lib=None):
     return dq, dk, dv
 
 
+def attention_bwd_rows(q, k, v, dout, *, heads, q_rows, k_rows, causal=False, nthreads=None, lib=None):
+    """dq at the query positions q_rows and dk, dv at the key positions k_rows, for the listed heads, in
+    fp64: the same definitions as :func:`attention_bwd` ("CHARM+ ...", abstract: the backward pass),
+    evaluated one row at a time.  The forward o and lse of every query of those heads come from
+    :func:`attention`; then, with p_ij = exp(q_i.k_j / sqrt(D) - lse_i) and delta_i = do_i . o_i,
+    dq_i = sum_j p_ij (do_i.v_j - delta_i) k_j / sqrt(D) over the keys query i sees, and
+    dv_j = sum_i p_ij do_i, dk_j = sum_i p_ij (do_i.v_j - delta_i) q_i / sqrt(D) over the queries that
+    see key j.  A row costs O(S D), so full-size workloads can be checked on sampled rows.
+
+    Returns dq [B, len(q_rows), len(heads), D] and dk, dv [B, len(k_rows), len(heads), D]."""
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, S, H, D = q.shape
+    hs = [int(h) for h in heads]
+    qh, kh, vh, dh = (np.ascontiguousarray(t[:, :, hs]) for t in (q, k, v, dout))
+    o, lse = attention(qh, kh, vh, causal=causal, nthreads=nthreads, lib=lib)
+    delta = np.einsum("bshd,bshd->bhs", dh, o)
+    scale = 1.0 / np.sqrt(D)
+    dq = np.zeros((B, len(q_rows), len(hs), D))
+    dk = np.zeros((B, len(k_rows), len(hs), D))
+    dv = np.zeros((B, len(k_rows), len(hs), D))
+    for b in range(B):
+        for n_h in range(len(hs)):
+            Q, K, V, dO = qh[b, :, n_h], kh[b, :, n_h], vh[b, :, n_h], dh[b, :, n_h]
+            L, dl = lse[b, n_h], delta[b, n_h]
+            for n, i in enumerate(q_rows):
+                je = i + 1 if causal else S  # keys query i sees
+                p = np.exp(K[:je] @ Q[i] * scale - L[i])
+                ds = p * (V[:je] @ dO[i] - dl[i])
+                dq[b, n, n_h] = ds @ K[:je] * scale
+            for n, j in enumerate(k_rows):
+                i0 = j if causal else 0  # queries that see key j
+                p = np.exp(Q[i0:] @ K[j] * scale - L[i0:])
+                dv[b, n, n_h] = p @ dO[i0:]
+                ds = p * (dO[i0:] @ V[j] - dl[i0:])
+                dk[b, n, n_h] = ds @ Q[i0:] * scale
+    return dq, dk, dv
+
+
 def attention_probs(q, k, v, *, causal=False, block_mask=None, tile=TILE, kv_begin=0, kv_end=None, lib=None):
     """As :func:`attention`, also returning the probabilities p [B, H, S, S] (tiny inputs only)."""
     q, k, v = _f64(q), _f64(k), _f64(v)

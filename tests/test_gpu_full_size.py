@@ -90,3 +90,36 @@ def test_block_sparse_dit():
     assert spattn.sp_check_device_error() == spattn.SP_OK
     o_s, l_s = _sampled(step.o, step.lse, rows)
     assert_close(o_s, ref[0], l_s, ref[1])
+
+
+def test_video_dit_rank_backward():
+    """The backward the benchmark times (sp_attn_bwd on one simulated rank's 10 heads of video_dit, dense,
+    B1 S32760 D128), checked on sampled query rows (dq) and key rows (dk, dv) of one head against the
+    oracle, which evaluates each sampled row over all keys or queries.  Tolerance as in
+    tests/test_gpu_attn_bwd.py (rel-L2 1e-2, max-abs 2e-2 of the largest reference value)."""
+    import numpy as np
+    w = synth.WORKLOADS["video_dit"]
+    hl = w.H // w.ranks
+    q, k, v = synth.qkv(w.B, w.S, w.H, w.D, seed=0, scale=w.scale)
+    q, k, v = (t[:, :, :hl].contiguous() for t in (q, k, v))
+    do = torch.randn(q.shape, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), do.cuda()
+    o = torch.empty_like(qd)
+    lse = torch.empty((w.B, hl, w.S), device="cuda")
+    spattn.sp_attn_fwd(qd, kd, vd, o, lse)
+    dq, dk, dv = (torch.full_like(qd, float("nan")) for _ in range(3))
+    spattn.sp_attn_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv)
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    rows = synth.sample_rows(w.S, 32, seed=5, must=[127, 128, 16383, 16384])
+    heads = [hl // 2]
+    rq, rk, rv = oracle.attention_bwd_rows(to64(q), to64(k), to64(v), to64(do), heads=heads, q_rows=rows,
+                                           k_rows=rows)
+    r = torch.tensor(rows)
+    for x, ref, name in ((dq, rq, "dq"), (dk, rk, "dk"), (dv, rv, "dv")):
+        got = to64(x.cpu()[:, r][:, :, heads])
+        d = got - ref
+        rel = np.linalg.norm(d) / max(np.linalg.norm(ref), 1e-3 * np.sqrt(ref.size))
+        mx = np.max(np.abs(d)) / max(np.max(np.abs(ref)), 1e-3)
+        assert np.all(np.isfinite(got)), name
+        assert rel <= 1e-2 and mx <= 2e-2, (name, rel, mx)

@@ -503,3 +503,45 @@ def test_attention_bwd_invariants_and_single_key():
     # causal: query 0 sees key 0 only, so its gradient does not reach later keys and dq_0 = 0
     dq, dk, dv = oracle.attention_bwd(q, k, v, do, causal=True)
     np.testing.assert_allclose(dq[:, 0], 0.0, atol=1e-15)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_bwd_rows_matches_finite_differences(causal):
+    """The row-sampled gradients equal central differences of L = sum(dO * O) through the forward oracle,
+    for the sampled query rows (dq) and key rows (dk, dv) of the sampled heads."""
+    rng = np.random.default_rng(11)
+    B, S, H, D = 2, 7, 3, 3
+    q, k, v, do = (rng.standard_normal((B, S, H, D)) for _ in range(4))
+    heads, q_rows, k_rows = [2, 0], [0, 4, 6], [6, 1]
+    dq, dk, dv = oracle.attention_bwd_rows(q, k, v, do, heads=heads, q_rows=q_rows, k_rows=k_rows, causal=causal)
+
+    def loss(qq, kk, vv):
+        return float((do * oracle.attention(qq, kk, vv, causal=causal)[0]).sum())
+
+    eps = 1e-6
+    for x, which, rows, g in ((q, 0, q_rows, dq), (k, 1, k_rows, dk), (v, 2, k_rows, dv)):
+        for b in range(B):
+            for n_h, h in enumerate(heads):
+                for n, r in enumerate(rows):
+                    for d in range(D):
+                        args_p, args_m = [q, k, v], [q, k, v]
+                        xp, xm = x.copy(), x.copy()
+                        xp[b, r, h, d] += eps
+                        xm[b, r, h, d] -= eps
+                        args_p[which], args_m[which] = xp, xm
+                        num = (loss(*args_p) - loss(*args_m)) / (2 * eps)
+                        np.testing.assert_allclose(g[b, n, n_h, d], num, atol=1e-7, rtol=1e-6)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_bwd_rows_agrees_with_full_backward(causal):
+    """Same numbers as the full C backward at the sampled rows (two implementations of one definition)."""
+    rng = np.random.default_rng(12)
+    B, S, H, D = 1, 300, 3, 16
+    q, k, v, do = (rng.standard_normal((B, S, H, D)) for _ in range(4))
+    heads, q_rows, k_rows = [1, 2], [0, 127, 128, 299], [0, 128, 255, 299]
+    dq, dk, dv = oracle.attention_bwd_rows(q, k, v, do, heads=heads, q_rows=q_rows, k_rows=k_rows, causal=causal)
+    fq, fk, fv = oracle.attention_bwd(q, k, v, do, causal=causal)
+    np.testing.assert_allclose(dq, fq[:, q_rows][:, :, heads], atol=1e-11, rtol=1e-9)
+    np.testing.assert_allclose(dk, fk[:, k_rows][:, :, heads], atol=1e-11, rtol=1e-9)
+    np.testing.assert_allclose(dv, fv[:, k_rows][:, :, heads], atol=1e-11, rtol=1e-9)
