@@ -90,6 +90,18 @@ def test_block_sparse_dit():
     assert spattn.sp_check_device_error() == spattn.SP_OK
     o_s, l_s = _sampled(step.o, step.lse, rows)
     assert_close(o_s, ref[0], l_s, ref[1])
+    # the db-SP launches the benchmark times: four simulated ranks' planned item lists write exactly what
+    # the single launch wrote (each item's arithmetic is the same)
+    o1, l1 = step.o.clone(), step.lse.clone()
+    step.o.fill_(float("nan"))
+    step.lse.fill_(float("nan"))
+    lists, imb = step.rank_items(4, planned=True)
+    for items in lists:
+        step.run_items(items)
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    assert imb < 1.01
+    assert torch.equal(step.o, o1) and torch.equal(step.lse, l1)
 
 
 def test_video_dit_rank_backward():
