@@ -70,7 +70,7 @@ struct Cfg {
   // columns), the MMA's B operand being split by N between the two SMs.
   static constexpr int kKVBytes = kPair ? kTileBytes / 2 : kTileBytes;
   static constexpr int kKSubBytes = kPair ? 8192 : 16384;  // between the 64-column sub-tiles of a K slot
-  static constexpr int kStages = kPair ? 8 : (D == 128 ? 4 : 8);  // K/V ring slots
+  static constexpr int kStages = kPair ? 6 : (D == 128 ? 4 : 8);  // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kKVBytes;
@@ -79,7 +79,11 @@ struct Cfg {
   static constexpr int kNumBars = 2 + 2 * kStages + 9;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // misc: TMEM base, abort flag, published-item count, per-warp item-read counts, the item ring
-  static constexpr int kSmemBytes = kMiscOff + 96 + 1024;  // + alignment slack
+  // then, 1024-aligned, staging for the O stores: per softmax warp two 4 KB buffers (32 rows x 128 bytes)
+  // where they fit in the 227 KB a CTA may have, else one
+  static constexpr int kStgOff = (kMiscOff + 96 + 1023) / 1024 * 1024;
+  static constexpr int kStgBufs = kStgOff + 2 * 8 * 4096 + 1024 <= 232448 ? 2 : 1;
+  static constexpr int kSmemBytes = kStgOff + kStgBufs * 8 * 4096 + 1024;  // + alignment slack
   static constexpr int kM = kPair ? 256 : 128;  // MMA rows: a pair computes both CTAs' 128 rows at once
   static constexpr uint32_t kIdescS = idesc_bf16_f32(kM, 128, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kM, D, false, true);
@@ -87,6 +91,11 @@ struct Cfg {
   static constexpr uint32_t kColS = 0;
   static constexpr uint32_t kColO = 256;
 };
+
+// every configuration fits the 227 KB of shared memory a CTA may have
+static_assert(Cfg<128, true>::kSmemBytes <= 232448 && Cfg<128, false>::kSmemBytes <= 232448 &&
+                  Cfg<64, false>::kSmemBytes <= 232448,
+              "shared memory");
 
 struct Bars {
   uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, pv_done0, o_done0, drain;
@@ -316,6 +325,7 @@ struct TMaps {
   CUtensorMap k[kMaxShards];
   CUtensorMap v[kMaxShards];
   CUtensorMap k64[kMaxShards];  // K with 64-row boxes: a CTA pair's halves of a key tile
+  CUtensorMap o[kMaxShards];    // O as a store target (bf16 or fp32), 32-row boxes
 };
 
 // ------------------------------------------------------------------------------------------------
@@ -610,8 +620,8 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
 // Softmax + epilogue: 4 warps per lane, one query row per thread.
 // ------------------------------------------------------------------------------------------------
 template <int D, bool kPair>
-__device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRing& ir, uint32_t tmem, int lane_t,
-                            volatile int* abort_flag) {
+__device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase, const Bars& bars, const ItemRing& ir,
+                            uint32_t tmem, int lane_t, volatile int* abort_flag) {
   using C = Cfg<D, kPair>;
   // A pair's rank 1 hands its P and its O read-outs to rank 0's barriers and counters.
   const bool remote = kPair && cluster_rank() != 0;
@@ -765,30 +775,56 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
         // A row that never saw a visible key is exactly 0 (the FMA-pipe exponentials of its masked
         // entries are tiny but not zero).
         const float inv_l = (l > 0.f && m_used != -INFINITY) ? 1.f / l : 0.f;
+        // O / l leaves through a per-warp staging buffer in shared memory, 128 bytes of each of the warp's
+        // 32 rows at a time (32 fp32 or 64 bf16 values, 128-byte swizzle), and a TMA store of that box:
+        // whole 128-byte lines reach L2, and rows past the shard's (or S's) end are not written.
+        const uint32_t stg0 = sbase + C::kStgOff + (uint32_t)warp * (4096u * C::kStgBufs);
+        const CUtensorMap* omap = &tm.o[p.n_shards > 1 ? it.shard : 0];
+        const int row0 = q_row - row + (warp & 3) * 32 - (p.n_shards > 1 ? it.shard * p.shard_rows : 0);
+        const int n_chunks = p.o_f32 ? D / 32 : D / 64;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_wait_ld();
-          if (row_ok) {
-            if (p.o_f32) {
-              float4* dst = reinterpret_cast<float4*>(static_cast<float*>(obase) + o_idx + c * 32);
+        for (int c = 0; c < n_chunks; ++c) {
+          uint32_t v[32];
+          if (p.o_f32) {
+            tmem_ld32(tO + c * 32, v);
+            tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 8; ++e)
-                dst[e] = make_float4(__uint_as_float(o[4 * e]) * inv_l, __uint_as_float(o[4 * e + 1]) * inv_l,
-                                     __uint_as_float(o[4 * e + 2]) * inv_l,
-                                     __uint_as_float(o[4 * e + 3]) * inv_l);
-            } else {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(obase) + o_idx + c * 32);
+            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv_l);
+          } else {
+            uint32_t o2[32];
+            tmem_ld32(tO + c * 64, v);
+            tmem_ld32(tO + c * 64 + 32, o2);
+            tmem_wait_ld();
 #pragma unroll
-              for (int e = 0; e < 4; ++e)
-                dst[e] = make_uint4(pack_bf16x2(__uint_as_float(o[8 * e]) * inv_l, __uint_as_float(o[8 * e + 1]) * inv_l),
-                                    pack_bf16x2(__uint_as_float(o[8 * e + 2]) * inv_l, __uint_as_float(o[8 * e + 3]) * inv_l),
-                                    pack_bf16x2(__uint_as_float(o[8 * e + 4]) * inv_l, __uint_as_float(o[8 * e + 5]) * inv_l),
-                                    pack_bf16x2(__uint_as_float(o[8 * e + 6]) * inv_l, __uint_as_float(o[8 * e + 7]) * inv_l));
+            for (int e = 0; e < 16; ++e)
+              v[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv_l, __uint_as_float(v[2 * e + 1]) * inv_l);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              v[16 + e] = pack_bf16x2(__uint_as_float(o2[2 * e]) * inv_l, __uint_as_float(o2[2 * e + 1]) * inv_l);
+          }
+          const uint32_t stg = stg0 + 4096u * (uint32_t)(c % C::kStgBufs);
+          if (c >= C::kStgBufs) {  // the store that last used this buffer must have read it
+            if (lane == 0) {
+              if (C::kStgBufs == 2)
+                bulk_wait_read_but1();
+              else
+                bulk_wait_read_all();
             }
+            __syncwarp();
+          }
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            st_shared_v4(stg + (uint32_t)lane * 128u + (uint32_t)(((e ^ (lane & 7)) << 4)), v[4 * e], v[4 * e + 1],
+                         v[4 * e + 2], v[4 * e + 3]);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_4d(omap, stg, c * (p.o_f32 ? 32 : 64), it.h, row0, it.b);
+            bulk_commit_group();
           }
         }
+        if (lane == 0) bulk_wait_read_all();  // the buffers are free for the next item
+        __syncwarp();
       } else if (row_ok) {
         if (p.o_f32) {
           float4* dst = reinterpret_cast<float4*>(static_cast<float*>(obase) + o_idx);
@@ -811,6 +847,8 @@ __device__ void run_softmax(const AttnParams& p, const Bars& bars, const ItemRin
         smem_counter_add_release(o_done_ctr, 1u);
     }
   }
+  if (lane == 0) bulk_wait_all();  // every O store of this warp has landed before the CTA exits
+  __syncwarp();
 }
 
 template <int D, bool kPair>
@@ -888,7 +926,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp < 8) {
     regs_inc<kRegsSoftmax>();
-    run_softmax<D, kPair>(p, bars, ir, tmem, warp >> 2, abort_flag);
+    run_softmax<D, kPair>(p, tm, smem_u32(smem), bars, ir, tmem, warp >> 2, abort_flag);
   } else {
     regs_dec<kRegsControl>();
     if (warp == kWarpProducer) {
@@ -1028,7 +1066,8 @@ sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
     if (!encode_bshd_tmap(&tm.q[r], p.q_shard[r], p.B, p.shard_rows, p.H, p.D) ||
         !encode_bshd_tmap(&tm.k[r], p.k_shard[r], p.B, p.shard_rows, p.H, p.D) ||
         !encode_bshd_tmap(&tm.v[r], p.v_shard[r], p.B, p.shard_rows, p.H, p.D) ||
-        (pair && !encode_bshd_tmap(&tm.k64[r], p.k_shard[r], p.B, p.shard_rows, p.H, p.D, 64)))
+        (pair && !encode_bshd_tmap(&tm.k64[r], p.k_shard[r], p.B, p.shard_rows, p.H, p.D, 64)) ||
+        !encode_o_tmap(&tm.o[r], p.o_shard[r], p.B, p.shard_rows, p.H, p.D, p.o_f32 != 0))
       return SP_ERR_CUDA;
   if (pair) {
     // work units of four query tiles (two per CTA of the pair), per shard

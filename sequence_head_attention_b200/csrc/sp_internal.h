@@ -79,6 +79,9 @@ struct BwdParams {
 // Device properties and driver entry points (cached per device).
 int num_sms(int device);
 bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, int D, int box_rows = 128);
+// O of an attention launch as a store target: [B, S, H, D] of bf16 or fp32, boxes of 128 bytes of one head
+// (64 bf16 or 32 fp32 values) by 32 positions, 128-byte swizzle.
+bool encode_o_tmap(CUtensorMap* map, void* base, int B, int S, int H, int D, bool f32);
 unsigned long long wait_timeout_ns();
 unsigned int* device_error_word();  // address of the current device's error word, or nullptr
 
