@@ -124,6 +124,18 @@ def test_kv_blocks_merge_equals_unsplit(n_kv, causal):
     assert_close(o, ref[0], lse, ref[1])
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_causal_kv_blocks_with_chunks_and_skipped_units(D):
+    """n_kv_blocks > 1, causal, uneven head chunks and two batches at a size where the later blocks skip
+    whole leading query units (filled 0 / -inf) before the merge: equals the unsplit oracle."""
+    B, S, H = 2, 2100, 3
+    q, k, v = synth.qkv(B, S, H, D, seed=D + 5, scale=0.5)
+    ref = ref_attn(q, k, v, causal=True)
+    for n_kv in (2, 3):
+        o, lse = gpu_attn(q, k, v, chunks=[1, 2], n_kv=n_kv, causal=True)
+        assert_close(o, ref[0], lse, ref[1])
+
+
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("n_kv", [1, 2])
 def test_block_sparse(causal, n_kv):
