@@ -33,6 +33,12 @@
  *     failure returns SP_ERR_CUDA.  A device-side wait that exceeds its time limit (the kernels never
  *     spin without bound) records an error word that sp_check_device_error() reports as SP_ERR_TIMEOUT.
  *   - Device pointers must be 16-byte aligned.
+ *   - Concurrency: the attention entry points (sp_attn_fwd, sp_attn_fwd_partial, sp_attn_fwd_seq_sharded,
+ *     sp_attn_fwd_items, sp_attn_fwd_sparse_noalloc) hand out work through per-launch counters in a fixed
+ *     device array of 64 slots, given to launches in rotation.  At most 64 attention launches may be in
+ *     flight at once on one device (e.g. on different streams, or in graphs replayed concurrently); a
+ *     65th concurrent launch would share a counter with the launch 64 before it and both would compute
+ *     wrong results.  Launches ordered on one stream never overlap and are unaffected.
  */
 #ifndef SP_ATTN_H
 #define SP_ATTN_H
@@ -93,7 +99,9 @@ SP_API size_t sp_attn_fwd_workspace_bytes(int B, int S, int H, int D, int n_kv_b
  * n_kv_blocks  >= 1 and <= ceil(S/128).  1: keys are processed in one pass.  > 1: the key range is cut
  *           into n_kv_blocks contiguous blocks of ceil(S/n) keys (rounded up to a multiple of 128 when a
  *           block mask is given), each block's partial (O, LSE) is computed over all queries into the
- *           workspace, and the partials are re-merged (sp_merge_partials) into o and lse.
+ *           workspace, and the partials are re-merged (sp_merge_partials) into o and lse.  With a mask
+ *           the rounding can leave trailing blocks that would start at or past S: they hold no key and
+ *           are dropped, so fewer than n_kv_blocks partials may be merged.
  * causal    0 or 1: key j is visible to query i only if j <= i (square, top-left aligned).
  * block_mask  device uint8 [H, ceil(S/128), ceil(S/128)] or NULL (dense).  Tile (i, j) of head h is
  *           computed iff block_mask[h][i][j] != 0; combined with causal by AND.  Shared by all b.

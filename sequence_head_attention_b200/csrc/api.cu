@@ -326,21 +326,26 @@ sp_status sp_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
   const size_t o_elems = (size_t)B * S * H * D, l_elems = (size_t)B * H * S;
   const float* op[SP_MAX_PARTS];
   const float* lp[SP_MAX_PARTS];
+  int n_parts = 0;
   for (int i = 0; i < n_kv_blocks; ++i) {
     const long long a = i * blk, e = (i + 1) * blk < S ? (i + 1) * blk : S;
+    // With a mask the block size is rounded up to whole tiles, so trailing blocks can start at or past S:
+    // they hold no key and are dropped (never launched with a kv_begin off the tile grid).
+    if (a >= S) break;
     AttnParams pi = p;
-    pi.kv_begin = (int)(a < S ? a : S);
-    pi.kv_lim = (int)(e > pi.kv_begin ? e : pi.kv_begin);
+    pi.kv_begin = (int)a;
+    pi.kv_lim = (int)e;
     pi.n_kv_tiles = (pi.kv_lim - pi.kv_begin + SP_TILE - 1) / SP_TILE;
     pi.o = parts_o + i * o_elems;
     pi.o_f32 = 1;
     pi.lse = parts_l + i * l_elems;
     s = launch_attn(pi, q, k, v, st);
     if (s != SP_OK) return s;
-    op[i] = parts_o + i * o_elems;
-    lp[i] = parts_l + i * l_elems;
+    op[n_parts] = parts_o + i * o_elems;
+    lp[n_parts] = parts_l + i * l_elems;
+    ++n_parts;
   }
-  return launch_merge(op, lp, n_kv_blocks, o, lse, 0, B, S, H, D, st);
+  return launch_merge(op, lp, n_parts, o, lse, 0, B, S, H, D, st);
 }
 
 sp_status sp_merge_partials(const float* const* o_parts, const float* const* lse_parts, int n, void* o,

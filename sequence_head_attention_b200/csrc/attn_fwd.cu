@@ -52,9 +52,12 @@ constexpr uint32_t kRegsControl = 104;
 constexpr uint32_t kRegsSoftmax = 200;
 static_assert(128 * kRegsControl + 256 * kRegsSoftmax <= kThreads * kRegsLaunch, "register split");
 constexpr int kItemRing = 8;     // work-item ids in flight between the producer and the other roles
-constexpr int kSchedSlots = 64;  // launch-rotated work counters, so concurrent launches never share one
-// Per-launch work counters [next item, CTAs finished], kSchedSlots pairs handed out in rotation.  A
-// launch leaves its pair at zero when its last CTA ends.
+constexpr int kSchedSlots = 64;  // launch-rotated work counters
+// Per-launch work counters [next item, CTAs finished], kSchedSlots pairs handed out in rotation, so that
+// up to kSchedSlots launches in flight at once (on different streams) draw different pairs.  Launches
+// kSchedSlots apart draw the same pair: if two such launches overlapped on the GPU they would claim from
+// one counter and skip or repeat items, so at most kSchedSlots attention launches may be in flight on a
+// device (the C header states this limit).  A launch leaves its pair at zero when its last CTA ends.
 __device__ unsigned int g_attn_sched[2 * kSchedSlots];
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and l are rescaled when m grows by > 2^8
 #ifndef SP_EXP2_POLY_PAIRS

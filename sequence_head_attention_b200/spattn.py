@@ -116,6 +116,30 @@ def _bshd(t, name, dtype=torch.bfloat16):
     _need(t.is_cuda and t.is_contiguous(), f"{name} must be a contiguous CUDA tensor")
 
 
+def _same_device(ts, ref):
+    for t in ts:
+        if t is not None:
+            _need(t.device == ref.device, "all tensors must be on one device")
+
+
+def _check_mask(block_mask, H, S, device):
+    """A block mask the kernels may read: contiguous uint8 [H, ceil(S/128), ceil(S/128)] on `device`.  The
+    library receives only a pointer, so a wrong shape or a host tensor is refused here, before any call."""
+    T = (S + SP_TILE - 1) // SP_TILE
+    _need(isinstance(block_mask, torch.Tensor) and block_mask.dtype == torch.uint8 and block_mask.is_contiguous(),
+          "block_mask must be a contiguous uint8 tensor")
+    _need(tuple(block_mask.shape) == (H, T, T), f"block_mask must be [H, ceil(S/128), ceil(S/128)] = [{H}, {T}, {T}]")
+    _need(block_mask.is_cuda and block_mask.device == torch.device(device),
+          "block_mask must be a CUDA tensor on the device of q")
+
+
+def _check_lse(lse, B, H, S, device):
+    """An lse output the kernels may write: contiguous fp32 [B, H, S] on `device`."""
+    _need(isinstance(lse, torch.Tensor) and lse.dtype == torch.float32 and lse.is_contiguous()
+          and tuple(lse.shape) == (B, H, S), "lse must be contiguous fp32 [B, H, S]")
+    _need(lse.is_cuda and lse.device == torch.device(device), "lse must be a CUDA tensor on the device of q")
+
+
 # ------------------------------------------------------------------------------------------------------
 def sp_status_string(status: int) -> str:
     return lib().sp_status_string(int(status)).decode()
@@ -137,12 +161,12 @@ def sp_attn_fwd(q, k, v, o, lse=None, head_chunks=None, n_kv_blocks=1, causal=Fa
     (device memory is the caller's: the library itself never allocates)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _bshd(t, n)
+    _same_device((k, v, o), q)
     B, S, H, D = q.shape
     if lse is not None:
-        _need(lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, S),
-              "lse must be contiguous fp32 [B, H, S]")
+        _check_lse(lse, B, H, S, q.device)
     if block_mask is not None:
-        _need(block_mask.dtype == torch.uint8 and block_mask.is_contiguous(), "block_mask must be uint8")
+        _check_mask(block_mask, H, S, q.device)
     ws_bytes = sp_attn_fwd_workspace_bytes(B, S, H, D, n_kv_blocks, block_mask is not None)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
@@ -166,8 +190,11 @@ def sp_attn_fwd_partial(q, k, v, o_part, lse_part, kv_begin, kv_end, causal=Fals
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _bshd(t, n)
     _bshd(o_part, "o_part", torch.float32)
+    _same_device((k, v, o_part), q)
     B, S, H, D = q.shape
-    _need(lse_part.dtype == torch.float32 and tuple(lse_part.shape) == (B, H, S), "lse_part must be fp32 [B,H,S]")
+    _check_lse(lse_part, B, H, S, q.device)
+    if block_mask is not None:
+        _check_mask(block_mask, H, S, q.device)
     ws_bytes = sp_attn_fwd_workspace_bytes(B, S, H, D, 1, block_mask is not None)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
@@ -307,13 +334,13 @@ def sp_attn_fwd_items(q, k, v, o, lse, items, causal=False, block_mask=None, wor
     """Attention of the listed work items only (items: device int32 tensor of item ids)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _bshd(t, n)
+    _same_device((k, v, o, items), q)
     B, S, H, D = q.shape
     _need(items.dtype == torch.int32 and items.is_cuda and items.is_contiguous(), "items must be CUDA int32")
     if lse is not None:
-        _need(lse.dtype == torch.float32 and lse.is_contiguous() and tuple(lse.shape) == (B, H, S),
-              "lse must be contiguous fp32 [B, H, S]")
+        _check_lse(lse, B, H, S, q.device)
     if block_mask is not None:
-        _need(block_mask.dtype == torch.uint8 and block_mask.is_contiguous(), "block_mask must be uint8")
+        _check_mask(block_mask, H, S, q.device)
     ws_bytes = sp_attn_fwd_workspace_bytes(B, S, H, D, 1, block_mask is not None)
     if workspace is None and ws_bytes > 0:
         workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
@@ -378,9 +405,12 @@ def sp_attn_fwd_sparse_noalloc(q, k, v, o, lse, block_mask, causal=False, stream
     array inside the library instead (size limits and the no-overlap rule in include/sp_attn.h)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _bshd(t, n)
+    _same_device((k, v, o), q)
     B, S, H, D = q.shape
-    _need(block_mask is not None and block_mask.dtype == torch.uint8 and block_mask.is_contiguous(),
-          "block_mask must be a contiguous uint8 tensor")
+    _need(block_mask is not None, "block_mask is required")
+    _check_mask(block_mask, H, S, q.device)
+    if lse is not None:
+        _check_lse(lse, B, H, S, q.device)
     st = lib().sp_attn_fwd_sparse_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, S, H, D,
                                           int(bool(causal)), _ptr(block_mask), _stream(stream))
     _check("sp_attn_fwd_sparse_noalloc", st)
@@ -390,6 +420,11 @@ def sp_attn_fwd_sparse_noalloc(q, k, v, o, lse, block_mask, causal=False, stream
 def sp_build_tile_list(block_mask, S, row_ptr, col_idx, counts, stream=None):
     """CSR of the kept key tiles of a uint8 [H, T, T] block mask (T = ceil(S/128))."""
     H = block_mask.shape[0]
+    _check_mask(block_mask, H, S, block_mask.device)
+    T = (S + SP_TILE - 1) // SP_TILE
+    for t, n, size in ((row_ptr, "row_ptr", H * T + 1), (col_idx, "col_idx", H * T * T), (counts, "counts", H * T)):
+        _need(t.dtype == torch.int32 and t.is_contiguous() and t.numel() >= size and t.device == block_mask.device,
+              f"{n} must be a contiguous int32 tensor of at least {size} elements on the mask's device")
     st = lib().sp_build_tile_list(_ptr(block_mask), H, S, _ptr(row_ptr), _ptr(col_idx), _ptr(counts),
                                   _stream(stream))
     _check("sp_build_tile_list", st)

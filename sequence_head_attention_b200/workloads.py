@@ -59,6 +59,8 @@ class UlyssesStep:
         self.launches = P if fused else 3 + P + 1
         self.flops = w.flops()
         self.relayout_bytes = 4 * 2 * B * S * H * D * 2  # 4 tensors, each read once and written once
+        # one rank's attention launch: its heads of Q, K, V read and of O written (bf16), and its lse rows
+        self.attn_bytes_per_launch = 4 * B * S * self.Hl * D * 2 + B * self.Hl * S * 4
 
     def relayout_in(self, stream=None):
         spattn.sp_seq_to_head_relayout(self.q_seq, self.q_head, stream=stream)
@@ -107,6 +109,7 @@ class RingStep:
         self.l_parts = [torch.empty((B, H, S), dtype=torch.float32, device=device) for _ in range(n)]
         self.o = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=device)
         self.lse = torch.empty((B, H, S), dtype=torch.float32, device=device)
+        self.attn_launches = n
         self.launches = n + 1
         self.flops = w.flops()
         # merge: read n fp32 partials (O and LSE), write bf16 O and fp32 LSE

@@ -96,3 +96,31 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(spattn, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         spattn.sp_version()
+
+
+def test_binding_refuses_bad_masks_and_lse_before_any_call():
+    """The library gets only pointers, so the binding refuses a mask or lse of the wrong shape, type or
+    device before calling it (a host or undersized mask would be read out of bounds by the kernels)."""
+    import torch
+    S, H = 1000, 3  # T = ceil(1000 / 128) = 8
+    good = torch.zeros((H, 8, 8), dtype=torch.uint8)
+    with pytest.raises(ValueError, match=r"\[3, 8, 8\]"):
+        spattn._check_mask(torch.zeros((H, 7, 8), dtype=torch.uint8), H, S, "cuda:0")
+    with pytest.raises(ValueError, match=r"\[3, 8, 8\]"):
+        spattn._check_mask(torch.zeros((H + 1, 8, 8), dtype=torch.uint8), H, S, "cuda:0")
+    with pytest.raises(ValueError, match="uint8"):
+        spattn._check_mask(good.float(), H, S, "cuda:0")
+    with pytest.raises(ValueError, match="uint8"):
+        spattn._check_mask(torch.zeros((H, 8, 16), dtype=torch.uint8)[:, :, ::2], H, S, "cuda:0")
+    with pytest.raises(ValueError, match="CUDA"):
+        spattn._check_mask(good, H, S, "cuda:0")  # a host tensor
+    with pytest.raises(ValueError, match="lse"):
+        spattn._check_lse(torch.zeros((1, H, S - 1)), 1, H, S, "cuda:0")
+    with pytest.raises(ValueError, match="lse"):
+        spattn._check_lse(torch.zeros((1, H, S), dtype=torch.float64), 1, H, S, "cuda:0")
+    with pytest.raises(ValueError, match="CUDA"):
+        spattn._check_lse(torch.zeros((1, H, S)), 1, H, S, "cuda:0")
+    # the tile-list wrapper checks its mask too, before touching the library
+    i32 = torch.zeros(H * 64, dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        spattn.sp_build_tile_list(good, S, i32, i32, i32)

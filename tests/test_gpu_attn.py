@@ -147,6 +147,20 @@ def test_block_sparse(causal, n_kv):
     assert_close(o, ref[0], lse, ref[1])
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_sparse_kv_blocks_rounded_past_s(causal):
+    """With a mask the KV block size is rounded up to whole tiles: S = 1200 in 7 blocks gives blocks of
+    256 keys, so blocks 5 and 6 would start at or past S.  They hold no key and are dropped; the keys of
+    the last tile (1152..1199) are counted once, and the result equals the unsplit oracle."""
+    B, S, H, D = 1, 1200, 3, 128
+    q, k, v = synth.qkv(B, S, H, D, seed=12, scale=0.5)
+    mask = synth.block_mask(H, S, seed=12)
+    ref = ref_attn(q, k, v, causal=causal, mask=mask)
+    for n_kv in (7, 10):
+        o, lse = gpu_attn(q, k, v, causal=causal, mask=mask, n_kv=n_kv)
+        assert_close(o, ref[0], lse, ref[1])
+
+
 def test_block_sparse_partial_and_empty_rows():
     B, S, H, D = 1, 1000, 3, 64
     q, k, v = synth.qkv(B, S, H, D, seed=4, scale=0.5)
@@ -254,3 +268,28 @@ def test_concurrent_launches_on_two_streams():
     for oa, la, ob, lb in outs:
         assert torch.equal(oa, ref_a[0]) and torch.equal(la, ref_a[1])
         assert torch.equal(ob, ref_b[0]) and torch.equal(lb, ref_b[1])
+
+
+def test_binding_refuses_host_or_undersized_masks():
+    """Masks the kernels would read out of bounds (a host tensor, too few tiles) and a wrong lse are
+    refused by the binding before the library is called."""
+    B, S, H, D = 1, 1000, 3, 128
+    q, k, v = (t.cuda() for t in synth.qkv(B, S, H, D, seed=2))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, S), device="cuda")
+    good = synth.block_mask(H, S, seed=2)
+    bad = [good, good[:, :4, :4].contiguous().cuda(), good[:2].contiguous().cuda()]
+    items = torch.zeros(1, dtype=torch.int32, device="cuda")
+    for m in bad:
+        with pytest.raises(ValueError):
+            spattn.sp_attn_fwd(q, k, v, o, lse, block_mask=m)
+        with pytest.raises(ValueError):
+            spattn.sp_attn_fwd_sparse_noalloc(q, k, v, o, lse, m)
+        with pytest.raises(ValueError):
+            spattn.sp_attn_fwd_items(q, k, v, o, lse, items, block_mask=m)
+        with pytest.raises(ValueError):
+            spattn.sp_attn_fwd_partial(q, k, v, o.float(), lse, 0, S, block_mask=m)
+    with pytest.raises(ValueError):
+        spattn.sp_attn_fwd_sparse_noalloc(q, k, v, o, lse[:, :, :-1], good.cuda())
+    with pytest.raises(ValueError):
+        spattn.sp_attn_fwd_sparse_noalloc(q, k, v, o, lse.cpu(), good.cuda())
