@@ -11,8 +11,10 @@ in the same run, each with its own CUDA-event timing and roofline block under "k
                         ranks); every rank's attention on its 10 heads with the head chunks [3,7,10,10,10]
                         split at rank boundaries, read from and written into the shards.  Also measured: the
                         seq<->head relayouts on their own (HBM GB/s) and the backward of one rank's heads.
-  ring_causal           B1 S57344 H40 D128 causal: 8 KV blocks, one launch each, whose partial (O, LSE) is
-                        re-merged (attention TFLOPS, merge GB/s, step time).
+  ring_causal           B1 S57344 H40 D128 causal: 8 KV blocks, one launch each; the first writes the running
+                        (O, LSE), each later one merges its partial into it in place, and the running O is
+                        rounded to bf16 (attention TFLOPS, step time).  The standalone re-merge of 8
+                        materialised partials (sp_merge_partials) is timed on its own (merge GB/s).
   block_sparse          B1 S32768 H40 D128, per-head tile mask of density U[0.1, 0.9]: tile list +
                         attention (TFLOPS on kept tiles), and the db-SP split over 4 simulated ranks.
   tiny_dense, megatron  the two latency configurations: microseconds per call and TFLOPS, back to back
@@ -344,12 +346,12 @@ def check_device(where):
         raise SystemExit(f"device error {spattn.sp_status_string(st)} (bits {bits:#x}) {where}")
 
 
-def make_step(wname, w, q, k, v, mask, dev, fused=True):
+def make_step(wname, w, q, k, v, mask, dev, fused=True, with_partials=False):
     from sequence_head_attention_b200 import workloads
     if wname == "video_dit":
         return workloads.UlyssesStep(w, q, k, v, device=dev, fused=fused)
     if wname == "ring_causal":
-        return workloads.RingStep(w, q, k, v, device=dev)
+        return workloads.RingStep(w, q, k, v, device=dev, with_partials=with_partials)
     return workloads.SparseStep(w, q, k, v, mask, device=dev)
 
 
@@ -368,7 +370,7 @@ def step_phases(wname, step, fused, timer: Timer):
         timer.phase("relayout", step.relayout_out)
     elif wname == "ring_causal":
         timer.phase("attn_all", step.attention)
-        timer.phase("merge", step.merge)
+        timer.phase("finish", step.finish)
     else:
         timer.phase("attn", step.run)
 
@@ -463,7 +465,7 @@ def measure_main(wname, args, peaks, dev, stream, world, seed, headline):
     w, q, k, v, mask = build_inputs(wname, seed=seed, seq_len=args.seq_len if headline else 0,
                                     ranks=args.ranks if headline else 0)
     fused = wname == "video_dit" and args.ulysses == "fused"
-    step = make_step(wname, w, q, k, v, mask, dev, fused)
+    step = make_step(wname, w, q, k, v, mask, dev, fused, with_partials=wname == "ring_causal")
     for _ in range(args.warmup):
         step.run()
     torch.cuda.synchronize(dev)
@@ -497,16 +499,17 @@ def measure_main(wname, args, peaks, dev, stream, world, seed, headline):
             rec["relayout_in_step_ms"] = sum(timer.spans("relayout")) / args.steps
     elif wname == "ring_causal":
         attn_ms = timer.mean_ms("attn_all")
-        m_ms = timer.mean_ms("merge")
+        f_ms = timer.mean_ms("finish")
         rec["attention"] = {"tflops": step.flops / (attn_ms / 1000.0) / 1e12, "ms_per_step": attn_ms,
                             "launches_per_step": step.attn_launches,
+                            "how": "first KV block written, every later block merged into the running result "
+                                   "in its epilogue (sp_attn_fwd_partial_merge); no partial is materialised",
                             "roofline": tensor_roofline(step.flops, attn_ms, peaks, None)}
         rec["attention"]["roofline"]["traffic_note"] = ("the attention of a ring step is several launches; "
                                                         "traffic per launch is not recorded")
-        rec["merge"] = {"gbs": step.merge_bytes / (m_ms / 1000.0) / 1e9, "ms": m_ms, "bytes": step.merge_bytes,
-                        "frac_of_measured_hbm": step.merge_bytes / (m_ms / 1000.0) / 1e9 / peaks["hbm_gbs"],
-                        "roofline": hbm_roofline(step.merge_bytes, m_ms, peaks,
-                                                 "merge.ring_causal" if not args.seq_len else None)}
+        rec["finish"] = {"what": "running fp32 O rounded to bf16", "ms": f_ms,
+                         "gbs": step.convert_bytes / (f_ms / 1000.0) / 1e9}
+        rec["merge"] = merge_report(step, args, peaks, stream)
     else:
         attn_ms = timer.mean_ms("attn")
         rec["attention"] = {"tflops": step.flops / (attn_ms / 1000.0) / 1e12, "ms_per_launch": attn_ms,
@@ -514,6 +517,25 @@ def measure_main(wname, args, peaks, dev, stream, world, seed, headline):
                                                         "attn_fwd.block_sparse" if not args.seq_len else None),
                             "mask_density": step.density, "kept_tiles": step.kept_tiles}
     return rec, step, (w, q, k, v, mask, fused)
+
+
+def merge_report(step, args, peaks, stream):
+    """The standalone re-merge (sp_merge_partials) of the ring's 8 materialised fp32 partials into bf16 O and
+    fp32 LSE, timed on its own after the timed steps."""
+    import torch
+    step.partials()
+    step.merge()
+    torch.cuda.synchronize()
+    t = Timer(stream)
+    for _ in range(args.steps):
+        t.phase("merge", step.merge)
+    torch.cuda.synchronize()
+    check_device("in the standalone merge")
+    m_ms = t.mean_ms("merge")
+    gbs = step.merge_bytes / (m_ms / 1000.0) / 1e9
+    return {"gbs": gbs, "ms": m_ms, "bytes": step.merge_bytes, "parts": len(step.o_parts),
+            "frac_of_measured_hbm": gbs / peaks["hbm_gbs"], "in_timed_step": False,
+            "roofline": hbm_roofline(step.merge_bytes, m_ms, peaks, "merge.ring_causal" if not args.seq_len else None)}
 
 
 def latency_report(wname, dev, stream, peaks, reps=200):

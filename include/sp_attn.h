@@ -34,7 +34,7 @@
  *     spin without bound) records an error word that sp_check_device_error() reports as SP_ERR_TIMEOUT.
  *   - Device pointers must be 16-byte aligned.
  *   - Concurrency: the attention entry points (sp_attn_fwd, sp_attn_fwd_partial, sp_attn_fwd_seq_sharded,
- *     sp_attn_fwd_items, sp_attn_fwd_sparse_noalloc) hand out work through per-launch counters in a fixed
+ *     sp_attn_fwd_partial_merge, sp_attn_fwd_items, sp_attn_fwd_sparse_noalloc) hand out work through per-launch counters in a fixed
  *     device array of 64 slots, given to launches in rotation.  At most 64 attention launches may be in
  *     flight at once on one device (e.g. on different streams, or in graphs replayed concurrently); a
  *     65th concurrent launch would share a counter with the launch 64 before it and both would compute
@@ -128,6 +128,29 @@ SP_API sp_status sp_attn_fwd_partial(const void* q, const void* k, const void* v
                               float* lse_part, int B, int S, int H, int D, int kv_begin, int kv_end,
                               int causal, const uint8_t* block_mask, void* workspace,
                               size_t workspace_bytes, sp_stream stream);
+
+/*
+ * One KV block merged straight into a running result, the form in which a ring consumes its rounds
+ * ("CHARM+: How Cross-Hardware Attention Breaks Through ...", Ring-Attention paragraph: each round computes
+ * local attention on one KV block and accumulates the partial results; "CHARM+: Cross-Hardware Attention
+ * with Re-Merge ...", abstract: re-merge).  It computes the block's partial (O_b, LSE_b) over keys
+ * kv_begin <= j < kv_end exactly as sp_attn_fwd_partial does, and instead of writing it, merges it into
+ * (o_acc, lse_acc) in place with the log-sum-exp rule of sp_merge_partials:
+ *   lse' = ln(e^lse_acc + e^LSE_b),  o_acc' = e^(lse_acc - lse') o_acc + e^(LSE_b - lse') O_b.
+ * Rows that see no key of the block (e.g. causal queries before kv_begin) keep o_acc and lse_acc
+ * untouched; no partial is ever materialised.  A row whose lse_acc is -inf has no running result yet: its
+ * o_acc is not read into the sum (it may hold anything), so a caller starts a ring either with
+ * sp_attn_fwd_partial on its first block into (o_acc, lse_acc), or with lse_acc set to -inf.
+ * The order of the merges changes the result by rounding only.
+ *
+ * o_acc     device, fp32 BSHD [B,S,H,D], read and written.
+ * lse_acc   device, fp32 [B,H,S], read and written (natural log).  Neither may overlap q, k, v or the other.
+ * kv_end == kv_begin is allowed and changes nothing.  Other arguments as in sp_attn_fwd_partial.
+ */
+SP_API sp_status sp_attn_fwd_partial_merge(const void* q, const void* k, const void* v, float* o_acc,
+                                           float* lse_acc, int B, int S, int H, int D, int kv_begin, int kv_end,
+                                           int causal, const uint8_t* block_mask, void* workspace,
+                                           size_t workspace_bytes, sp_stream stream);
 
 /*
  * Re-merge of n partials with the log-sum-exp rule ("CHARM+ ... Re-Merge", abstract):
@@ -305,7 +328,7 @@ SP_API sp_status sp_check_device_error(sp_stream stream);
 /*
  * As sp_check_device_error, and also returns the raw error word in *bits (may be NULL): one bit per
  * kind of wait that expired (Q loaded, Q free, K/V loaded, K/V free, S ready, P ready, P V done, O read
- * out, drain, debug), for diagnosing which hand-off gave up.
+ * out, drain, debug, running-O load of a merge), for diagnosing which hand-off gave up.
  */
 SP_API sp_status sp_check_device_error_bits(sp_stream stream, unsigned int* bits);
 

@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <utility>
 
 #include "sp_internal.h"
 #include "sp_ptx.cuh"
@@ -253,6 +254,55 @@ sp_status sp_attn_fwd_partial(const void* q, const void* k, const void* v, float
   p.o = o_part;
   p.o_f32 = 1;
   p.lse = lse_part;
+  if (block_mask) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    int32_t* row_ptr = reinterpret_cast<int32_t*>(ws + wl.row_ptr);
+    int32_t* col_idx = reinterpret_cast<int32_t*>(ws + wl.col_idx);
+    s = launch_tile_list(block_mask, H, p.mask_T, row_ptr, col_idx, reinterpret_cast<int32_t*>(ws + wl.counts), st);
+    if (s != SP_OK) return s;
+    p.row_ptr = row_ptr;
+    p.col_idx = col_idx;
+  }
+  return launch_attn(p, q, k, v, st);
+}
+
+sp_status sp_attn_fwd_partial_merge(const void* q, const void* k, const void* v, float* o_acc, float* lse_acc,
+                                    int B, int S, int H, int D, int kv_begin, int kv_end, int causal,
+                                    const uint8_t* block_mask, void* workspace, size_t workspace_bytes,
+                                    sp_stream stream) {
+  if (!sizes_ok(B, S, H, D)) return SP_ERR_INVALID_ARG;
+  if (!q || !k || !v || !o_acc || !lse_acc) return SP_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_acc) || !aligned16(lse_acc))
+    return SP_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return SP_ERR_INVALID_ARG;
+  if (kv_begin < 0 || kv_end < kv_begin || kv_end > S) return SP_ERR_INVALID_ARG;
+  if (block_mask && kv_begin % SP_TILE != 0) return SP_ERR_INVALID_ARG;
+  // the running result is read and written in place: it may not overlap the inputs
+  const size_t tb = (size_t)B * S * H * D * 2, ob = (size_t)B * S * H * D * 4, lb = (size_t)B * H * S * 4;
+  for (const void* in : {q, k, v}) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(in);
+    for (const auto& out : {std::make_pair((const void*)o_acc, ob), std::make_pair((const void*)lse_acc, lb)}) {
+      const uintptr_t b0 = reinterpret_cast<uintptr_t>(out.first);
+      if (a0 < b0 + out.second && b0 < a0 + tb) return SP_ERR_INVALID_ARG;
+    }
+  }
+  {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(o_acc), b0 = reinterpret_cast<uintptr_t>(lse_acc);
+    if (a0 < b0 + lb && b0 < a0 + ob) return SP_ERR_INVALID_ARG;
+  }
+  const WsLayout wl = ws_layout(B, S, H, D, 1, block_mask != nullptr);
+  if (wl.total > 0 && (!workspace || workspace_bytes < wl.total || !aligned16(workspace)))
+    return SP_ERR_INVALID_ARG;
+  if (kv_end == kv_begin) return SP_OK;  // no key: every row keeps its running result
+  cudaStream_t st = as_stream(stream);
+  AttnParams p;
+  int h0[2] = {0, H};
+  sp_status s = fill_attn_params(p, B, S, H, D, kv_begin, kv_end, causal, h0, 1);
+  if (s != SP_OK) return s;
+  p.o = o_acc;
+  p.o_f32 = 1;
+  p.lse = lse_acc;
+  p.o_merge = 1;
   if (block_mask) {
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     int32_t* row_ptr = reinterpret_cast<int32_t*>(ws + wl.row_ptr);

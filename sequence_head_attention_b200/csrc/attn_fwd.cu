@@ -77,9 +77,10 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kKVBytes;
-  // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2], drain, and
-  // 8-byte slots for the o_done[2] counters
-  static constexpr int kNumBars = 2 + 2 * kStages + 9;
+  // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2], drain, 8-byte
+  // slots for the o_done[2] counters, and stg_full[8][2] (a merging epilogue's loads of the running O into
+  // each softmax warp's staging buffers)
+  static constexpr int kNumBars = 2 + 2 * kStages + 9 + 16;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // misc: TMEM base, abort flag, published-item count, per-warp item-read counts, the item ring
   // then, 1024-aligned, staging for the O stores: per softmax warp two 4 KB buffers (32 rows x 128 bytes)
@@ -101,7 +102,9 @@ static_assert(Cfg<128, true>::kSmemBytes <= 232448 && Cfg<128, false>::kSmemByte
               "shared memory");
 
 struct Bars {
-  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, pv_done0, o_done0, drain;
+  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, pv_done0, o_done0, drain, stg_full0;
+  // stg_full[w][b]: staging buffer b of softmax warp w holds the running O loaded for a merge
+  __device__ uint32_t stg_full(int w, int b) const { return stg_full0 + 8u * (2 * w + b); }
   __device__ uint32_t kv_full(int s) const { return kv_full0 + 8u * s; }
   __device__ uint32_t kv_empty(int s) const { return kv_empty0 + 8u * s; }
   __device__ uint32_t s_full(int t) const { return s_full0 + 8u * t; }
@@ -620,6 +623,117 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
 }
 
 // ------------------------------------------------------------------------------------------------
+// Epilogue of a launch that merges its rows into a running result (o fp32, lse), the re-merge of one KV
+// block's partial into the accumulated earlier blocks ("CHARM+: Cross-Hardware Attention with Re-Merge
+// ...", abstract; the Ring-Attention paragraph of "CHARM+: How Cross-Hardware Attention Breaks Through
+// ...": each round's partial result is accumulated).  With this block's row maximum m and sum l (log2
+// units) and the running lse a (natural log):
+//   b = m + log2 l,  c = max(a log2 e, b),  wa = 2^(a log2 e - c),  wb = 2^(b - c),
+//   o <- (o wa + (O / l) wb) / (wa + wb),   lse <- (c + log2(wa + wb)) ln 2.
+// A row whose running lse is -inf has no running result: its o is not read into the sum (it may hold
+// anything).  A row that saw no key of this block keeps o and lse as they are.
+// The warp's 32 rows of the running o move as 32 x 32 fp32 boxes: TMA loads into the warp's staging
+// buffers (issued before the last P V is awaited, so they overlap it), the merge in shared memory, TMA
+// stores from the same buffers.  Returns false when a wait gave up (the error is recorded).
+// ------------------------------------------------------------------------------------------------
+template <int D, bool kPair>
+__device__ __forceinline__ bool merge_epilogue(const AttnParams& p, const TMaps& tm, uint32_t sbase, const Bars& bars,
+                                               uint32_t tO, const Item& it, int q_row, int row, int warp, int lane,
+                                               int lane_t, bool row_ok, float l, float m_used, uint32_t total_pv,
+                                               uint32_t& stg_ph, volatile int* abort_flag) {
+  using C = Cfg<D, kPair>;
+  constexpr int kBoxes = D / 32;  // fp32 boxes of 32 columns per row
+  constexpr int kFirst = C::kStgBufs < kBoxes ? C::kStgBufs : kBoxes;
+  const uint64_t tmo = p.timeout_ns;
+  const uint32_t stg0 = sbase + C::kStgOff + (uint32_t)warp * (4096u * C::kStgBufs);
+  const CUtensorMap* omap = &tm.o[0];
+  const int row0 = q_row - row + (warp & 3) * 32;
+  if (lane == 0) {
+#pragma unroll
+    for (int c = 0; c < kFirst; ++c) {
+      mbar_arrive_expect_tx(bars.stg_full(warp, c), 4096u);
+      tma_load_4d(stg0 + 4096u * c, omap, bars.stg_full(warp, c), 32 * c, it.h, row0, it.b);
+    }
+  }
+  __syncwarp();
+  uint32_t pending = (1u << kFirst) - 1u;  // staging buffers with a load in flight
+  // Weights of the running result and of this block's rows (no global read yet depends on the MMAs).
+  const size_t l_idx = ((size_t)it.b * p.H + it.h) * p.S + q_row;
+  const float la = row_ok ? p.lse[l_idx] * 1.4426950408889634f : -INFINITY;
+  const bool has = l > 0.f && m_used != -INFINITY;
+  float wa = 1.f, wb = 0.f, lnew = la;
+  if (has) {
+    const float lb = m_used + log2f(l);
+    const float c = fmaxf(la, lb);
+    const float ea = la == -INFINITY ? 0.f : ex2_approx(la - c);
+    const float eb = ex2_approx(lb - c);
+    const float inv = 1.f / (ea + eb);
+    wa = ea * inv;
+    wb = eb * inv / l;  // O in TMEM is not yet divided by l
+    lnew = c + log2f(ea + eb);
+  }
+  bool ok = mbar_wait(bars.pv_done(lane_t), (total_pv - 1) & 1, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err);
+  ok = __all_sync(0xffffffffu, ok);
+  if (ok) {
+    tc_fence_after();
+#pragma unroll 1
+    for (int c = 0; c < kBoxes; ++c) {
+      const int b = c % C::kStgBufs;
+      const uint32_t stg = stg0 + 4096u * (uint32_t)b;
+      ok = mbar_wait(bars.stg_full(warp, b), (stg_ph >> b) & 1u, tmo, ERR_TIMEOUT_STG, abort_flag, p.err);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      stg_ph ^= 1u << b;
+      pending &= ~(1u << b);
+      uint32_t v[32];
+      tmem_ld32(tO + c * 32, v);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t addr = stg + (uint32_t)lane * 128u + (uint32_t)((e ^ (lane & 7)) << 4);
+        uint32_t a[4];
+        ld_shared_v4(addr, a[0], a[1], a[2], a[3]);
+        uint32_t r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float x = wa > 0.f ? __uint_as_float(a[j]) * wa : 0.f;
+          const float y = wb > 0.f ? __uint_as_float(v[4 * e + j]) * wb : 0.f;
+          r[j] = __float_as_uint(x + y);
+        }
+        st_shared_v4(addr, r[0], r[1], r[2], r[3]);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_4d(omap, stg, 32 * c, it.h, row0, it.b);
+        bulk_commit_group();
+        if (c + C::kStgBufs < kBoxes) {  // refill this buffer with a later box once the store has read it
+          bulk_wait_read_all();
+          mbar_arrive_expect_tx(bars.stg_full(warp, b), 4096u);
+          tma_load_4d(stg, omap, bars.stg_full(warp, b), 32 * (c + C::kStgBufs), it.h, row0, it.b);
+        }
+      }
+      if (c + C::kStgBufs < kBoxes) pending |= 1u << b;
+      __syncwarp();
+    }
+  }
+  if (!ok) {
+    // Leave no load in flight into shared memory: wait (bounded) for every outstanding one.
+#pragma unroll 1
+    for (int b = 0; b < C::kStgBufs; ++b)
+      if (pending & (1u << b)) {
+        warp_mbar_wait(bars.stg_full(warp, b), (stg_ph >> b) & 1u, tmo, ERR_TIMEOUT_STG, nullptr, p.err);
+        stg_ph ^= 1u << b;
+      }
+    return false;
+  }
+  if (lane == 0) bulk_wait_read_all();  // the buffers are free for the next item
+  __syncwarp();
+  if (row_ok && has) p.lse[l_idx] = lnew * 0.69314718055994531f;
+  return true;
+}
+
+// ------------------------------------------------------------------------------------------------
 // Softmax + epilogue: 4 warps per lane, one query row per thread.
 // ------------------------------------------------------------------------------------------------
 template <int D, bool kPair>
@@ -641,6 +755,7 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
   const float scale_log2 = p.scale_log2;
   uint32_t s_full_ph = 0;
   uint32_t total_pv = 0;
+  uint32_t stg_ph = 0;  // bit b: phase of this warp's staging-buffer-b load barrier (merging epilogues)
   bool ok = true;
 
   for (int n_item = 0;; ++n_item) {
@@ -770,7 +885,14 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
         orows = p.shard_rows;
       }
       const size_t o_idx = (((size_t)it.b * orows + orow) * p.H + it.h) * D;
-      if (n_kept > 0) {
+      if (p.o_merge) {
+        // Merge into the running result: rows that saw no key of this launch's range keep it unchanged.
+        if (n_kept > 0) {
+          ok = merge_epilogue<D, kPair>(p, tm, sbase, bars, tO, it, q_row, row, warp, lane, lane_t, row_ok, l,
+                                        m_used, total_pv, stg_ph, abort_flag);
+          if (!ok) break;
+        }
+      } else if (n_kept > 0) {
         ok = mbar_wait(bars.pv_done(lane_t), (total_pv - 1) & 1, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
@@ -837,7 +959,7 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
           for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
         }
       }
-      if (row_ok && p.lse)
+      if (row_ok && p.lse && !p.o_merge)
         p.lse[((size_t)it.b * p.H + it.h) * p.S + q_row] =
             (l > 0.f && m_used != -INFINITY) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
@@ -871,6 +993,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   bars.pv_done0 = bars.p_full0 + 16;
   bars.o_done0 = bars.pv_done0 + 16;
   bars.drain = bars.o_done0 + 16;
+  bars.stg_full0 = bars.drain + 8;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   ItemRing ir;
@@ -895,6 +1018,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int k = 0; k < 2; ++k)  // o_done[0..1] counters
       *reinterpret_cast<volatile uint32_t*>(smem + C::kBarOff + (bars.o_done0 - bar0) + 8 * k) = 0u;
     mbar_init(bars.drain, 2);
+    for (int k = 0; k < 16; ++k) mbar_init(bars.stg_full0 + 8u * k, 1);
     *abort_flag = 0;
     *reinterpret_cast<volatile uint32_t*>(smem + C::kMiscOff + 8) = 0u;  // items published
     for (int k = 0; k < 8; ++k)                                          // items read, per softmax warp
@@ -1086,13 +1210,14 @@ sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
     p.n_items = (int)items;
   }
   // A causal launch over keys from kv_begin: queries before kv_begin see none of them.  Whole leading
-  // work units of such rows get no item; their rows are written here (O = 0, lse = -inf) at HBM speed.
+  // work units of such rows get no item; their rows are written here (O = 0, lse = -inf) at HBM speed,
+  // except when the launch merges into a running result, which those rows keep unchanged.
   p.qp_skip = 0;
   if (p.causal && p.kv_begin > 0 && p.n_shards == 1 && !p.item_list && !p.row_ptr) {
     const int unit_rows = (pair ? 4 : 2) * kTile;
     p.qp_skip = p.kv_begin / unit_rows < p.n_qpairs ? p.kv_begin / unit_rows : p.n_qpairs;
     const int rows = p.qp_skip * unit_rows < p.S ? p.qp_skip * unit_rows : p.S;
-    if (rows > 0) {
+    if (rows > 0 && !p.o_merge) {
       const int h0 = p.chunk_h0[0], h1 = p.chunk_h0[p.n_chunks];
       const long long n = (long long)p.B * rows * (h1 - h0) * p.D * (p.o_f32 ? 4 : 2) / 16;
       long long blocks = (n + 255) / 256;

@@ -29,6 +29,8 @@ struct AttnParams {
   void* o;          // bf16 or fp32 BSHD
   int o_f32;
   float* lse;       // [B, H, S] or nullptr
+  int o_merge;      // 1: o (fp32) and lse hold a running result that this launch's rows are merged into in
+                    // place (log-sum-exp rule); rows that see no key of the range are left untouched
   const int* item_list; // device list of work-item ids (nullptr: items 0 .. n_items-1); ids index the
                         // one-chunk layout (b * H + h) * n_qpairs + qp, and ids outside it are skipped
   int item_space;       // number of valid ids (B * H * n_qpairs) when item_list is set

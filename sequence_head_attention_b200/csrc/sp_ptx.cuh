@@ -22,7 +22,7 @@ enum : unsigned int {
   ERR_TIMEOUT_O_FREE = 1u << 7,
   ERR_TIMEOUT_DRAIN = 1u << 8,
   ERR_TIMEOUT_DEBUG = 1u << 9,
-  // 1u << 10: unused
+  ERR_TIMEOUT_STG = 1u << 10,        // a merging epilogue's load of the running O
   ERR_TIMEOUT_ITEM = 1u << 11,       // waiting for the next work-item id
   ERR_TIMEOUT_ITEM_FREE = 1u << 12,  // waiting for a work-item slot to be read by every role
   ERR_ANY_TIMEOUT = 0x1fffu,
@@ -166,6 +166,9 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int
 }
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
+}
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& x, uint32_t& y, uint32_t& z, uint32_t& w) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(w) : "r"(addr) : "memory");
 }
 __device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Waits until this thread's committed bulk stores have finished reading shared memory / have completed.

@@ -49,6 +49,7 @@ def lib() -> ctypes.CDLL:
                 "sp_attn_fwd_workspace_bytes": (Z, [I, I, I, I, I, I]),
                 "sp_attn_fwd": (I, [P, P, P, P, P, I, I, I, I, P, I, I, I, P, P, Z, P]),
                 "sp_attn_fwd_partial": (I, [P, P, P, P, P, I, I, I, I, I, I, I, P, P, Z, P]),
+                "sp_attn_fwd_partial_merge": (I, [P, P, P, P, P, I, I, I, I, I, I, I, P, P, Z, P]),
                 "sp_merge_partials": (I, [P, P, I, P, P, I, I, I, I, I, P]),
                 "sp_seq_to_head_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_head_to_seq_relayout": (I, [P, P, I, I, I, I, I, I, P]),
@@ -192,6 +193,7 @@ def sp_attn_fwd_partial(q, k, v, o_part, lse_part, kv_begin, kv_end, causal=Fals
     _bshd(o_part, "o_part", torch.float32)
     _same_device((k, v, o_part), q)
     B, S, H, D = q.shape
+    _need(tuple(o_part.shape) == (B, S, H, D), "o_part must be [B, S, H, D]")
     _check_lse(lse_part, B, H, S, q.device)
     if block_mask is not None:
         _check_mask(block_mask, H, S, q.device)
@@ -205,6 +207,31 @@ def sp_attn_fwd_partial(q, k, v, o_part, lse_part, kv_begin, kv_end, causal=Fals
                                    _stream(stream))
     _check("sp_attn_fwd_partial", st)
     return o_part, lse_part
+
+
+def sp_attn_fwd_partial_merge(q, k, v, o_acc, lse_acc, kv_begin, kv_end, causal=False, block_mask=None,
+                              workspace=None, stream=None):
+    """One KV block [kv_begin, kv_end) merged in place into the running result o_acc (fp32 [B,S,H,D]) and
+    lse_acc (fp32 [B,H,S]); rows that see no key of the block are left untouched."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _bshd(t, n)
+    _bshd(o_acc, "o_acc", torch.float32)
+    _same_device((k, v, o_acc), q)
+    B, S, H, D = q.shape
+    _need(tuple(o_acc.shape) == (B, S, H, D), "o_acc must be [B, S, H, D]")
+    _check_lse(lse_acc, B, H, S, q.device)
+    if block_mask is not None:
+        _check_mask(block_mask, H, S, q.device)
+    ws_bytes = sp_attn_fwd_workspace_bytes(B, S, H, D, 1, block_mask is not None)
+    if workspace is None and ws_bytes > 0:
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=q.device)
+    st = lib().sp_attn_fwd_partial_merge(_ptr(q), _ptr(k), _ptr(v), _ptr(o_acc), _ptr(lse_acc), B, S, H, D,
+                                         int(kv_begin), int(kv_end), int(bool(causal)), _ptr(block_mask),
+                                         _ptr(workspace),
+                                         0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                         _stream(stream))
+    _check("sp_attn_fwd_partial_merge", st)
+    return o_acc, lse_acc
 
 
 def sp_merge_partials(o_parts, lse_parts, o, lse=None, stream=None):

@@ -8,8 +8,10 @@ UlyssesStep   video-DiT shape: Q, K, V arrive as P sequence shards (one buffer p
               head chunks split at the rank boundaries; head -> seq relayout of O back to sequence shards.
               With fused=True each rank's attention reads the sequence shards and writes O into them
               directly (sp_attn_fwd_seq_sharded), with the same result and no relayout pass.
-RingStep      long causal shape: 8 contiguous KV blocks, one partial launch each (every query against one
-              block, fp32 partials), then the log-sum-exp re-merge into bf16 O and fp32 LSE.
+RingStep      long causal shape: 8 contiguous KV blocks, one launch each (every query against one block),
+              the first writing the running fp32 result and every later one merging its rows into it in
+              place (log-sum-exp rule), then the running O rounded to bf16.  The standalone re-merge of
+              materialised partials (sp_merge_partials) is kept for its own measurement.
 SparseStep    block-sparse DiT shape: tile-list build from the mask, then one attention launch that
               skips dropped tiles.
 """
@@ -99,35 +101,54 @@ class UlyssesStep:
 
 
 class RingStep:
-    def __init__(self, w: Workload, q, k, v, device="cuda"):
+    def __init__(self, w: Workload, q, k, v, device="cuda", with_partials=False):
         self.w = w
         B, S, H, D = w.B, w.S, w.H, w.D
         self.q, self.k, self.v = q.to(device), k.to(device), v.to(device)
         n = w.n_kv_blocks
         self.blk = (S + n - 1) // n
-        self.o_parts = [torch.empty((B, S, H, D), dtype=torch.float32, device=device) for _ in range(n)]
-        self.l_parts = [torch.empty((B, H, S), dtype=torch.float32, device=device) for _ in range(n)]
-        self.o = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=device)
+        self.blocks = [(i * self.blk, min(S, (i + 1) * self.blk)) for i in range(n) if i * self.blk < S]
+        self.o_acc = torch.empty((B, S, H, D), dtype=torch.float32, device=device)
         self.lse = torch.empty((B, H, S), dtype=torch.float32, device=device)
-        self.attn_launches = n
-        self.launches = n + 1
+        self.o = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=device)
+        self.attn_launches = len(self.blocks)
+        self.launches = len(self.blocks) + 1  # the block launches and the bf16 rounding
         self.flops = w.flops()
-        # merge: read n fp32 partials (O and LSE), write bf16 O and fp32 LSE
+        # the bf16 rounding of the running O: read fp32, write bf16
+        self.convert_bytes = B * S * H * D * (4 + 2)
+        # standalone re-merge of n materialised partials: read n fp32 partials (O and LSE), write bf16 O, fp32 LSE
         self.merge_bytes = n * (B * S * H * D * 4 + B * H * S * 4) + B * S * H * D * 2 + B * H * S * 4
+        self.o_parts = self.l_parts = None
+        if with_partials:
+            self.o_parts = [torch.empty((B, S, H, D), dtype=torch.float32, device=device) for _ in range(n)]
+            self.l_parts = [torch.empty((B, H, S), dtype=torch.float32, device=device) for _ in range(n)]
+            self.o_merged = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=device)
+            self.lse_merged = torch.empty((B, H, S), dtype=torch.float32, device=device)
 
     def attention(self, stream=None):
-        S = self.w.S
-        for i in range(self.w.n_kv_blocks):
-            a, e = i * self.blk, min(S, (i + 1) * self.blk)
+        """The ring's rounds: the first block's partial into the running result, later blocks merged in."""
+        causal = self.w.causal
+        a, e = self.blocks[0]
+        spattn.sp_attn_fwd_partial(self.q, self.k, self.v, self.o_acc, self.lse, a, e, causal=causal, stream=stream)
+        for a, e in self.blocks[1:]:
+            spattn.sp_attn_fwd_partial_merge(self.q, self.k, self.v, self.o_acc, self.lse, a, e, causal=causal,
+                                             stream=stream)
+
+    def finish(self, stream=None):
+        spattn.sp_convert_f32_to_bf16(self.o_acc, self.o, stream=stream)
+
+    def run(self, stream=None):
+        self.attention(stream)
+        self.finish(stream)
+
+    def partials(self, stream=None):
+        """Every block's partial materialised (sp_attn_fwd_partial), the input of the standalone merge."""
+        for i, (a, e) in enumerate(self.blocks):
             spattn.sp_attn_fwd_partial(self.q, self.k, self.v, self.o_parts[i], self.l_parts[i], a, e,
                                        causal=self.w.causal, stream=stream)
 
     def merge(self, stream=None):
-        spattn.sp_merge_partials(self.o_parts, self.l_parts, self.o, self.lse, stream=stream)
-
-    def run(self, stream=None):
-        self.attention(stream)
-        self.merge(stream)
+        spattn.sp_merge_partials(self.o_parts, self.l_parts, self.o_merged, self.lse_merged, stream=stream)
 
     def workspace_for_fwd(self):
         w = self.w

@@ -124,3 +124,16 @@ def test_binding_refuses_bad_masks_and_lse_before_any_call():
     i32 = torch.zeros(H * 64, dtype=torch.int32)
     with pytest.raises(ValueError, match="CUDA"):
         spattn.sp_build_tile_list(good, S, i32, i32, i32)
+
+
+def test_partial_merge_rejects_on_host(L):
+    f = L.sp_attn_fwd_partial_merge
+    q, o, l = 1 << 24, 2 << 24, 3 << 24  # distinct, 16-byte aligned, never dereferenced
+    assert f(q, q, q, o, None, 1, 256, 4, 64, 0, 128, 0, None, None, 0, None) == spattn.SP_ERR_INVALID_ARG
+    assert f(q, q, q, o, l, 1, 256, 4, 64, 10, 5, 0, None, None, 0, None) == spattn.SP_ERR_INVALID_ARG
+    assert f(q, q, q, o, l, 1, 256, 4, 64, 0, 300, 0, None, None, 0, None) == spattn.SP_ERR_INVALID_ARG
+    assert f(q, q, q, o, l, 1, 256, 4, 64, 64, 256, 0, 16, None, 0, None) == spattn.SP_ERR_INVALID_ARG
+    assert f(q, q, q, q + 64, l, 1, 256, 4, 64, 0, 256, 0, None, None, 0, None) == spattn.SP_ERR_INVALID_ARG
+    assert f(q, q, q, o, o + 64, 1, 256, 4, 64, 0, 256, 0, None, None, 0, None) == spattn.SP_ERR_INVALID_ARG
+    assert f(q, q, q, o, l, 1, 256, 4, 96, 0, 256, 0, None, None, 0, None) == spattn.SP_ERR_INVALID_ARG
+    assert f(q, q, q, o, l, 1, 256, 4, 64, 128, 128, 0, None, None, 0, None) == spattn.SP_OK  # empty: no launch

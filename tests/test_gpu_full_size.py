@@ -58,23 +58,33 @@ def test_video_dit_ulysses_step():
 
 
 def test_ring_causal_partials_and_merge():
+    """The ring step the benchmark times (8 KV blocks of 7168: the first block's partial, seven blocks merged
+    in place, the running O rounded to bf16), the standalone re-merge of the 8 materialised partials, and
+    sp_attn_fwd with n_kv_blocks = 8: each checked on sampled rows against the oracle."""
     w = synth.WORKLOADS["ring_causal"]
     q, k, v = synth.qkv(w.B, w.S, w.H, w.D, seed=0, scale=w.scale)
     blk = w.S // w.n_kv_blocks
     rows = synth.sample_rows(w.S, N_ROWS, seed=1, must=[blk - 1, blk, 4 * blk, 4 * blk - 1, w.S - blk])
     ref = _oracle_rows(q, k, v, rows, causal=True)
-    step = workloads.RingStep(w, q, k, v)
+    step = workloads.RingStep(w, q, k, v, with_partials=True)
     step.run()
     torch.cuda.synchronize()
     assert spattn.sp_check_device_error() == spattn.SP_OK
     o_s, l_s = _sampled(step.o, step.lse, rows)
     assert_close(o_s, ref[0], l_s, ref[1])
+    step.partials()
+    step.merge()
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    o_s, l_s = _sampled(step.o_merged, step.lse_merged, rows)
+    assert_close(o_s, ref[0], l_s, ref[1])
     # one call with n_kv_blocks = 8 does the same partials and merge
     o2 = torch.empty_like(step.o)
     l2 = torch.empty_like(step.lse)
+    del step.o_parts, step.l_parts
     spattn.sp_attn_fwd(step.q, step.k, step.v, o2, l2, n_kv_blocks=w.n_kv_blocks, causal=True,
                        workspace=step.workspace_for_fwd())
-    assert torch.equal(o2, step.o) and torch.equal(l2, step.lse)
+    assert torch.equal(o2, step.o_merged) and torch.equal(l2, step.lse_merged)
 
 
 def test_block_sparse_dit():
