@@ -57,10 +57,13 @@ def _load(path: str | None = None):
             lib.orc_merge.argtypes = [P, P, I, P, P, I, I, I, I]
             lib.orc_seq_to_head.argtypes = [P, P, I, I, I, I, I, I]
             lib.orc_head_to_seq.argtypes = [P, P, I, I, I, I, I, I]
+            lib.orc_split_heads.argtypes = [P, P, I, I, I, I, I, I]
+            lib.orc_merge_heads.argtypes = [P, P, I, I, I, I, I, I]
             lib.orc_tile_list.argtypes = [P, I, I, I, P, P, ctypes.c_long]
             lib.orc_attn_bwd.argtypes = [P, P, P, P, P, P, P, I, I, I, I, I, I]
             for f in (lib.orc_attn, lib.orc_attn_probs, lib.orc_merge, lib.orc_seq_to_head,
-                      lib.orc_head_to_seq, lib.orc_tile_list, lib.orc_attn_bwd):
+                      lib.orc_head_to_seq, lib.orc_split_heads, lib.orc_merge_heads, lib.orc_tile_list,
+                      lib.orc_attn_bwd):
                 f.restype = ctypes.c_int
             _libs[key] = lib
     return _libs[key]
@@ -258,6 +261,37 @@ def head_to_seq(in_ranks, S, *, lib=None):
     if rc:
         raise ValueError(f"orc_head_to_seq failed ({rc})")
     return outs
+
+
+def split_heads(x, P, *, lib=None):
+    """One rank's half of the Ulysses all-to-all on the way in ("HCMS", abstract: all-to-all sequence
+    parallelism, here between processes): its sequence shard x [B, S, H, D] cut into P head groups,
+    out_r [B, S, H/P, D] = x[:, :, r*H/P : (r+1)*H/P] (the block it sends to rank r)."""
+    xa = np.ascontiguousarray(x)
+    B, S, H, D = xa.shape
+    if H % P:
+        raise ValueError("bad head count")
+    outs = [np.zeros((B, S, H // P, D), dtype=xa.dtype) for _ in range(P)]
+    op = (ctypes.c_void_p * P)(*[a.ctypes.data for a in outs])
+    rc = _load(lib).orc_split_heads(xa.ctypes.data_as(ctypes.c_void_p), ctypes.cast(op, ctypes.c_void_p), P, B, S,
+                                    H, D, xa.itemsize)
+    if rc:
+        raise ValueError(f"orc_split_heads failed ({rc})")
+    return outs
+
+
+def merge_heads(parts, *, lib=None):
+    """The way back: P head groups [B, S, H/P, D] (group r from rank r) joined into [B, S, H, D]."""
+    ins = [np.ascontiguousarray(a) for a in parts]
+    P = len(ins)
+    B, S, Hl, D = ins[0].shape
+    out = np.zeros((B, S, Hl * P, D), dtype=ins[0].dtype)
+    ip = (ctypes.c_void_p * P)(*[a.ctypes.data for a in ins])
+    rc = _load(lib).orc_merge_heads(ctypes.cast(ip, ctypes.c_void_p), out.ctypes.data_as(ctypes.c_void_p), P, B, S,
+                                    Hl * P, D, ins[0].itemsize)
+    if rc:
+        raise ValueError(f"orc_merge_heads failed ({rc})")
+    return out
 
 
 def tile_list(block_mask, *, lib=None):

@@ -37,6 +37,10 @@
  *                 Ulysses).  Rank r holds sequence shard r of all heads before, and all positions of
  *                 head group r after:  out_r[b, s, h', :] = in_{s / (S/P)}[b, s % (S/P), r*H/P + h', :].
  *                 Byte copies, element by element.
+ *  orc_split_heads / orc_merge_heads
+ *                 The local halves of that all-to-all when the ranks are separate processes: a rank cuts
+ *                 its sequence shard into P head groups before the exchange (split) and joins the head
+ *                 groups it gets back after it (merge).  Byte copies, element by element.
  *  orc_tile_list  The compacted per-(head, query tile) list of kept key tiles of a block mask, in
  *                 increasing key-tile order (CSR: row_ptr, col_idx).
  *  orc_attn_bwd   The gradients of the attention above (dense or causal, all keys) for an upstream
@@ -323,6 +327,45 @@ int orc_head_to_seq(const void* const* in_ranks, void* const* out_ranks, int P, 
                                      ((((size_t)b * S + s) * Hl + src_h) * D) * elem_bytes;
           unsigned char* dst =
               (unsigned char*)out_ranks[r] + ((((size_t)b * Sl + sl) * H + h) * D) * elem_bytes;
+          for (size_t e = 0; e < (size_t)D * elem_bytes; ++e) dst[e] = src[e];
+        }
+  return ORC_OK;
+}
+
+/*
+ * The two local halves of the Ulysses all-to-all when the P ranks are P processes ("HCMS ...", abstract:
+ * all-to-all based sequence parallelism).  Before the exchange, rank g cuts its sequence shard [B, S, H, D]
+ * (S = its own positions) into P head groups, one per destination rank:
+ *   split_heads:  out_r[b, s, h', :] = in[b, s, r*H/P + h', :]          (out_r is [B, S, H/P, D])
+ * after the way back it joins the P head groups it received into its sequence shard:
+ *   merge_heads:  out[b, s, r*H/P + h', :] = in_r[b, s, h', :]
+ * Byte copies, element by element.
+ */
+int orc_split_heads(const void* in, void* const* out_ranks, int P, int B, int S, int H, int D, int elem_bytes) {
+  if (P < 1 || B < 0 || S < 0 || H < 1 || D < 1 || elem_bytes < 1 || H % P) return ORC_EINVAL;
+  const int Hl = H / P;
+  for (int r = 0; r < P; ++r)
+    for (int b = 0; b < B; ++b)
+      for (int s = 0; s < S; ++s)
+        for (int hh = 0; hh < Hl; ++hh) {
+          const unsigned char* src =
+              (const unsigned char*)in + ((((size_t)b * S + s) * H + r * Hl + hh) * D) * elem_bytes;
+          unsigned char* dst = (unsigned char*)out_ranks[r] + ((((size_t)b * S + s) * Hl + hh) * D) * elem_bytes;
+          for (size_t e = 0; e < (size_t)D * elem_bytes; ++e) dst[e] = src[e];
+        }
+  return ORC_OK;
+}
+
+int orc_merge_heads(const void* const* in_ranks, void* out, int P, int B, int S, int H, int D, int elem_bytes) {
+  if (P < 1 || B < 0 || S < 0 || H < 1 || D < 1 || elem_bytes < 1 || H % P) return ORC_EINVAL;
+  const int Hl = H / P;
+  for (int r = 0; r < P; ++r)
+    for (int b = 0; b < B; ++b)
+      for (int s = 0; s < S; ++s)
+        for (int hh = 0; hh < Hl; ++hh) {
+          const unsigned char* src =
+              (const unsigned char*)in_ranks[r] + ((((size_t)b * S + s) * Hl + hh) * D) * elem_bytes;
+          unsigned char* dst = (unsigned char*)out + ((((size_t)b * S + s) * H + r * Hl + hh) * D) * elem_bytes;
           for (size_t e = 0; e < (size_t)D * elem_bytes; ++e) dst[e] = src[e];
         }
   return ORC_OK;

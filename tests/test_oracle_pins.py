@@ -362,6 +362,35 @@ def test_relayout_byte_exact_for_float_payloads():
     assert outs[1].tobytes() == full[:, :, 2:].copy().tobytes()
 
 
+@pytest.mark.parametrize("P,B,S,H,D", [(4, 1, 6, 8, 6), (2, 2, 5, 6, 3), (1, 2, 3, 3, 4), (3, 1, 4, 9, 2)])
+def test_split_and_merge_heads_against_slices_and_the_exchange(P, B, S, H, D):
+    """The local halves of a multi-process Ulysses exchange: split_heads equals numpy slicing of the head
+    axis, merge_heads inverts it, and split on every rank followed by the all-to-all block transpose
+    (rank r receives block r of every rank, in rank order along the sequence) is the pinned seq_to_head."""
+    Sg = S * P  # the global sequence: rank g holds positions [g S, (g + 1) S)
+    full = RNG.integers(0, 2**16, size=(B, Sg, H, D), dtype=np.uint16)
+    shards = [full[:, g * S:(g + 1) * S].copy() for g in range(P)]
+    sent = [oracle.split_heads(shards[g], P) for g in range(P)]  # sent[g][r]: rank g's block for rank r
+    for g in range(P):
+        for r in range(P):
+            assert np.array_equal(sent[g][r], shards[g][:, :, r * (H // P):(r + 1) * (H // P)])
+        assert np.array_equal(oracle.merge_heads(sent[g]), shards[g])
+    ulysses = oracle.seq_to_head(shards, H)
+    for r in range(P):
+        received = np.concatenate([sent[g][r] for g in range(P)], axis=1)
+        assert np.array_equal(received, ulysses[r])
+    # and the way back: head_to_seq equals the block transpose followed by merge_heads on every rank
+    back = oracle.head_to_seq(ulysses, Sg)
+    for g in range(P):
+        got = oracle.merge_heads([ulysses[r][:, g * S:(g + 1) * S] for r in range(P)])
+        assert np.array_equal(got, back[g]) and np.array_equal(got, shards[g])
+    # a mistake in the head offset is caught: swapping two groups breaks the identity
+    if P > 1:
+        swapped = list(sent[0])
+        swapped[0], swapped[1] = swapped[1], swapped[0]
+        assert not np.array_equal(oracle.merge_heads(swapped), shards[0])
+
+
 def test_tile_list_against_nonzero():
     mask = (RNG.random((3, 7, 7)) < 0.4).astype(np.uint8)
     mask[1, 2, :] = 0
