@@ -59,11 +59,22 @@ def dist_env():
             int(os.environ.get("LOCAL_RANK", "0")))
 
 
-def init_dist(backend: str, timeout_s: int = 120):
+def init_dist(backend: str, timeout_s: int = 120, always: bool = False):
+    """Join the process group (torchrun's environment) when there are several ranks, or always (a group of
+    one without torchrun, so that code issuing collectives also runs on a single GPU)."""
     import torch.distributed as dist
     rank, world, _ = dist_env()
-    if world > 1 and not dist.is_initialized():
+    if dist.is_initialized():
+        return rank, world
+    if world > 1 or (always and "MASTER_ADDR" in os.environ):
         dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
+    elif always:
+        import socket
+        with socket.socket() as s:
+            s.bind(("127.0.0.1", 0))
+            port = s.getsockname()[1]
+        dist.init_process_group(backend=backend, init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=timeout_s))
     return rank, world
 
 
@@ -637,6 +648,78 @@ def free_gpu():
     torch.cuda.empty_cache()
 
 
+def run_sp(args):
+    """Real sequence parallelism over the N ranks (one GPU each): every rank holds only its sequence shard of
+    the one global problem; Ulysses (video_dit) exchanges Q, K, V and O with NCCL all-to-alls, the ring
+    (ring_causal) passes the KV blocks round the ranks with NCCL point-to-point sends, the library's kernels
+    computing in between (sequence_head_attention_b200/dist.py).  Total work is fixed: strong scaling."""
+    import torch
+    from sequence_head_attention_b200 import dist as sp_dist
+    from sequence_head_attention_b200 import spattn
+
+    rank, world, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist("nccl", timeout_s=180, always=True)
+    spattn.lib()
+    stream = torch.cuda.current_stream(dev)
+    peaks = measured_peaks()
+    wname = "video_dit" if args.sp == "ulysses" else "ring_causal"
+    w, q, k, v, _ = build_inputs(wname, seed=0)  # the same global problem on every rank
+    Sl = w.S // world
+    qs, ks, vs = (t[:, rank * Sl:(rank + 1) * Sl].contiguous().to(dev) for t in (q, k, v))
+    del q, k, v
+    if args.sp == "ulysses":
+        sp = sp_dist.UlyssesAttention(w.B, w.S, w.H, w.D, head_chunks=w.head_chunks, causal=w.causal, device=dev)
+        flops_rank = w.flops() / world  # every rank attends H/P heads over the whole sequence
+    else:
+        sp = sp_dist.RingAttention(w.B, w.S, w.H, w.D, causal=w.causal, device=dev)
+        # causal: rank r's queries see the blocks of ranks 0..r (its own one causally)
+        blk = 4.0 * w.B * w.H * Sl * Sl * w.D
+        flops_rank = blk * (rank + (0.5 if w.causal else 1.0)) if w.causal else blk * world
+    o = torch.empty_like(qs)
+    for _ in range(args.warmup):
+        sp.forward(qs, ks, vs, out=o)
+    torch.cuda.synchronize(dev)
+    check_device("during the sequence-parallel warm-up")
+    sampler = clock_sampler(dev).start()
+    barrier()
+    torch.cuda.synchronize(dev)
+    timer = Timer(stream)
+    t0, t1 = timer.E(), timer.E()
+    t0.record(stream)
+    for _ in range(args.steps):
+        sp.forward(qs, ks, vs, out=o, phase=timer.phase)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    clocks = sampler.stop()
+    check_device("during the sequence-parallel steps")
+    ms = max_over_ranks(t0.elapsed_time(t1), device=dev)
+    value = w.flops() * args.steps / (ms / 1000.0) / 1e12
+    attn_ms = sum(timer.spans("attn")) / args.steps  # this rank's attention launches per step
+    exch = timer.spans("exchange")
+    roofline = tensor_roofline(flops_rank, attn_ms, peaks)
+    roofline["note"] = "this rank's attention launches of one step, timed together"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": dict(config_of(w, wname, 1), parallelism=f"{args.sp}{world}",
+                           global_batch=w.B, sp=f"{args.sp}: each rank holds S/{world} positions of Q, K, V"),
+            "roofline": roofline, "cpu_baseline": None, "e2e": None,
+            "gpu_launches": None, "clocks": clocks, "impl": "ours",
+            "kernels": {"rank0": {"attention_ms_per_step": attn_ms, "flops_per_step": flops_rank,
+                                  "exchange_ms_per_step": sum(exch) / args.steps if exch else 0.0,
+                                  "bytes_sent_per_step": sp.bytes_exchanged(),
+                                  "rounds": getattr(sp, "rounds", None)}}}
+    emit(line, rank)
+    del sp
+    finish_dist()
+    return 0
+
+
 def run_ours(args):
     import torch
     from sequence_head_attention_b200 import spattn
@@ -715,6 +798,10 @@ def main(argv=None):
                     help="all (default): the S=32K headline plus every other configuration under kernels; "
                          "a single full-size workload for profiling captures; tiny_dense / megatron: "
                          "reference arm only")
+    ap.add_argument("--sp", choices=["replicas", "ulysses", "ring"], default="replicas",
+                    help="replicas (default): every rank runs its own batch of every workload (weak scaling); "
+                         "ulysses / ring: one global problem sequence-parallel over the ranks with NCCL "
+                         "collectives (video_dit all-to-all, ring_causal ring; strong scaling)")
     ap.add_argument("--ulysses", choices=["fused", "relayout"], default="fused",
                     help="video_dit step: attention straight on the sequence shards (fused), or the seq->head "
                          "relayout, per-rank attention and head->seq relayout")
@@ -736,6 +823,8 @@ def main(argv=None):
         return run_reference(args)
     if (args.seq_len or args.ranks) and args.workload == "all":
         ap.error("--seq-len / --ranks apply to a single --workload")
+    if args.sp != "replicas":
+        return run_sp(args)
     return run_ours(args)
 
 

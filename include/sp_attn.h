@@ -218,6 +218,23 @@ SP_API sp_status sp_head_to_seq_relayout(const void* const* in_ranks, void* cons
                                   int S, int H, int D, int elem_bytes, sp_stream stream);
 
 /*
+ * The local halves of the Ulysses all-to-all when the P ranks are P processes on P GPUs ("HCMS", abstract:
+ * all-to-all based sequence parallelism; "db-SP", abstract: parallelism along the head dimension as in
+ * Ulysses).  The exchange itself is a collective between contiguous per-destination blocks (NCCL
+ * all-to-all); around it, each rank copies its own sequence shard x [B, S, H, D] (S: the rank's own
+ * positions) into P head groups, and back:
+ *   sp_split_heads:  out_ranks[r] [B, S, H/P, D] = x[:, :, r*H/P : (r+1)*H/P, :]  (block sent to rank r)
+ *   sp_merge_heads:  out[:, :, r*H/P : (r+1)*H/P, :] = in_ranks[r] [B, S, H/P, D]  (block from rank r)
+ * Bit-exact byte copies.  Requires 1 <= P <= SP_MAX_RANKS, H % P == 0, elem_bytes in {1, 2, 4, 8},
+ * (D * elem_bytes) % 16 == 0, 16-byte aligned buffers, no overlap between any input and any output or
+ * between two outputs.  out_ranks / in_ranks are host arrays of P device pointers.
+ */
+SP_API sp_status sp_split_heads(const void* in, void* const* out_ranks, int P, int B, int S, int H, int D,
+                                int elem_bytes, sp_stream stream);
+SP_API sp_status sp_merge_heads(const void* const* in_ranks, void* out, int P, int B, int S, int H, int D,
+                                int elem_bytes, sp_stream stream);
+
+/*
  * One Ulysses rank's attention straight on the sequence shards, with both relayouts folded into the
  * kernel ("HCMS: ... Ulysses ... all-to-all", abstract: each rank attends over the whole sequence for its
  * share of the heads; "LLM Lab Notes 05", section 2: per head q @ k^T / sqrt(d), softmax, @ v).  It
@@ -331,6 +348,19 @@ SP_API sp_status sp_check_device_error(sp_stream stream);
  * out, drain, debug, running-O load of a merge), for diagnosing which hand-off gave up.
  */
 SP_API sp_status sp_check_device_error_bits(sp_stream stream, unsigned int* bits);
+
+/*
+ * Launch overlap (default off).  With it on, every attention launch (sp_attn_fwd and the other attention
+ * entry points) may start while the kernel enqueued just before it on the same stream is still finishing:
+ * its CTAs take the SMs that kernel frees (programmatic dependent launch), which fills the tail of a
+ * sequence of attention launches such as one launch per Ulysses rank or per ring round.  An overlapped
+ * launch reads only q, k and v early: it writes o and lse (and sp_attn_fwd_partial_merge reads its running
+ * result) only after the kernel before it has completed, and a masked or item-list launch waits for it
+ * before reading anything (that kernel may have built its tile list).  The caller promises that q, k and
+ * v are not written by the kernel enqueued just before the launch.  Kernels enqueued after an attention
+ * launch wait for it as usual.  Applies to later launches; process-wide.
+ */
+SP_API void sp_set_launch_overlap(int enable);
 
 /* Time limit of every device-side wait, in nanoseconds (default 2e9).  Applies to later launches. */
 SP_API void sp_set_wait_timeout_ns(unsigned long long ns);

@@ -10,5 +10,5 @@ from .spattn import (  # noqa: F401
     sp_attn_fwd_partial_merge, sp_attn_fwd_seq_sharded, sp_attn_fwd_sparse_noalloc, sp_attn_fwd_workspace_bytes,
     sp_build_tile_list, sp_check_device_error, sp_convert_f32_to_bf16, sp_dbsp_plan, sp_dbsp_rank_items,
     sp_dbsp_unit_costs, sp_debug_wait_timeout, sp_head_to_seq_relayout, sp_merge_partials,
-    sp_seq_to_head_relayout, sp_set_wait_timeout_ns, sp_status_string, sp_version,
+    sp_merge_heads, sp_seq_to_head_relayout, sp_set_wait_timeout_ns, sp_split_heads, sp_status_string, sp_version,
 )

@@ -24,6 +24,7 @@ int g_num_sms[kMaxDevices] = {};
 unsigned int* g_err_addr[kMaxDevices] = {};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 unsigned long long g_timeout_ns = 2000000000ull;
+bool g_overlap = false;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -118,6 +119,8 @@ int num_sms(int device) {
 
 unsigned long long wait_timeout_ns() { return g_timeout_ns; }
 
+bool launch_overlap() { return g_overlap; }
+
 unsigned int* device_error_word() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
@@ -195,6 +198,11 @@ const char* sp_status_string(sp_status s) {
 }
 
 const char* sp_version(void) { return "spattn 0.1 (sm_100a)"; }
+
+void sp_set_launch_overlap(int enable) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_overlap = enable != 0;
+}
 
 void sp_set_wait_timeout_ns(unsigned long long ns) {
   std::lock_guard<std::mutex> lk(g_mu);
@@ -653,6 +661,43 @@ sp_status sp_convert_f32_to_bf16(const float* in, void* out, long long n, sp_str
   const uintptr_t a0 = reinterpret_cast<uintptr_t>(in), b0 = reinterpret_cast<uintptr_t>(out);
   if (n > 0 && a0 < b0 + (size_t)n * 2 && b0 < a0 + (size_t)n * 4) return SP_ERR_INVALID_ARG;
   return launch_f32_to_bf16(in, out, n, as_stream(stream));
+}
+
+static sp_status head_groups_common(const void* const* ins, int n_in, void* const* outs, int n_out, bool split, int P,
+                                    int B, int S, int H, int D, int elem_bytes, sp_stream stream) {
+  if (!ins || !outs || P < 1 || P > SP_MAX_RANKS || B < 1 || S < 0 || H < 1 || D < 1) return SP_ERR_INVALID_ARG;
+  if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8) return SP_ERR_INVALID_ARG;
+  if (H % P != 0 || ((long long)D * elem_bytes) % 16 != 0) return SP_ERR_INVALID_ARG;
+  if ((double)B * S * H * D * elem_bytes > 9.0e15) return SP_ERR_INVALID_ARG;
+  const long long whole = (long long)B * S * H * D * elem_bytes, group = whole / P;
+  const long long in_bytes = split ? whole : group, out_bytes = split ? group : whole;
+  for (int r = 0; r < n_in; ++r)
+    if (!ins[r] || !aligned16(ins[r])) return SP_ERR_INVALID_ARG;
+  for (int r = 0; r < n_out; ++r)
+    if (!outs[r] || !aligned16(outs[r])) return SP_ERR_INVALID_ARG;
+  for (int r = 0; r < n_in; ++r)  // no input may overlap an output
+    for (int g = 0; g < n_out; ++g) {
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(ins[r]), b0 = reinterpret_cast<uintptr_t>(outs[g]);
+      if (a0 < b0 + out_bytes && b0 < a0 + in_bytes) return SP_ERR_INVALID_ARG;
+    }
+  for (int r = 0; r < n_out; ++r)  // nor two outputs one another
+    for (int g = r + 1; g < n_out; ++g) {
+      const uintptr_t a0 = reinterpret_cast<uintptr_t>(outs[r]), b0 = reinterpret_cast<uintptr_t>(outs[g]);
+      if (a0 < b0 + out_bytes && b0 < a0 + out_bytes) return SP_ERR_INVALID_ARG;
+    }
+  return launch_head_groups(ins, outs, split, P, B, S, H, D, elem_bytes, as_stream(stream));
+}
+
+sp_status sp_split_heads(const void* in, void* const* out_ranks, int P, int B, int S, int H, int D, int elem_bytes,
+                         sp_stream stream) {
+  const void* ins[1] = {in};
+  return head_groups_common(ins, 1, out_ranks, P, true, P, B, S, H, D, elem_bytes, stream);
+}
+
+sp_status sp_merge_heads(const void* const* in_ranks, void* out, int P, int B, int S, int H, int D, int elem_bytes,
+                         sp_stream stream) {
+  void* outs[1] = {out};
+  return head_groups_common(in_ranks, P, outs, 1, false, P, B, S, H, D, elem_bytes, stream);
 }
 
 sp_status sp_seq_to_head_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,

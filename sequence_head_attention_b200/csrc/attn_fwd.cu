@@ -65,40 +65,55 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and l are rescaled w
 #endif
 constexpr int kPolyPairs = SP_EXP2_POLY_PAIRS;
 
-template <int D, bool kPair = false>
+// kSplit: both lanes work on ONE query tile and take alternate kept key tiles of its list (lane 0 the even
+// ones, lane 1 the odd ones), each with its own running maximum, sum and O; the epilogue merges the two.
+template <int D, bool kPair = false, bool kSplit = false>
 struct Cfg {
+  static_assert(!(kPair && kSplit), "a CTA pair never splits keys");
   static constexpr int kSub = D / 64;                   // 64-column (128-byte) sub-tiles per row
   static constexpr int kTileBytes = kTile * D * 2;      // one 128 x D bf16 tile
+  static constexpr int kQTiles = kSplit ? 1 : 2;        // query tiles resident per work item
   // A K or V slot: a whole tile, or for a CTA pair this CTA's half (K: 64 of the 128 keys; V: 64 of the D
   // columns), the MMA's B operand being split by N between the two SMs.
   static constexpr int kKVBytes = kPair ? kTileBytes / 2 : kTileBytes;
   static constexpr int kKSubBytes = kPair ? 8192 : 16384;  // between the 64-column sub-tiles of a K slot
-  static constexpr int kStages = kPair ? 6 : (D == 128 ? 4 : 8);  // K/V ring slots
+  // K/V ring slots (with one query tile resident, D = 128 has room for a fifth)
+  static constexpr int kStages = kPair ? 6 : (D == 128 ? (kSplit ? 5 : 4) : 8);
   static constexpr int kQOff = 0;
-  static constexpr int kKVOff = 2 * kTileBytes;
+  static constexpr int kKVOff = kQTiles * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kKVBytes;
   // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2], drain, 8-byte
   // slots for the o_done[2] counters, and stg_full[8][2] (a merging epilogue's loads of the running O into
   // each softmax warp's staging buffers)
   static constexpr int kNumBars = 2 + 2 * kStages + 9 + 16;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  // misc: TMEM base, abort flag, published-item count, per-warp item-read counts, the item ring
+  // misc: TMEM base, abort flag, published-item count, per-warp item-read counts, the item ring (96
+  // bytes); with kSplit also the lanes' exchange: one 8-byte slot per query row (lane 1 posts its row
+  // maximum and sum, lane 0 answers with both lanes' weights) and four hand-off counters, one per TMEM
+  // lane quadrant.
+  static constexpr int kXchOff = kMiscOff + 96;
+  static constexpr int kXcntOff = kXchOff + 128 * 8;
+  static constexpr int kMiscBytes = kSplit ? 96 + 128 * 8 + 16 : 96;
   // then, 1024-aligned, staging for the O stores: per softmax warp two 4 KB buffers (32 rows x 128 bytes)
   // where they fit in the 227 KB a CTA may have, else one
-  static constexpr int kStgOff = (kMiscOff + 96 + 1023) / 1024 * 1024;
+  static constexpr int kStgOff = (kMiscOff + kMiscBytes + 1023) / 1024 * 1024;
   static constexpr int kStgBufs = kStgOff + 2 * 8 * 4096 + 1024 <= 232448 ? 2 : 1;
   static constexpr int kSmemBytes = kStgOff + kStgBufs * 8 * 4096 + 1024;  // + alignment slack
   static constexpr int kM = kPair ? 256 : 128;  // MMA rows: a pair computes both CTAs' 128 rows at once
   static constexpr uint32_t kIdescS = idesc_bf16_f32(kM, 128, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kM, D, false, true);
   static constexpr uint32_t kRowWarps = kPair ? 8u : 4u;  // softmax warps per lane over the (pair of) CTAs
+  // o_done[t] counts, per item, the softmax warps that have read out O_t: lane t's (kRowWarps), or with
+  // kSplit every softmax warp of the CTA, since each reads both lanes' O for its half of the columns
+  static constexpr uint32_t kODoneWarps = kSplit ? 8u : kRowWarps;
   static constexpr uint32_t kColS = 0;
   static constexpr uint32_t kColO = 256;
 };
 
 // every configuration fits the 227 KB of shared memory a CTA may have
 static_assert(Cfg<128, true>::kSmemBytes <= 232448 && Cfg<128, false>::kSmemBytes <= 232448 &&
-                  Cfg<64, false>::kSmemBytes <= 232448,
+                  Cfg<64, false>::kSmemBytes <= 232448 && Cfg<128, false, true>::kSmemBytes <= 232448 &&
+                  Cfg<64, false, true>::kSmemBytes <= 232448,
               "shared memory");
 
 struct Bars {
@@ -116,6 +131,7 @@ struct Bars {
 
 struct Item {
   int b, h, qp;
+  int sub;         // kSplit: which query tile of the pair (2 qp + sub) both lanes work on
   int shard;       // sequence shard holding both query tiles (0 when not sharded)
   int q_start[2];  // first row of each lane's query tile (global position)
   int q_last[2];   // last row of each lane's tile that exists (global position)
@@ -128,8 +144,11 @@ struct Item {
   bool valid_u[2];
 };
 
-template <bool kPair = false>
+template <bool kPair = false, bool kSplit = false>
 __device__ __forceinline__ Item decode_item(const AttnParams& p, int w) {
+  // kSplit: the ring carries one entry per query tile, 2 * (item id) + tile within the item's pair
+  const int sub = kSplit ? (w & 1) : 0;
+  if (kSplit) w >>= 1;
   bool id_ok = true;
   if (p.item_list) {  // an explicit list: ids of the one-chunk layout, query-tile pair as given
     w = __ldg(p.item_list + w);
@@ -159,13 +178,14 @@ __device__ __forceinline__ Item decode_item(const AttnParams& p, int w) {
   const int lp = it.qp - it.shard * p.pairs_per_shard;
   it.q_end = min(p.S, (it.shard + 1) * p.shard_rows);
   const int rk = kPair ? (int)cluster_rank() : 0;
+  it.sub = sub;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     it.valid_u[t] = false;
     it.q_last_u[t] = -1;
 #pragma unroll
     for (int rr = 0; rr < (kPair ? 2 : 1); ++rr) {
-      const int lt = kPair ? 4 * lp + 2 * rr + t : 2 * lp + t;
+      const int lt = kPair ? 4 * lp + 2 * rr + t : (kSplit ? 2 * lp + sub : 2 * lp + t);
       const int start = it.shard * p.shard_rows + lt * kTile;
       const bool valid = lt < p.tiles_per_shard && start < it.q_end;
       const int last = min(it.q_end, start + kTile) - 1;
@@ -196,6 +216,8 @@ struct StepIter {
   int key_end;     // one past that shard's last row (INT_MAX when not sharded)
   int q_last0, q_last1;
   bool v0, v1;
+  bool split;      // both lanes on one query tile: the walked tiles go to lane 0 and lane 1 in turn
+  int par;         // split: the lane that takes the next tile
   int j, n_dense;
   const int* l0;
   const int* l1;
@@ -209,7 +231,9 @@ struct StepIter {
     return lo;
   }
 
-  __device__ __forceinline__ void init(const AttnParams& p, const Item& it) {
+  __device__ __forceinline__ void init(const AttnParams& p, const Item& it, bool split_keys = false) {
+    split = split_keys;
+    par = 0;
     causal = p.causal != 0;
     kv_begin = p.kv_begin;
     q_last0 = it.q_last_u[0];
@@ -245,8 +269,19 @@ struct StepIter {
     const int t_hi = (p.kv_lim + kTile - 1) / kTile;  // exclusive
     l0 = p.col_idx;
     l1 = p.col_idx;
-    const int row0 = it.h * p.mask_T + 2 * it.qp;
+    const int row0 = it.h * p.mask_T + 2 * it.qp + (split ? it.sub : 0);
     i0 = e0 = i1 = e1 = 0;
+    if (split) {  // one list (the tile's row), dealt to the lanes in turn by next()
+      if (v0) {
+        i0 = __ldg(p.row_ptr + row0);
+        e0 = __ldg(p.row_ptr + row0 + 1);
+        const int hi0 = causal ? min(t_hi, q_last0 / kTile + 1) : t_hi;
+        if (t_lo > 0) i0 = lower_bound(l0, i0, e0, t_lo);
+        if (hi0 < p.mask_T) e0 = lower_bound(l0, i0, e0, hi0);
+      }
+      c0 = c1 = INT_MAX;
+      return;
+    }
     if (v0) {
       i0 = __ldg(p.row_ptr + row0);
       e0 = __ldg(p.row_ptr + row0 + 1);
@@ -282,6 +317,20 @@ struct StepIter {
       ++j;
       k0 = v0 && (!causal || kv_start <= q_last0);
       k1 = v1 && (!causal || kv_start <= q_last1);
+      if (split) {
+        k0 = k0 && par == 0;
+        k1 = k1 && par == 1;
+        par ^= 1;
+      }
+      return true;
+    }
+    if (split) {
+      if (i0 >= e0) return false;
+      kv_start = __ldg(l0 + i0) * kTile;
+      ++i0;
+      k0 = par == 0;
+      k1 = par == 1;
+      par ^= 1;
       return true;
     }
     const int t = min(c0, c1);
@@ -338,10 +387,10 @@ struct TMaps {
 // Producer: one warp walks the work in lockstep (all values warp-uniform); one elected lane issues the
 // TMA loads.
 // ------------------------------------------------------------------------------------------------
-template <int D, bool kPair>
+template <int D, bool kPair, bool kSplit>
 __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem, const Bars& bars,
                              const ItemRing& ir, volatile int* abort_flag) {
-  using C = Cfg<D, kPair>;
+  using C = Cfg<D, kPair, kSplit>;
   const uint32_t sbase = smem_u32(smem);
   const uint64_t tmo = p.timeout_ns;
   // A CTA pair: each CTA loads its own query tiles and its half of every K/V tile, and the bytes complete
@@ -357,15 +406,18 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
   // claiming from the launch's counter; ids go into the item ring of the CTA (or of both CTAs of the pair).
   const int n_workers = kPair ? (int)(gridDim.x >> 1) : (int)gridDim.x;
   int w = kPair ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;
+  int id = w;  // the ring entry: the item id, or with kSplit 2 * item + query tile within the item's pair
   for (;; ++n_item) {
     bool done;
     if (kPair && rk != 0) {  // rank 1 reads what rank 0 published into its ring
       ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err, true);
       if (!ok) break;
+      id = w;
       done = w < 0;
       if (done) break;
     } else {
-      if (n_item > 0) {  // claim the next item
+      // claim the next item (kSplit: every item runs as two ring entries, one per query tile of its pair)
+      if (n_item > 0 && (!kSplit || (n_item & 1) == 0)) {
         int claimed = 0;
         if (elect_one_sync()) claimed = n_workers + (int)atomicAdd(p.sched, 1u);
         w = __shfl_sync(0xffffffffu, claimed, __ffs(__ballot_sync(0xffffffffu, claimed != 0)) - 1);
@@ -385,8 +437,8 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
         }
         if (!ok) break;
       }
+      id = done ? -1 : (kSplit ? 2 * w + (n_item & 1) : w);
       if (elect_one_sync()) {
-        const int id = done ? -1 : w;
         ir.ids[n_item % kItemRing] = id;
         smem_counter_add_release(ir.pub, 1u);
         if constexpr (kPair) {
@@ -397,8 +449,8 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
       __syncwarp();
       if (done) break;
     }
-    const Item it = decode_item<kPair>(p, w);
-    if (!it.id_ok && elect_one_sync()) atomicOr(p.err, ERR_BAD_ITEM);
+    const Item it = decode_item<kPair, kSplit>(p, id);
+    if (!it.id_ok && elect_one_sync() && (!kSplit || it.sub == 0)) atomicOr(p.err, ERR_BAD_ITEM);
     if (n_item > 0) {
       ok = warp_mbar_wait(bars.q_empty, q_empty_ph, tmo, ERR_TIMEOUT_Q_EMPTY, abort_flag, p.err);
       q_empty_ph ^= 1;
@@ -406,9 +458,9 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
     }
     if (elect_one_sync()) {
       const int y0 = it.shard * p.shard_rows;  // the item's shard starts at this global row
-      if (rk == 0) mbar_arrive_expect_tx(bars.q_full, (kPair ? 4 : 2) * C::kTileBytes);
+      if (rk == 0) mbar_arrive_expect_tx(bars.q_full, (kPair ? 4 : C::kQTiles) * C::kTileBytes);
 #pragma unroll
-      for (int t = 0; t < 2; ++t)
+      for (int t = 0; t < C::kQTiles; ++t)
 #pragma unroll
         for (int c = 0; c < C::kSub; ++c) {
           const uint32_t dst = sbase + C::kQOff + t * C::kTileBytes + c * 16384;
@@ -421,7 +473,7 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
     __syncwarp();
     last_q_item = n_item;
     StepIter st;
-    st.init(p, it);
+    st.init(p, it, kSplit);
     int kv_start;
     bool k0, k1;
     while (ok && st.next(kv_start, k0, k1)) {
@@ -483,16 +535,16 @@ __device__ void run_producer(const AttnParams& p, const TMaps& tm, uint8_t* smem
 // core interleaves the two lanes.  Shared K/V slots and the Q buffer are released when both lanes are
 // done with them (the "empty" barriers count two arrivals; a lane that skips a tile arrives directly).
 // ------------------------------------------------------------------------------------------------
-template <int D, bool kPair>
+template <int D, bool kPair, bool kSplit>
 __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, const ItemRing& ir, uint32_t tmem_in,
                         int t, volatile int* abort_flag) {
-  using C = Cfg<D, kPair>;
+  using C = Cfg<D, kPair, kSplit>;
   const uint32_t sbase = smem_u32(smem);
   const uint64_t tmo = p.timeout_ns;
   const uint32_t tmem = __shfl_sync(0xffffffffu, tmem_in, 0);  // provably warp-uniform
   // Descriptors of K-step 0; later K-steps add their byte offset / 16 to the start-address field.  For a
   // pair the same shared-memory offsets name both CTAs' halves of each operand.
-  const uint64_t q_desc = smem_desc_sw128(sbase + C::kQOff + t * C::kTileBytes, 16, 1024);
+  const uint64_t q_desc = smem_desc_sw128(sbase + C::kQOff + (kSplit ? 0 : t) * C::kTileBytes, 16, 1024);
   const uint64_t kv_desc0 = smem_desc_sw128(sbase + C::kKVOff, 16, 1024);
   const uint64_t v_desc0 = smem_desc_sw128(sbase + C::kKVOff, 16384, 1024);
   const uint32_t s_tmem = tmem + C::kColS + t * 128;  // S_t, and P_t over its first 64 columns
@@ -514,7 +566,7 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
   for (;; ++n_item) {
     ok = ring_read(ir, n_item, w, tmo, abort_flag, p.err);
     if (!ok || w < 0) break;
-    const Item it = decode_item<kPair>(p, w);
+    const Item it = decode_item<kPair, kSplit>(p, w);
     ok = warp_mbar_wait(bars.q_full, q_full_ph, tmo, ERR_TIMEOUT_Q_FULL, abort_flag, p.err);
     q_full_ph ^= 1;
     if (!ok) break;
@@ -524,97 +576,117 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
     bool need_odone = n_item > 0;
     bool first_pv = true;
     StepIter st;
-    st.init(p, it);
-    bool prev_has = false, prev_keep = false;
-    int prev_v_pos = 0;
+    st.init(p, it, kSplit);
+    // A kept step's O_t += P_t V_j is issued lazily, just before this lane's next S MMA (which overwrites
+    // P_t: tcgen05 MMAs from one thread execute in issue order, so no wait is needed) or after the item's
+    // last step.  Steps this lane does not keep release their K and V slots at once, without waiting for
+    // this lane's softmax, so that the other lane (and the producer) can run ahead.
+    bool pend = false;  // a P V not yet issued
+    int pend_v_pos = 0;
+    auto issue_pv = [&]() -> bool {
+      const int vs = pend_v_pos % C::kStages;
+      bool good = warp_mbar_wait(bars.kv_full(vs), (pend_v_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
+                                 abort_flag, p.err);
+      if (good && need_odone) {
+        const uint32_t target = C::kODoneWarps * (uint32_t)n_item;
+        good = kPair ? warp_counter_wait_cluster(bars.o_done(t), target, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err)
+                     : warp_counter_wait(bars.o_done(t), target, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err);
+        need_odone = false;
+      }
+      if (good) {
+        good = warp_mbar_wait(p_full, p_full_ph, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
+        p_full_ph ^= 1;
+      }
+      if (!good) return false;
+      tc_fence_after();
+      const uint64_t v_desc = v_desc0 + (uint64_t)((vs * C::kKVBytes) >> 4);
+      const uint32_t acc0 = first_pv ? 0u : 1u;
+      if (elect_one_sync()) {
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          if constexpr (kPair)
+            mma_ts_pair(o_tmem, s_tmem + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
+          else
+            mma_ts(o_tmem, s_tmem + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
+        }
+        commit(pv_done);
+        commit(bars.kv_empty(vs));
+      }
+      __syncwarp();
+      first_pv = false;
+      return true;
+    };
     for (;;) {
       int kv_start;
       bool k0, k1;
-      const bool has = st.next(kv_start, k0, k1);
-      const bool keep = has && (t ? k1 : k0);
+      if (!st.next(kv_start, k0, k1)) break;
+      const bool keep = t ? k1 : k0;
       const int k_pos = ring;
-      // O_t += P_t V_{j-1} for the previous step (or release V_{j-1} if this lane did not use it).
-      if (prev_has) {
-        const int vs = prev_v_pos % C::kStages;
-        if (prev_keep) {
-          ok = warp_mbar_wait(bars.kv_full(vs), (prev_v_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
-                              abort_flag, p.err);
-          if (ok && need_odone) {
-            const uint32_t target = C::kRowWarps * (uint32_t)n_item;
-            ok = kPair ? warp_counter_wait_cluster(bars.o_done(t), target, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err)
-                       : warp_counter_wait(bars.o_done(t), target, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err);
-            need_odone = false;
-          }
-          if (ok) {
-            ok = warp_mbar_wait(p_full, p_full_ph, tmo, ERR_TIMEOUT_P_FULL, abort_flag, p.err);
-            p_full_ph ^= 1;
-          }
+      const int ks = k_pos % C::kStages;
+      ring += 2;
+      if (!keep) {
+        // A pending P V still holds its V slot: issue it before waiting on a position that reuses that slot
+        // (its next load needs the slot released), so that the walk can never wait on itself.  Its P needs
+        // only this lane's softmax, which depends on nothing of the walk.
+        if (pend && k_pos + 1 >= pend_v_pos + C::kStages) {
+          ok = issue_pv();
+          pend = false;
           if (!ok) break;
-          tc_fence_after();
-          const uint64_t v_desc = v_desc0 + (uint64_t)((vs * C::kKVBytes) >> 4);
-          const uint32_t acc0 = first_pv ? 0u : 1u;
-          if (elect_one_sync()) {
-#pragma unroll
-            for (int kk = 0; kk < kTile / 16; ++kk) {
-              if constexpr (kPair)
-                mma_ts_pair(o_tmem, s_tmem + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
-              else
-                mma_ts(o_tmem, s_tmem + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
-            }
-            commit(pv_done);
-            commit(bars.kv_empty(vs));
-          }
+        }
+        // Not used by this lane: still wait for both loads, so that this warp consumes every phase of every
+        // slot (a skipped phase would let a later parity wait see a stale one), and release them.
+        ok = warp_mbar_wait(bars.kv_full(ks), (k_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+        if (ok) {
+          if (elect_one_sync()) release(bars.kv_empty(ks));
           __syncwarp();
-          first_pv = false;
-        } else {
-          // Not used by this lane: still wait for its load, so that this warp consumes every phase
-          // of every slot in order (a skipped phase would let a later parity wait see a stale one).
-          ok = warp_mbar_wait(bars.kv_full(vs), (prev_v_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
-                              abort_flag, p.err);
-          if (!ok) break;
-          if (elect_one_sync()) release(bars.kv_empty(vs));
+          const int vs = (k_pos + 1) % C::kStages;
+          ok = warp_mbar_wait(bars.kv_full(vs), ((k_pos + 1) / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag,
+                              p.err);
+          if (ok && elect_one_sync()) release(bars.kv_empty(vs));
           __syncwarp();
         }
+        if (!ok) break;
+        continue;
       }
-      if (!has) break;
+      if (pend) {  // O_t += P_t V of this lane's previous step
+        ok = issue_pv();
+        pend = false;
+        if (!ok) break;
+      }
       // S_t = Q_t K_j^T.  It overwrites P_t, which the P V just issued reads: tcgen05.mma operations
       // issued by one thread execute in issue order, so no wait is needed here, and the commit below
       // (which fires once all earlier MMAs of this thread are complete) also tells the softmax that
       // O_t is no longer being written.
-      const int ks = k_pos % C::kStages;
-      if (keep) {
-        ok = warp_mbar_wait(bars.kv_full(ks), (k_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
-        if (!ok) break;
-        tc_fence_after();
-        const uint64_t k_desc = kv_desc0 + (uint64_t)((ks * C::kKVBytes) >> 4);
-        if (elect_one_sync()) {
+      ok = warp_mbar_wait(bars.kv_full(ks), (k_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
+      if (!ok) break;
+      tc_fence_after();
+      const uint64_t k_desc = kv_desc0 + (uint64_t)((ks * C::kKVBytes) >> 4);
+      if (elect_one_sync()) {
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t qo = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
-            const uint64_t ko = (uint64_t)(((kk / 4) * C::kKSubBytes + (kk % 4) * 32) >> 4);
-            if constexpr (kPair)
-              mma_ss_pair(s_tmem, q_desc + qo, k_desc + ko, C::kIdescS, kk > 0 ? 1u : 0u);
-            else
-              mma_ss(s_tmem, q_desc + qo, k_desc + ko, C::kIdescS, kk > 0 ? 1u : 0u);
-          }
-          commit(s_full);
-          commit(bars.kv_empty(ks));
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint64_t qo = (uint64_t)(((kk / 4) * 16384 + (kk % 4) * 32) >> 4);
+          const uint64_t ko = (uint64_t)(((kk / 4) * C::kKSubBytes + (kk % 4) * 32) >> 4);
+          if constexpr (kPair)
+            mma_ss_pair(s_tmem, q_desc + qo, k_desc + ko, C::kIdescS, kk > 0 ? 1u : 0u);
+          else
+            mma_ss(s_tmem, q_desc + qo, k_desc + ko, C::kIdescS, kk > 0 ? 1u : 0u);
         }
-        __syncwarp();
-      } else {
-        ok = warp_mbar_wait(bars.kv_full(ks), (k_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL, abort_flag, p.err);
-        if (!ok) break;
-        if (elect_one_sync()) release(bars.kv_empty(ks));
-        __syncwarp();
+        commit(s_full);
+        commit(bars.kv_empty(ks));
       }
-      ring += 2;
-      prev_has = true;
-      prev_keep = keep;
-      prev_v_pos = k_pos + 1;
+      __syncwarp();
+      pend = true;
+      pend_v_pos = k_pos + 1;
     }
     if (!ok) break;
-    if (elect_one_sync()) commit(bars.q_empty);  // this lane's S MMAs of the item are all issued
+    // This lane's S MMAs of the item are all issued: Q is free once they complete (the producer loads the
+    // next item's Q while the last softmax runs).
+    if (elect_one_sync()) commit(bars.q_empty);
     __syncwarp();
+    if (pend) {
+      ok = issue_pv();
+      if (!ok) break;
+    }
   }
   // Drain: nothing of ours may still run on the tensor cores when TMEM is released.
   if (elect_one_sync()) commit(bars.drain);
@@ -636,12 +708,12 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
 // buffers (issued before the last P V is awaited, so they overlap it), the merge in shared memory, TMA
 // stores from the same buffers.  Returns false when a wait gave up (the error is recorded).
 // ------------------------------------------------------------------------------------------------
-template <int D, bool kPair>
+template <int D, bool kPair, bool kSplit>
 __device__ __forceinline__ bool merge_epilogue(const AttnParams& p, const TMaps& tm, uint32_t sbase, const Bars& bars,
                                                uint32_t tO, const Item& it, int q_row, int row, int warp, int lane,
                                                int lane_t, bool row_ok, float l, float m_used, uint32_t total_pv,
                                                uint32_t& stg_ph, volatile int* abort_flag) {
-  using C = Cfg<D, kPair>;
+  using C = Cfg<D, kPair, kSplit>;
   constexpr int kBoxes = D / 32;  // fp32 boxes of 32 columns per row
   constexpr int kFirst = C::kStgBufs < kBoxes ? C::kStgBufs : kBoxes;
   const uint64_t tmo = p.timeout_ns;
@@ -734,12 +806,133 @@ __device__ __forceinline__ bool merge_epilogue(const AttnParams& p, const TMaps&
 }
 
 // ------------------------------------------------------------------------------------------------
+// Epilogue of a split-keys item: the two lanes hold one query tile's O_0, O_1 (TMEM), row maxima m_0, m_1
+// and sums l_0, l_1 over disjoint halves of its key tiles.  The row's result is their log-sum-exp merge
+//   M = max(m_0, m_1),  w_t = 2^(m_t - M),  L = l_0 w_0 + l_1 w_1,  O = (O_0 w_0 + O_1 w_1) / L,
+//   lse = (M + log2 L) ln 2
+// (the same rule as the KV-block re-merge).  The two warps of a TMEM lane quadrant (one per lane) hand
+// (m_1, l_1) to lane 0 and (w_0 / L, w_1 / L) back through shared memory; then each writes half of the D
+// columns, reading both lanes' O for them.  A lane that took no tile has weight 0 and its (stale) O is
+// never read into the sum.  Returns false when a wait gave up (the error is recorded).
+// ------------------------------------------------------------------------------------------------
+template <int D>
+__device__ __forceinline__ bool split_epilogue(const AttnParams& p, const TMaps& tm, uint32_t sbase, const Bars& bars,
+                                               uint32_t trow, const Item& it, int q_row, int row, int warp, int lane,
+                                               int lane_t, bool row_ok, float l, float m_used, int n_kept,
+                                               uint32_t total_pv, uint32_t n_xch, volatile int* abort_flag) {
+  using C = Cfg<D, false, true>;
+  const uint64_t tmo = p.timeout_ns;
+  const int quad = warp & 3;
+  if (n_kept > 0) {
+    bool ok = mbar_wait(bars.pv_done(lane_t), (total_pv - 1) & 1, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return false;
+  }
+  const bool has = n_kept > 0 && l > 0.f && m_used != -INFINITY;
+  const float m = has ? m_used : -INFINITY;
+  const float s = has ? l : 0.f;
+  const uint32_t slot = sbase + C::kXchOff + (uint32_t)(quad * 32 + lane) * 8u;
+  const uint32_t cnt = sbase + C::kXcntOff + 4u * (uint32_t)quad;
+  float c0, c1, lse2 = -INFINITY;
+  tc_fence_before();  // this lane's O is complete; the other lane's warp reads it after the hand-off
+  if (lane_t == 1) {
+    st_shared_v2f(slot, m, s);
+    __syncwarp();
+    if (lane == 0) smem_counter_add_release(cnt, 1u);
+    bool ok = counter_wait(cnt, 2u * n_xch + 2u, tmo, ERR_TIMEOUT_XCH, abort_flag, p.err);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return false;
+    ld_shared_v2f(slot, c0, c1);
+  } else {
+    bool ok = counter_wait(cnt, 2u * n_xch + 1u, tmo, ERR_TIMEOUT_XCH, abort_flag, p.err);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return false;
+    float m1, s1;
+    ld_shared_v2f(slot, m1, s1);
+    const float mx = fmaxf(m, m1);
+    const float w0 = m == -INFINITY ? 0.f : ex2_approx(m - mx);
+    const float w1 = m1 == -INFINITY ? 0.f : ex2_approx(m1 - mx);
+    const float L = s * w0 + s1 * w1;
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    c0 = w0 * inv;
+    c1 = w1 * inv;
+    if (L > 0.f) lse2 = mx + log2f(L);
+    st_shared_v2f(slot, c0, c1);
+    __syncwarp();
+    if (lane == 0) smem_counter_add_release(cnt, 1u);
+  }
+  tc_fence_after();
+  // Boxes of 128 bytes of each of the warp's 32 rows (64 bf16 or 32 fp32 columns): lane t takes half of them
+  // (with one box per row, lane 0 takes it).
+  const int n_boxes = p.o_f32 ? D / 32 : D / 64;
+  const int b_lo = n_boxes >= 2 ? lane_t * (n_boxes / 2) : 0;
+  const int b_hi = n_boxes >= 2 ? (lane_t + 1) * (n_boxes / 2) : (lane_t == 0 ? 1 : 0);
+  const uint32_t tO0 = trow + C::kColO, tO1 = trow + C::kColO + D;
+  const uint32_t stg0 = sbase + C::kStgOff + (uint32_t)warp * (4096u * C::kStgBufs);
+  const CUtensorMap* omap = &tm.o[0];
+  const int row0 = q_row - row + quad * 32;
+  auto mix = [&](uint32_t a, uint32_t b) {
+    const float x = c0 > 0.f ? __uint_as_float(a) * c0 : 0.f;
+    const float y = c1 > 0.f ? __uint_as_float(b) * c1 : 0.f;
+    return x + y;
+  };
+#pragma unroll 1
+  for (int c = b_lo; c < b_hi; ++c) {
+    uint32_t v[32];
+    if (p.o_f32) {
+      uint32_t a[32], b[32];
+      tmem_ld32(tO0 + c * 32, a);
+      tmem_ld32(tO1 + c * 32, b);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(mix(a[e], b[e]));
+    } else {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        uint32_t a[32], b[32];
+        tmem_ld32(tO0 + c * 64 + h * 32, a);
+        tmem_ld32(tO1 + c * 64 + h * 32, b);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 16; ++e) v[16 * h + e] = pack_bf16x2(mix(a[2 * e], b[2 * e]), mix(a[2 * e + 1], b[2 * e + 1]));
+      }
+    }
+    const int k = c - b_lo;
+    const uint32_t stg = stg0 + 4096u * (uint32_t)(k % C::kStgBufs);
+    if (k >= C::kStgBufs) {  // the store that last used this buffer must have read it
+      if (lane == 0) {
+        if (C::kStgBufs == 2)
+          bulk_wait_read_but1();
+        else
+          bulk_wait_read_all();
+      }
+      __syncwarp();
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      st_shared_v4(stg + (uint32_t)lane * 128u + (uint32_t)(((e ^ (lane & 7)) << 4)), v[4 * e], v[4 * e + 1],
+                   v[4 * e + 2], v[4 * e + 3]);
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_4d(omap, stg, c * (p.o_f32 ? 32 : 64), it.h, row0, it.b);
+      bulk_commit_group();
+    }
+  }
+  if (lane == 0) bulk_wait_read_all();  // the buffers are free for the next item
+  __syncwarp();
+  if (lane_t == 0 && row_ok && p.lse)
+    p.lse[((size_t)it.b * p.H + it.h) * p.S + q_row] = lse2 == -INFINITY ? -INFINITY : lse2 * 0.69314718055994531f;
+  return true;
+}
+
+// ------------------------------------------------------------------------------------------------
 // Softmax + epilogue: 4 warps per lane, one query row per thread.
 // ------------------------------------------------------------------------------------------------
-template <int D, bool kPair>
+template <int D, bool kPair, bool kSplit>
 __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase, const Bars& bars, const ItemRing& ir,
                             uint32_t tmem, int lane_t, volatile int* abort_flag) {
-  using C = Cfg<D, kPair>;
+  using C = Cfg<D, kPair, kSplit>;
   // A pair's rank 1 hands its P and its O read-outs to rank 0's barriers and counters.
   const bool remote = kPair && cluster_rank() != 0;
   const uint32_t p_full_bar = remote ? map_shared(bars.p_full(lane_t), 0) : bars.p_full(lane_t);
@@ -756,6 +949,7 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
   uint32_t s_full_ph = 0;
   uint32_t total_pv = 0;
   uint32_t stg_ph = 0;  // bit b: phase of this warp's staging-buffer-b load barrier (merging epilogues)
+  uint32_t n_xch = 0;   // split keys: epilogue hand-offs this warp has taken part in
   bool ok = true;
 
   for (int n_item = 0;; ++n_item) {
@@ -764,9 +958,9 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
     if (!ok || w < 0) break;
     __syncwarp();
     if (lane == 0) smem_counter_add_release(ir.used0 + 4u * warp, 1u);  // this warp is done with the slot
-    const Item it = decode_item<kPair>(p, w);
+    const Item it = decode_item<kPair, kSplit>(p, w);
     StepIter st;
-    st.init(p, it);
+    st.init(p, it, kSplit);
     const int q_row = (lane_t ? it.q_start[1] : it.q_start[0]) + row;
     const bool lane_valid = lane_t ? it.valid[1] : it.valid[0];
     const int lim_row = p.causal ? min(p.kv_lim, q_row + 1) : p.kv_lim;
@@ -874,8 +1068,15 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
       ++total_pv;
     }
     if (!ok) break;
+    // Overlapped launch: nothing is written (or, merging, read) before the kernel before it has completed.
+    if (p.pdl) pdl_wait();
     // Epilogue: O / l and lse for the rows of this lane.
-    if (lane_valid) {
+    if (kSplit && lane_valid) {
+      ok = split_epilogue<D>(p, tm, sbase, bars, trow, it, q_row, row, warp, lane, lane_t, q_row < it.q_end, l, m_used,
+                             n_kept, total_pv, n_xch, abort_flag);
+      ++n_xch;
+      if (!ok) break;
+    } else if (lane_valid) {
       const bool row_ok = q_row < it.q_end;  // inside S and inside the pair's shard
       void* obase = p.o;
       int orow = q_row, orows = p.S;
@@ -888,7 +1089,7 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
       if (p.o_merge) {
         // Merge into the running result: rows that saw no key of this launch's range keep it unchanged.
         if (n_kept > 0) {
-          ok = merge_epilogue<D, kPair>(p, tm, sbase, bars, tO, it, q_row, row, warp, lane, lane_t, row_ok, l,
+          ok = merge_epilogue<D, kPair, kSplit>(p, tm, sbase, bars, tO, it, q_row, row, warp, lane, lane_t, row_ok, l,
                                         m_used, total_pv, stg_ph, abort_flag);
           if (!ok) break;
         }
@@ -970,16 +1171,17 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
         counter_add_cluster(o_done_ctr, 1u);
       else
         smem_counter_add_release(o_done_ctr, 1u);
+      if (kSplit) smem_counter_add_release(bars.o_done(lane_t ^ 1), 1u);  // it also read the other lane's O
     }
   }
   if (lane == 0) bulk_wait_all();  // every O store of this warp has landed before the CTA exits
   __syncwarp();
 }
 
-template <int D, bool kPair>
+template <int D, bool kPair, bool kSplit>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_kernel(const __grid_constant__ TMaps tm, const __grid_constant__ AttnParams p) {
-  using C = Cfg<D, kPair>;
+  using C = Cfg<D, kPair, kSplit>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t bar0 = smem_u32(smem + C::kBarOff);
@@ -1019,6 +1221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       *reinterpret_cast<volatile uint32_t*>(smem + C::kBarOff + (bars.o_done0 - bar0) + 8 * k) = 0u;
     mbar_init(bars.drain, 2);
     for (int k = 0; k < 16; ++k) mbar_init(bars.stg_full0 + 8u * k, 1);
+    if (kSplit)  // the lanes' epilogue hand-off counters
+      for (int k = 0; k < 4; ++k) *reinterpret_cast<volatile uint32_t*>(smem + C::kXcntOff + 4 * k) = 0u;
     *abort_flag = 0;
     *reinterpret_cast<volatile uint32_t*>(smem + C::kMiscOff + 8) = 0u;  // items published
     for (int k = 0; k < 8; ++k)                                          // items read, per softmax warp
@@ -1050,16 +1254,23 @@ __global__ void __launch_bounds__(kThreads, 1)
   if constexpr (kPair) cluster_sync(); else __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
+  if (p.pdl) {
+    // Set up: the next launch may start on the SMs this grid frees.  A launch whose tile or item list the
+    // kernel before it wrote waits for that kernel here; every launch waits for it before its epilogue
+    // writes (run_softmax), so only Q, K and V are read early: they are the caller's promise.
+    if (threadIdx.x == 0) pdl_launch_dependents();
+    if (p.pdl_wait_start) pdl_wait();
+  }
 
   if (warp < 8) {
     regs_inc<kRegsSoftmax>();
-    run_softmax<D, kPair>(p, tm, smem_u32(smem), bars, ir, tmem, warp >> 2, abort_flag);
+    run_softmax<D, kPair, kSplit>(p, tm, smem_u32(smem), bars, ir, tmem, warp >> 2, abort_flag);
   } else {
     regs_dec<kRegsControl>();
     if (warp == kWarpProducer) {
-      run_producer<D, kPair>(p, tm, smem, bars, ir, abort_flag);
+      run_producer<D, kPair, kSplit>(p, tm, smem, bars, ir, abort_flag);
     } else if ((warp == kWarpMma || warp == kWarpMma + 1) && (!kPair || cluster_rank() == 0)) {
-      run_mma<D, kPair>(p, smem, bars, ir, tmem, warp - kWarpMma, abort_flag);  // a pair's MMAs: rank 0
+      run_mma<D, kPair, kSplit>(p, smem, bars, ir, tmem, warp - kWarpMma, abort_flag);  // a pair's MMAs: rank 0
     }
     __syncwarp();
   }
@@ -1114,41 +1325,62 @@ static bool pair_enabled() {
   return on == 1;
 }
 
-template <int D, bool kPair>
+// Split keys (both lanes on one query tile, alternate kept key tiles) for block-sparse launches that write
+// their result (not merging into a running one); SP_ATTN_SPLIT=0 in the environment walks the union of two
+// query tiles' lists instead.
+static bool split_enabled() {
+  static int on = -1;
+  if (on < 0) {
+    const char* e = std::getenv("SP_ATTN_SPLIT");
+    on = (e && e[0] == '0') ? 0 : 1;
+  }
+  return on == 1;
+}
+
+template <int D, bool kPair, bool kSplit>
 static sp_status launch_kernel(const TMaps& tm, const AttnParams& p, int grid, cudaStream_t stream, int dev) {
-  using C = Cfg<D, kPair>;
+  using C = Cfg<D, kPair, kSplit>;
   static int regs_ok[kMaxDevices] = {};
   static bool attr_set[kMaxDevices] = {};
   // The warpgroups re-divide the registers the CTA was launched with; a kernel built with another
   // per-thread count would make that division wait forever, so it is never launched.
   if (regs_ok[dev] == 0) {
     cudaFuncAttributes fa;
-    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kPair>) != cudaSuccess) return SP_ERR_CUDA;
+    if (cudaFuncGetAttributes(&fa, attn_fwd_kernel<D, kPair, kSplit>) != cudaSuccess) return SP_ERR_CUDA;
     regs_ok[dev] = fa.numRegs == kRegsLaunch ? 1 : -1;
   }
   if (regs_ok[dev] < 0) return SP_ERR_UNSUPPORTED;
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kPair>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+    if (cudaFuncSetAttribute(attn_fwd_kernel<D, kPair, kSplit>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
         cudaSuccess)
       return SP_ERR_CUDA;
     attr_set[dev] = true;
   }
-  if constexpr (kPair) {
+  if (kPair || p.pdl) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid, 1, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = C::kSmemBytes;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    int n = 0;
+    if (kPair) {
+      attr[n].id = cudaLaunchAttributeClusterDimension;
+      attr[n].val.clusterDim.x = 2;
+      attr[n].val.clusterDim.y = 1;
+      attr[n].val.clusterDim.z = 1;
+      ++n;
+    }
+    if (p.pdl) {
+      attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+      attr[n].val.programmaticStreamSerializationAllowed = 1;
+      ++n;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, attn_fwd_kernel<D, kPair>, tm, p) != cudaSuccess) return SP_ERR_CUDA;
+    cfg.numAttrs = n;
+    if (cudaLaunchKernelEx(&cfg, attn_fwd_kernel<D, kPair, kSplit>, tm, p) != cudaSuccess) return SP_ERR_CUDA;
   } else {
-    attn_fwd_kernel<D, kPair><<<grid, kThreads, C::kSmemBytes, stream>>>(tm, p);
+    attn_fwd_kernel<D, kPair, kSplit><<<grid, kThreads, C::kSmemBytes, stream>>>(tm, p);
   }
   return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
 }
@@ -1187,6 +1419,8 @@ sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SP_ERR_CUDA;
   const int sms = num_sms(dev);
+  p.pdl = launch_overlap() ? 1 : 0;
+  p.pdl_wait_start = (p.row_ptr || p.item_list) ? 1 : 0;  // lists built by the kernel just before
   const bool pair = p.D == 128 && !p.row_ptr && !p.item_list && sms >= 2 && pair_enabled();
   TMaps tm{};  // the kernel argument (copied at launch)
   for (int r = 0; r < p.n_shards; ++r)
@@ -1249,11 +1483,15 @@ sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
   if (pair) {
     const long long want = 2LL * p.n_items;
     const int grid = (int)(want < (sms & ~1) ? want : (sms & ~1));
-    return launch_kernel<128, true>(tm, p, grid, stream, dev);
+    return launch_kernel<128, true, false>(tm, p, grid, stream, dev);
   }
   const int grid = p.n_items < sms ? p.n_items : sms;
-  return p.D == 128 ? launch_kernel<128, false>(tm, p, grid, stream, dev)
-                    : launch_kernel<64, false>(tm, p, grid, stream, dev);
+  const bool split = p.row_ptr && !p.o_merge && p.n_shards == 1 && split_enabled();
+  if (split)
+    return p.D == 128 ? launch_kernel<128, false, true>(tm, p, grid, stream, dev)
+                      : launch_kernel<64, false, true>(tm, p, grid, stream, dev);
+  return p.D == 128 ? launch_kernel<128, false, false>(tm, p, grid, stream, dev)
+                    : launch_kernel<64, false, false>(tm, p, grid, stream, dev);
 }
 
 }  // namespace spattn

@@ -6,9 +6,12 @@
 // [r H/P, (r+1) H/P):
 //   seq -> head:  out_r[b, s, h', :] = in_{s / (S/P)}[b, s % (S/P), r H/P + h', :]
 //   head -> seq:  out_r[b, s', h, :] = in_{h / (H/P)}[b, r S/P + s', h % (H/P), :]
-// Both directions move contiguous runs of (H/P) * D elements: one warp copies one run with 16-byte
-// vector loads and stores, up to 4 KB per lane group in flight, so both sides are fully coalesced.
-// Bit-exact.
+// When the P ranks are separate processes, the all-to-all itself is a collective (NCCL) between contiguous
+// per-destination blocks, and each rank's local halves are copies of its own shard:
+//   split heads:  out_r[b, s, h', :] = in[b, s, r H/P + h', :]       (before the exchange)
+//   merge heads:  out[b, s, r H/P + h', :] = in_r[b, s, h', :]       (after the way back)
+// All four move contiguous runs of (H/P) * D elements: one warp copies one run with 16-byte vector loads
+// and stores, up to 4 KB per lane group in flight, so both sides are fully coalesced.  Bit-exact.
 #include <cstdint>
 
 #include "sp_internal.h"
@@ -21,7 +24,9 @@ struct RankPtrs {
   uint8_t* out[SP_MAX_RANKS];
 };
 
-template <bool kSeqToHead>
+enum RelayoutMode { kHeadToSeq = 0, kSeqToHead = 1, kSplitHeads = 2, kMergeHeads = 3 };
+
+template <int kMode>
 __global__ void __launch_bounds__(256) relayout_kernel(const __grid_constant__ RankPtrs rp, int P, int B,
                                                        int S, int H, long long run_bytes) {
   const int Sl = S / P;
@@ -32,7 +37,19 @@ __global__ void __launch_bounds__(256) relayout_kernel(const __grid_constant__ R
   for (long long run = (blockIdx.x * (long long)blockDim.x + threadIdx.x) >> 5; run < n_runs; run += warps) {
     const uint8_t* src;
     uint8_t* dst;
-    if (kSeqToHead) {
+    if (kMode == kSplitHeads) {
+      // run = (r, b, s): destination out_r[b, s, :, :] (S here is the rank's own sequence length)
+      const long long bs = run % ((long long)B * S);
+      const int r = (int)(run / ((long long)B * S));
+      src = rp.in[0] + (bs * P + r) * run_bytes;
+      dst = rp.out[r] + bs * run_bytes;
+    } else if (kMode == kMergeHeads) {
+      // run = (b, s, r): destination out[b, s, r H/P : (r+1) H/P, :], contiguous in r
+      const int r = (int)(run % P);
+      const long long bs = run / P;
+      src = rp.in[r] + bs * run_bytes;
+      dst = rp.out[0] + (bs * P + r) * run_bytes;
+    } else if (kMode == kSeqToHead) {
       // run = (r, b, s): destination out_r[b, s, :, :], contiguous in s
       const int s = (int)(run % S);
       const long long rb = run / S;
@@ -76,13 +93,8 @@ __global__ void __launch_bounds__(256) relayout_kernel(const __grid_constant__ R
 
 }  // namespace
 
-sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,
-                          int H, int D, int elem_bytes, bool seq_to_head, cudaStream_t stream) {
-  RankPtrs rp = {};
-  for (int r = 0; r < P; ++r) {
-    rp.in[r] = static_cast<const uint8_t*>(in_ranks[r]);
-    rp.out[r] = static_cast<uint8_t*>(out_ranks[r]);
-  }
+static sp_status launch_runs(const RankPtrs& rp, int mode, int P, int B, int S, int H, int D, int elem_bytes,
+                             cudaStream_t stream) {
   // A run is the H/P heads of one (rank, b, s): H/P * D elements.  In the seq-sharded layout a row of
   // H heads holds P consecutive runs, which is what the kernel's "* P + r" indexing uses.
   const long long run_bytes = (long long)(H / P) * D * elem_bytes;
@@ -93,11 +105,32 @@ sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, i
   long long blocks = (n_runs + 7) / 8;
   const long long cap = (long long)num_sms(dev) * 8;
   if (blocks > cap) blocks = cap;
-  if (seq_to_head)
-    relayout_kernel<true><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes);
-  else
-    relayout_kernel<false><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes);
+  switch (mode) {
+    case kSeqToHead: relayout_kernel<kSeqToHead><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes); break;
+    case kHeadToSeq: relayout_kernel<kHeadToSeq><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes); break;
+    case kSplitHeads: relayout_kernel<kSplitHeads><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes); break;
+    default: relayout_kernel<kMergeHeads><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes); break;
+  }
   return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+}
+
+sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,
+                          int H, int D, int elem_bytes, bool seq_to_head, cudaStream_t stream) {
+  RankPtrs rp = {};
+  for (int r = 0; r < P; ++r) {
+    rp.in[r] = static_cast<const uint8_t*>(in_ranks[r]);
+    rp.out[r] = static_cast<uint8_t*>(out_ranks[r]);
+  }
+  return launch_runs(rp, seq_to_head ? kSeqToHead : kHeadToSeq, P, B, S, H, D, elem_bytes, stream);
+}
+
+sp_status launch_head_groups(const void* const* in, void* const* out, bool split, int P, int B, int S, int H, int D,
+                             int elem_bytes, cudaStream_t stream) {
+  RankPtrs rp = {};
+  const int n_in = split ? 1 : P, n_out = split ? P : 1;
+  for (int r = 0; r < n_in; ++r) rp.in[r] = static_cast<const uint8_t*>(in[r]);
+  for (int r = 0; r < n_out; ++r) rp.out[r] = static_cast<uint8_t*>(out[r]);
+  return launch_runs(rp, split ? kSplitHeads : kMergeHeads, P, B, S, H, D, elem_bytes, stream);
 }
 
 }  // namespace spattn

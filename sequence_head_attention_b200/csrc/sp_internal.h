@@ -31,6 +31,9 @@ struct AttnParams {
   float* lse;       // [B, H, S] or nullptr
   int o_merge;      // 1: o (fp32) and lse hold a running result that this launch's rows are merged into in
                     // place (log-sum-exp rule); rows that see no key of the range are left untouched
+  int pdl;          // 1: launched to overlap the kernel before it on the stream (programmatic dependent
+                    // launch); reads of what that kernel writes wait for it (pdl_wait below)
+  int pdl_wait_start;  // 1: wait for the previous kernel before reading anything (its output is an input here)
   const int* item_list; // device list of work-item ids (nullptr: items 0 .. n_items-1); ids index the
                         // one-chunk layout (b * H + h) * n_qpairs + qp, and ids outside it are skipped
   int item_space;       // number of valid ids (B * H * n_qpairs) when item_list is set
@@ -85,6 +88,7 @@ bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, i
 // (64 bf16 or 32 fp32 values) by 32 positions, 128-byte swizzle.
 bool encode_o_tmap(CUtensorMap* map, void* base, int B, int S, int H, int D, bool f32);
 unsigned long long wait_timeout_ns();
+bool launch_overlap();  // sp_set_launch_overlap
 unsigned int* device_error_word();  // address of the current device's error word, or nullptr
 
 // Launchers (host validation is done by the C entry points before these are called).
@@ -100,6 +104,10 @@ sp_status launch_merge(const float* const* o_parts, const float* const* lse_part
                        float* lse, int o_f32, int B, int S, int H, int D, cudaStream_t stream);
 sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,
                           int H, int D, int elem_bytes, bool seq_to_head, cudaStream_t stream);
+// The local halves of a multi-process Ulysses exchange: split (in[0] -> out[0..P-1]) or merge
+// (in[0..P-1] -> out[0]) of the P head groups of a [B, S, H, D] sequence shard.
+sp_status launch_head_groups(const void* const* in, void* const* out, bool split, int P, int B, int S, int H, int D,
+                             int elem_bytes, cudaStream_t stream);
 sp_status launch_tile_list(const uint8_t* mask, int H, int T, int32_t* row_ptr, int32_t* col_idx,
                            int32_t* counts, cudaStream_t stream);
 sp_status launch_debug_wait(unsigned long long timeout_ns, cudaStream_t stream);

@@ -25,7 +25,8 @@ enum : unsigned int {
   ERR_TIMEOUT_STG = 1u << 10,        // a merging epilogue's load of the running O
   ERR_TIMEOUT_ITEM = 1u << 11,       // waiting for the next work-item id
   ERR_TIMEOUT_ITEM_FREE = 1u << 12,  // waiting for a work-item slot to be read by every role
-  ERR_ANY_TIMEOUT = 0x1fffu,
+  ERR_TIMEOUT_XCH = 1u << 13,        // split keys: waiting for the other lane's row maximum and sum
+  ERR_ANY_TIMEOUT = 0x3fffu,
   ERR_BAD_ITEM = 1u << 16,           // an item list named a work item that does not exist (skipped)
 };
 
@@ -167,6 +168,12 @@ __device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t src, int
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w) : "memory");
 }
+__device__ __forceinline__ void st_shared_v2f(uint32_t addr, float x, float y) {
+  asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
+}
+__device__ __forceinline__ void ld_shared_v2f(uint32_t addr, float& x, float& y) {
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(x), "=f"(y) : "r"(addr) : "memory");
+}
 __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& x, uint32_t& y, uint32_t& z, uint32_t& w) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(x), "=r"(y), "=r"(z), "=r"(w) : "r"(addr) : "memory");
 }
@@ -177,6 +184,12 @@ __device__ __forceinline__ void bulk_wait_read_but1() {  // all but the newest g
   asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
 }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Programmatic dependent launch: let the next kernel on the stream (launched with programmatic stream
+// serialisation) start on SMs this grid frees; and wait until every kernel this grid depends on has
+// completed and its memory is visible (returns at once when none is in flight).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");

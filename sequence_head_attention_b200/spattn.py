@@ -54,6 +54,8 @@ def lib() -> ctypes.CDLL:
                 "sp_seq_to_head_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_head_to_seq_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_attn_fwd_seq_sharded": (I, [P, P, P, P, P, I, I, I, I, I, I, I, P, I, I, P]),
+                "sp_split_heads": (I, [P, P, I, I, I, I, I, I, P]),
+                "sp_merge_heads": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_attn_fwd_items": (I, [P, P, P, P, P, I, I, I, I, P, I, I, P, P, Z, P]),
                 "sp_attn_bwd_workspace_bytes": (Z, [I, I, I, I]),
                 "sp_attn_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, P, Z, P]),
@@ -68,6 +70,7 @@ def lib() -> ctypes.CDLL:
                 "sp_check_device_error": (I, [P]),
                 "sp_check_device_error_bits": (I, [P, P]),
                 "sp_set_wait_timeout_ns": (None, [U64]),
+                "sp_set_launch_overlap": (None, [I]),
                 "sp_debug_wait_timeout": (I, [U64, P]),
                 "sp_debug_exp2_poly": (I, [P, P, I, P]),
                 "sp_version": (ctypes.c_char_p, []),
@@ -278,6 +281,32 @@ def sp_head_to_seq_relayout(in_ranks, out_ranks, S=None, H=None, stream=None):
     return out_ranks
 
 
+def sp_split_heads(x, out_ranks, stream=None):
+    """x [B, S, H, D] (this rank's sequence shard) -> P head groups out_ranks[r] [B, S, H/P, D] (bit-exact)."""
+    P = len(out_ranks)
+    B, S, H, D = x.shape
+    _need(x.is_cuda and x.is_contiguous(), "x must be a contiguous CUDA tensor")
+    for t in out_ranks:
+        _need(t.is_cuda and t.is_contiguous() and t.dtype == x.dtype and tuple(t.shape) == (B, S, H // P, D)
+              and t.device == x.device, "out_ranks must be contiguous [B, S, H/P, D] of x's dtype and device")
+    op, _k = _ptr_array(out_ranks)
+    _check("sp_split_heads", lib().sp_split_heads(_ptr(x), op, P, B, S, H, D, x.element_size(), _stream(stream)))
+    return out_ranks
+
+
+def sp_merge_heads(in_ranks, out, stream=None):
+    """P head groups in_ranks[r] [B, S, H/P, D] -> out [B, S, H, D] (bit-exact)."""
+    P = len(in_ranks)
+    B, S, H, D = out.shape
+    _need(out.is_cuda and out.is_contiguous(), "out must be a contiguous CUDA tensor")
+    for t in in_ranks:
+        _need(t.is_cuda and t.is_contiguous() and t.dtype == out.dtype and tuple(t.shape) == (B, S, H // P, D)
+              and t.device == out.device, "in_ranks must be contiguous [B, S, H/P, D] of out's dtype and device")
+    ip, _k = _ptr_array(in_ranks)
+    _check("sp_merge_heads", lib().sp_merge_heads(ip, _ptr(out), P, B, S, H, D, out.element_size(), _stream(stream)))
+    return out
+
+
 def sp_attn_fwd_seq_sharded(q_shards, k_shards, v_shards, o_shards, lse=None, heads=None, head_chunks=None,
                             causal=False, stream=None):
     """One Ulysses rank's attention on the sequence shards (bf16 [B, S/P, H, D] each, P of them):
@@ -472,6 +501,12 @@ def sp_check_device_error_bits(stream=None):
 
 def sp_set_wait_timeout_ns(ns: int) -> None:
     lib().sp_set_wait_timeout_ns(int(ns))
+
+
+def sp_set_launch_overlap(enable: bool) -> None:
+    """Let each attention launch start while the kernel before it on the stream finishes (see the header
+    for what the caller promises)."""
+    lib().sp_set_launch_overlap(int(bool(enable)))
 
 
 def sp_debug_wait_timeout(timeout_ns: int, stream=None) -> None:

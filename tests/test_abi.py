@@ -137,3 +137,19 @@ def test_partial_merge_rejects_on_host(L):
     assert f(q, q, q, o, o + 64, 1, 256, 4, 64, 0, 256, 0, None, None, 0, None) == spattn.SP_ERR_INVALID_ARG
     assert f(q, q, q, o, l, 1, 256, 4, 96, 0, 256, 0, None, None, 0, None) == spattn.SP_ERR_INVALID_ARG
     assert f(q, q, q, o, l, 1, 256, 4, 64, 128, 128, 0, None, None, 0, None) == spattn.SP_OK  # empty: no launch
+
+
+def test_split_and_merge_heads_reject_on_host(L):
+    outs = (ctypes.c_void_p * 4)(1 << 24, 2 << 24, 3 << 24, 4 << 24)
+    o = ctypes.cast(outs, ctypes.c_void_p)
+    x = 5 << 24
+    f, g = L.sp_split_heads, L.sp_merge_heads
+    assert f(x, o, 4, 1, 16, 6, 64, 2, None) == spattn.SP_ERR_INVALID_ARG     # H % P
+    assert f(x, o, 4, 1, 16, 8, 4, 2, None) == spattn.SP_ERR_INVALID_ARG     # D * elem not a multiple of 16
+    assert f(x, o, 4, 1, 16, 8, 64, 3, None) == spattn.SP_ERR_INVALID_ARG    # elem_bytes
+    assert f(x + 8, o, 4, 1, 16, 8, 64, 2, None) == spattn.SP_ERR_INVALID_ARG  # misaligned
+    assert f(1 << 24, o, 4, 1, 16, 8, 64, 2, None) == spattn.SP_ERR_INVALID_ARG  # input overlaps output 0
+    same = (ctypes.c_void_p * 4)(1 << 24, 1 << 24, 3 << 24, 4 << 24)
+    assert f(x, ctypes.cast(same, ctypes.c_void_p), 4, 1, 16, 8, 64, 2, None) == spattn.SP_ERR_INVALID_ARG
+    assert g(o, x, 0, 1, 16, 8, 64, 2, None) == spattn.SP_ERR_INVALID_ARG     # P
+    assert g(o, 2 << 24, 4, 1, 16, 8, 64, 2, None) == spattn.SP_ERR_INVALID_ARG  # output overlaps input 1

@@ -66,3 +66,31 @@ def test_relayout_leaves_bytes_outside_outputs_untouched():
     spattn.sp_seq_to_head_relayout(ins, outs)
     for buf in bufs:
         assert torch.all(buf[:guard] == 12345) and torch.all(buf[-guard:] == 12345)
+
+
+@pytest.mark.parametrize("P,B,S,H,D,dtype", [
+    (4, 1, 8190, 40, 128, torch.bfloat16),    # one video-DiT rank's sequence shard, 4 ranks
+    (8, 2, 300, 8, 64, torch.bfloat16),
+    (2, 1, 7, 6, 8, torch.float32),
+    (1, 1, 100, 4, 64, torch.bfloat16),       # P = 1: a copy
+    (3, 2, 5, 9, 2, torch.float64),
+])
+def test_split_and_merge_heads_bit_exact(P, B, S, H, D, dtype):
+    """The local halves of a multi-process exchange: every head group equals the oracle's, bytes exact,
+    and merging them back gives the shard; nothing outside the outputs is written."""
+    g = torch.Generator().manual_seed(P * 100 + S)
+    x = torch.randn((B, S, H, D), generator=g, dtype=torch.float32).to(dtype)
+    ref = oracle.split_heads(_bits(x), P)
+    xd = x.cuda()
+    guard = 1 << 12
+    outs_buf = [torch.full((B * S * (H // P) * D + 2 * guard,), 7, dtype=dtype, device="cuda") for _ in range(P)]
+    outs = [b[guard:-guard].view(B, S, H // P, D) for b in outs_buf]
+    spattn.sp_split_heads(xd, outs)
+    back = torch.empty_like(xd)
+    spattn.sp_merge_heads(outs, back)
+    torch.cuda.synchronize()
+    for r in range(P):
+        assert np.array_equal(_bits(outs[r]), ref[r])
+        assert torch.all(outs_buf[r][:guard] == 7) and torch.all(outs_buf[r][-guard:] == 7)
+    assert np.array_equal(_bits(back), oracle.merge_heads(ref))
+    assert np.array_equal(_bits(back), _bits(x))
