@@ -473,9 +473,14 @@ def measure_main(wname, args, peaks, dev, stream, world, seed, headline):
     """Time one full-size workload: W warm-up steps, then K steps between barrier + synchronize, CUDA events
     on the launching stream, max over ranks.  Returns (record, step, inputs)."""
     import torch
+    from sequence_head_attention_b200 import spattn
     w, q, k, v, mask = build_inputs(wname, seed=seed, seq_len=args.seq_len if headline else 0,
                                     ranks=args.ranks if headline else 0)
     fused = wname == "video_dit" and args.ulysses == "fused"
+    # Launch overlap where the step's attention launches follow one another and no kernel writes the Q, K, V
+    # of the launch after it: the per-rank launches on the shards, the ring's blocks, the masked launches.
+    overlap = not args.no_overlap and (fused or wname != "video_dit")
+    spattn.sp_set_launch_overlap(overlap)
     step = make_step(wname, w, q, k, v, mask, dev, fused, with_partials=wname == "ring_causal")
     for _ in range(args.warmup):
         step.run()
@@ -497,7 +502,8 @@ def measure_main(wname, args, peaks, dev, stream, world, seed, headline):
     ms = max_over_ranks(t_start.elapsed_time(t_end), device=dev)
     value = step.flops * args.steps * world / (ms / 1000.0) / 1e12
     rec = {"workload": workload_name(w, wname), "steps": args.steps, "warmup": args.warmup,
-           "ms_per_step": ms / args.steps, "tflops": value, "launches_per_step": step.launches, "clocks": clocks}
+           "ms_per_step": ms / args.steps, "tflops": value, "launches_per_step": step.launches, "clocks": clocks,
+           "launch_overlap": overlap}
     if wname == "video_dit":
         attn_ms = timer.mean_ms("attn")
         rec["attention"] = {"tflops": step.flops / step.P / (attn_ms / 1000.0) / 1e12, "ms_per_launch": attn_ms,
@@ -555,6 +561,7 @@ def latency_report(wname, dev, stream, peaks, reps=200):
     import torch
     from sequence_head_attention_b200 import spattn, synth
     w = synth.WORKLOADS[wname]
+    spattn.sp_set_launch_overlap(False)  # plain calls, each launch after the previous kernel
     q, k, v = (t.to(dev) for t in synth.qkv(w.B, w.S, w.H, w.D, seed=0, scale=w.scale)[:3])
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)
@@ -672,7 +679,8 @@ def run_sp(args):
     qs, ks, vs = (t[:, rank * Sl:(rank + 1) * Sl].contiguous().to(dev) for t in (q, k, v))
     del q, k, v
     if args.sp == "ulysses":
-        sp = sp_dist.UlyssesAttention(w.B, w.S, w.H, w.D, head_chunks=w.head_chunks, causal=w.causal, device=dev)
+        sp = sp_dist.UlyssesAttention(w.B, w.S, w.H, w.D, head_chunks=w.head_chunks, causal=w.causal, device=dev,
+                                      stages=args.sp_stages)
         flops_rank = w.flops() / world  # every rank attends H/P heads over the whole sequence
     else:
         sp = sp_dist.RingAttention(w.B, w.S, w.H, w.D, causal=w.causal, device=dev)
@@ -707,7 +715,8 @@ def run_sp(args):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": dict(config_of(w, wname, 1), parallelism=f"{args.sp}{world}",
-                           global_batch=w.B, sp=f"{args.sp}: each rank holds S/{world} positions of Q, K, V"),
+                           global_batch=w.B, sp=f"{args.sp}: each rank holds S/{world} positions of Q, K, V",
+                           sp_stages=args.sp_stages if args.sp == "ulysses" else None),
             "roofline": roofline, "cpu_baseline": None, "e2e": None,
             "gpu_launches": None, "clocks": clocks, "impl": "ours",
             "kernels": {"rank0": {"attention_ms_per_step": attn_ms, "flops_per_step": flops_rank,
@@ -760,6 +769,7 @@ def run_ours(args):
                  else "seq->head relayout, per-rank attention, head->seq relayout"}
     if head == "block_sparse":
         extra = {"mask_density": step.density, "kept_tiles": step.kept_tiles}
+    extra["launch_overlap"] = rec["launch_overlap"]
     line = {"metric": METRIC, "value": rec["tflops"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -802,6 +812,9 @@ def main(argv=None):
                     help="replicas (default): every rank runs its own batch of every workload (weak scaling); "
                          "ulysses / ring: one global problem sequence-parallel over the ranks with NCCL "
                          "collectives (video_dit all-to-all, ring_causal ring; strong scaling)")
+    ap.add_argument("--sp-stages", type=int, default=2,
+                    help="--sp ulysses: head-chunk stages per rank (HCMS), each stage's all-to-all overlapping "
+                         "the previous stage's attention")
     ap.add_argument("--ulysses", choices=["fused", "relayout"], default="fused",
                     help="video_dit step: attention straight on the sequence shards (fused), or the seq->head "
                          "relayout, per-rank attention and head->seq relayout")
@@ -809,6 +822,8 @@ def main(argv=None):
                     help="block_sparse: also time the work split over this many simulated ranks, head split "
                          "vs db-SP plan (0: off)")
     ap.add_argument("--no-backward", action="store_true", help="video_dit: skip the backward-pass measurement")
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch every attention kernel only after the previous kernel has completed")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

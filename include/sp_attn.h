@@ -222,17 +222,19 @@ SP_API sp_status sp_head_to_seq_relayout(const void* const* in_ranks, void* cons
  * all-to-all based sequence parallelism; "db-SP", abstract: parallelism along the head dimension as in
  * Ulysses).  The exchange itself is a collective between contiguous per-destination blocks (NCCL
  * all-to-all); around it, each rank copies its own sequence shard x [B, S, H, D] (S: the rank's own
- * positions) into P head groups, and back:
- *   sp_split_heads:  out_ranks[r] [B, S, H/P, D] = x[:, :, r*H/P : (r+1)*H/P, :]  (block sent to rank r)
- *   sp_merge_heads:  out[:, :, r*H/P : (r+1)*H/P, :] = in_ranks[r] [B, S, H/P, D]  (block from rank r)
- * Bit-exact byte copies.  Requires 1 <= P <= SP_MAX_RANKS, H % P == 0, elem_bytes in {1, 2, 4, 8},
- * (D * elem_bytes) % 16 == 0, 16-byte aligned buffers, no overlap between any input and any output or
- * between two outputs.  out_ranks / in_ranks are host arrays of P device pointers.
+ * positions) into P head groups, and back.  With g = H/P and heads [h0, h0 + n) of every group (the whole
+ * group, h0 = 0 and n = g, or one stage of an exchange done in head chunks, "HCMS", abstract):
+ *   sp_split_heads:  out_ranks[r] [B, S, n, D] = x[:, :, r*g + h0 : r*g + h0 + n, :]  (block sent to rank r)
+ *   sp_merge_heads:  out[:, :, r*g + h0 : r*g + h0 + n, :] = in_ranks[r] [B, S, n, D] (block from rank r)
+ * Bit-exact byte copies; merge leaves the other heads of out untouched.  Requires 1 <= P <= SP_MAX_RANKS,
+ * H % P == 0, 0 <= h0, n >= 1, h0 + n <= H/P, elem_bytes in {1, 2, 4, 8}, (D * elem_bytes) % 16 == 0,
+ * 16-byte aligned buffers, no overlap between any input and any output or between two outputs.
+ * out_ranks / in_ranks are host arrays of P device pointers.
  */
-SP_API sp_status sp_split_heads(const void* in, void* const* out_ranks, int P, int B, int S, int H, int D,
-                                int elem_bytes, sp_stream stream);
-SP_API sp_status sp_merge_heads(const void* const* in_ranks, void* out, int P, int B, int S, int H, int D,
-                                int elem_bytes, sp_stream stream);
+SP_API sp_status sp_split_heads(const void* in, void* const* out_ranks, int P, int B, int S, int H, int D, int h0,
+                                int n_heads, int elem_bytes, sp_stream stream);
+SP_API sp_status sp_merge_heads(const void* const* in_ranks, void* out, int P, int B, int S, int H, int D, int h0,
+                                int n_heads, int elem_bytes, sp_stream stream);
 
 /*
  * One Ulysses rank's attention straight on the sequence shards, with both relayouts folded into the

@@ -664,12 +664,13 @@ sp_status sp_convert_f32_to_bf16(const float* in, void* out, long long n, sp_str
 }
 
 static sp_status head_groups_common(const void* const* ins, int n_in, void* const* outs, int n_out, bool split, int P,
-                                    int B, int S, int H, int D, int elem_bytes, sp_stream stream) {
+                                    int B, int S, int H, int D, int h0, int n_heads, int elem_bytes, sp_stream stream) {
   if (!ins || !outs || P < 1 || P > SP_MAX_RANKS || B < 1 || S < 0 || H < 1 || D < 1) return SP_ERR_INVALID_ARG;
   if (elem_bytes != 1 && elem_bytes != 2 && elem_bytes != 4 && elem_bytes != 8) return SP_ERR_INVALID_ARG;
   if (H % P != 0 || ((long long)D * elem_bytes) % 16 != 0) return SP_ERR_INVALID_ARG;
+  if (h0 < 0 || n_heads < 1 || h0 + n_heads > H / P) return SP_ERR_INVALID_ARG;
   if ((double)B * S * H * D * elem_bytes > 9.0e15) return SP_ERR_INVALID_ARG;
-  const long long whole = (long long)B * S * H * D * elem_bytes, group = whole / P;
+  const long long whole = (long long)B * S * H * D * elem_bytes, group = (long long)B * S * n_heads * D * elem_bytes;
   const long long in_bytes = split ? whole : group, out_bytes = split ? group : whole;
   for (int r = 0; r < n_in; ++r)
     if (!ins[r] || !aligned16(ins[r])) return SP_ERR_INVALID_ARG;
@@ -685,19 +686,19 @@ static sp_status head_groups_common(const void* const* ins, int n_in, void* cons
       const uintptr_t a0 = reinterpret_cast<uintptr_t>(outs[r]), b0 = reinterpret_cast<uintptr_t>(outs[g]);
       if (a0 < b0 + out_bytes && b0 < a0 + out_bytes) return SP_ERR_INVALID_ARG;
     }
-  return launch_head_groups(ins, outs, split, P, B, S, H, D, elem_bytes, as_stream(stream));
+  return launch_head_groups(ins, outs, split, P, B, S, H, D, h0, n_heads, elem_bytes, as_stream(stream));
 }
 
-sp_status sp_split_heads(const void* in, void* const* out_ranks, int P, int B, int S, int H, int D, int elem_bytes,
-                         sp_stream stream) {
+sp_status sp_split_heads(const void* in, void* const* out_ranks, int P, int B, int S, int H, int D, int h0, int n_heads,
+                         int elem_bytes, sp_stream stream) {
   const void* ins[1] = {in};
-  return head_groups_common(ins, 1, out_ranks, P, true, P, B, S, H, D, elem_bytes, stream);
+  return head_groups_common(ins, 1, out_ranks, P, true, P, B, S, H, D, h0, n_heads, elem_bytes, stream);
 }
 
-sp_status sp_merge_heads(const void* const* in_ranks, void* out, int P, int B, int S, int H, int D, int elem_bytes,
-                         sp_stream stream) {
+sp_status sp_merge_heads(const void* const* in_ranks, void* out, int P, int B, int S, int H, int D, int h0,
+                         int n_heads, int elem_bytes, sp_stream stream) {
   void* outs[1] = {out};
-  return head_groups_common(in_ranks, P, outs, 1, false, P, B, S, H, D, elem_bytes, stream);
+  return head_groups_common(in_ranks, P, outs, 1, false, P, B, S, H, D, h0, n_heads, elem_bytes, stream);
 }
 
 sp_status sp_seq_to_head_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,

@@ -23,7 +23,7 @@
 //               when both are in their softmax phase the two warps per SMSP hide each other's latency.
 //   warp 11     idle (it completes the third warpgroup, which gives its registers to the softmax).
 //   TMEM (512 columns): S_0 [0,128), S_1 [128,256), O_0 [256, 256+D), O_1 [256+D, 256+2D); P_t
-//   overwrites the first 64 columns of S_t.  Each lane's issuer queues S_t(j+1) right behind
+//   overwrites the last 64 columns of S_t.  Each lane's issuer queues S_t(j+1) right behind
 //   O_t += P_t(j) V_j: MMAs from one thread execute in issue order, so S_t(j+1) cannot overwrite P_t(j)
 //   before the P V has read it.
 // Every barrier wait is bounded in time; on expiry the kernel records an error and returns cleanly.
@@ -31,6 +31,7 @@
 #include <climits>
 #include <cstdint>
 #include <cstdlib>
+#include <type_traits>
 
 #include "sp_internal.h"
 #include "sp_ptx.cuh"
@@ -60,6 +61,7 @@ constexpr int kSchedSlots = 64;  // launch-rotated work counters
 // device (the C header states this limit).  A launch leaves its pair at zero when its last CTA ends.
 __device__ unsigned int g_attn_sched[2 * kSchedSlots];
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and l are rescaled when m grows by > 2^8
+constexpr uint32_t kPCol = 64;  // P_t (bf16 pairs) lives over the last 64 of S_t's 128 columns
 #ifndef SP_EXP2_POLY_PAIRS
 #define SP_EXP2_POLY_PAIRS 0  // of every 8 pairs of exponentials, this many run on the FMA pipe
 #endif
@@ -547,7 +549,7 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
   const uint64_t q_desc = smem_desc_sw128(sbase + C::kQOff + (kSplit ? 0 : t) * C::kTileBytes, 16, 1024);
   const uint64_t kv_desc0 = smem_desc_sw128(sbase + C::kKVOff, 16, 1024);
   const uint64_t v_desc0 = smem_desc_sw128(sbase + C::kKVOff, 16384, 1024);
-  const uint32_t s_tmem = tmem + C::kColS + t * 128;  // S_t, and P_t over its first 64 columns
+  const uint32_t s_tmem = tmem + C::kColS + t * 128;  // S_t, and P_t over its last 64 columns
   const uint32_t o_tmem = tmem + C::kColO + t * D;
   const uint32_t s_full = bars.s_full(t), p_full = bars.p_full(t), pv_done = bars.pv_done(t);  // pv_done: for the epilogue
   uint32_t q_full_ph = 0, p_full_ph = 0;
@@ -605,9 +607,10 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
 #pragma unroll
         for (int kk = 0; kk < kTile / 16; ++kk) {
           if constexpr (kPair)
-            mma_ts_pair(o_tmem, s_tmem + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
+            mma_ts_pair(o_tmem, s_tmem + kPCol + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV,
+                        kk > 0 ? 1u : acc0);
           else
-            mma_ts(o_tmem, s_tmem + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
+            mma_ts(o_tmem, s_tmem + kPCol + kk * 8, v_desc + (uint64_t)(kk * 128), C::kIdescPV, kk > 0 ? 1u : acc0);
         }
         commit(pv_done);
         commit(bars.kv_empty(vs));
@@ -926,6 +929,22 @@ __device__ __forceinline__ bool split_epilogue(const AttnParams& p, const TMaps&
   return true;
 }
 
+// A thread's O row in TMEM multiplied by alpha (warp-collective: every lane of the warp calls it); it runs
+// only when a row's maximum grows by more than 2^8 (log2 units).  Inlined: out of line, the call measured
+// 10% slower block-sparse launches although it never runs there.
+template <int D>
+__device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
+#pragma unroll 1
+  for (int c = 0; c < D / 16; ++c) {
+    uint32_t o[16];
+    tmem_ld16(tO + c * 16, o);
+    tmem_wait_ld();
+#pragma unroll
+    for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+    tmem_st16(tO + c * 16, o);
+  }
+}
+
 // ------------------------------------------------------------------------------------------------
 // Softmax + epilogue: 4 warps per lane, one query row per thread.
 // ------------------------------------------------------------------------------------------------
@@ -991,69 +1010,110 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
           for (int e = 0; e < 32; ++e)
             if (c * 32 + e >= n_valid) sr[c][e] = __float_as_uint(-INFINITY);
       }
-      // Row maximum: eight independent chains of three-input maxima, then a small tree.
-      float mx8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(SV(2 * k), SV(2 * k + 1));
-#pragma unroll
-      for (int i = 16; i < 128; i += 16)
-#pragma unroll
-        for (int k = 0; k < 8; ++k) mx8[k] = fmax3f(mx8[k], SV(i + 2 * k), SV(i + 2 * k + 1));
-      const float mx = fmax3f(fmax3f(mx8[0], mx8[1], mx8[2]), fmax3f(mx8[3], mx8[4], mx8[5]),
-                              fmaxf(mx8[6], mx8[7]));
-      const float m_tile = mx * scale_log2;
-      const bool grow = m_tile > m_used + kRescaleThreshold;
-      float alpha = 1.f;
-      if (grow) {
-        alpha = ex2_approx(m_used - m_tile);  // 0 when nothing was seen before
-        l *= alpha;
-        m_used = m_tile;
-      }
-      if (n_kept > 0 && __any_sync(0xffffffffu, grow)) {
-        // O row *= alpha.  The previous O += P V of this lane has completed (the S_t commit that
-        // signalled this step fires only after every earlier MMA of its issuer), and the next one
-        // waits for this thread's P.
-#pragma unroll 1
-        for (int c = 0; c < D / 16; ++c) {
-          uint32_t o[16];
-          tmem_ld16(tO + c * 16, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-          tmem_st16(tO + c * 16, o);
-        }
-      }
-      const float neg_m = m_used == -INFINITY ? 0.f : -m_used;
       const f2 sc2 = {scale_log2, scale_log2};
-      const f2 nm2 = {neg_m, neg_m};
-      f2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
-      // P = 2^(s * scale - m), bf16, two per column over the first 64 columns of S_t: the A operand of
-      // O += P V.  Each quarter is stored as soon as it is packed.  Of every 8 pairs, kPolyPairs go
-      // through the FMA-pipe polynomial and the rest through ex2.approx, so neither pipe saturates.
-#pragma unroll
-      for (int quarter = 0; quarter < 4; ++quarter) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const int i = quarter * 32 + e;
-          const f2 x = ffma2(f2{SV(i), SV(i + 1)}, sc2, nm2);
-          f2 pr;
-          if (((e >> 1) & 7) >= 8 - kPolyPairs) {
-            pr = exp2_poly2(x);
-          } else {
-            pr.x = ex2_approx(x.x);
-            pr.y = ex2_approx(x.y);
-          }
-          acc[(e >> 1) & 3] = fadd2(acc[(e >> 1) & 3], pr);
-          pk[e >> 1] = pack_bf16x2(pr.x, pr.y);
+      // 2^(s * scale - m) for the two columns of pair e of the row (of every 8 pairs, kPolyPairs go through
+      // the FMA-pipe polynomial and the rest through ex2.approx).
+      auto exp_pair = [&](int i, int e, f2 nm2) -> f2 {
+        const f2 x = ffma2(f2{SV(i), SV(i + 1)}, sc2, nm2);
+        f2 pr;
+        if (((e >> 1) & 7) >= 8 - kPolyPairs) {
+          pr = exp2_poly2(x);
+        } else {
+          pr.x = ex2_approx(x.x);
+          pr.y = ex2_approx(x.y);
         }
-        tmem_st16(tS + quarter * 16, pk);
+        return pr;
+      };
+      // P = 2^(s * scale - m), bf16, two per column over the last 64 columns of S_t (the A operand of
+      // O += P V), each quarter stored as soon as it is packed; returns the row sum.  With the maximum
+      // (mx4 given), the row's maximum is formed in the same pass: four chains of three-input maxima on
+      // the ALU pipe, beside the FMA and MUFU work.  P over the last 64 columns leaves S's first 64 columns
+      // in TMEM, and the pass reads the last 64 from registers last, so a pass can be redone.
+      float mx4[4];
+      auto exp_pass = [&](float neg_m, auto with_max) -> float {
+        const f2 nm2 = {neg_m, neg_m};
+        f2 acc[4] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+        for (int quarter = 0; quarter < 4; ++quarter) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const int i = quarter * 32 + e;
+            if constexpr (decltype(with_max)::value) {
+              const int k = (e >> 1) & 3;
+              mx4[k] = (quarter == 0 && e < 8) ? fmaxf(SV(i), SV(i + 1)) : fmax3f(mx4[k], SV(i), SV(i + 1));
+            }
+            const f2 pr = exp_pair(i, e, nm2);
+            acc[(e >> 1) & 3] = fadd2(acc[(e >> 1) & 3], pr);
+            pk[e >> 1] = pack_bf16x2(pr.x, pr.y);
+          }
+          tmem_st16(tS + kPCol + quarter * 16, pk);
+        }
+        const f2 acc4 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+        return acc4.x + acc4.y;
+      };
+      float rowsum;
+      if (kSplit || n_kept == 0) {
+        // The row maximum first, then the exponentials against it: the item's first step for this lane,
+        // and every step of split-key items (each lane has half the steps, and measured, the speculative
+        // pass below costs them more than the maximum's latency).
+        float mx8[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) mx8[k] = fmaxf(SV(2 * k), SV(2 * k + 1));
+#pragma unroll
+        for (int i = 16; i < 128; i += 16)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) mx8[k] = fmax3f(mx8[k], SV(i + 2 * k), SV(i + 2 * k + 1));
+        const float m_tile =
+            fmax3f(fmax3f(mx8[0], mx8[1], mx8[2]), fmax3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])) * scale_log2;
+        const bool grow = m_tile > m_used + kRescaleThreshold;
+        float alpha = 1.f;
+        if (grow) {
+          alpha = ex2_approx(m_used - m_tile);  // 0 when nothing was seen before
+          l *= alpha;
+          m_used = m_tile;
+        }
+        rowsum = exp_pass(m_used == -INFINITY ? 0.f : -m_used, std::false_type{});
+        // O row *= alpha, after the pass (the S registers are free by then): the previous O += P V of
+        // this lane has completed (the S_t commit that signalled this step fires only after every earlier
+        // MMA of its issuer), and the next one waits for this thread's P, which is announced only after
+        // these stores have completed.
+        if (n_kept > 0 && __any_sync(0xffffffffu, grow)) rescale_o_row<D>(tO, alpha);
+      } else {
+        // Later steps: the exponentials run against the running maximum while this tile's maximum is
+        // formed in the same pass, so they need not wait for it.  Where it grew by more than 2^8 (log2
+        // units) the pass was against too small a reference: that row's sum and O are rescaled and the warp
+        // redoes the pass against the new maximum (S's first 64 columns reloaded from TMEM, the last 64 still
+        // in registers), which is rare after a row's first tiles.  Otherwise P <= 2^8 stays finite in bf16
+        // and the result is exact after the final O / l.
+        rowsum = exp_pass(m_used == -INFINITY ? 0.f : -m_used, std::true_type{});
+        const float m_tile = fmaxf(fmax3f(mx4[0], mx4[1], mx4[2]), mx4[3]) * scale_log2;
+        const bool grow = m_tile > m_used + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, grow)) {
+          float alpha = 1.f;
+          if (grow) {
+            alpha = ex2_approx(m_used - m_tile);  // 0 when nothing was seen before
+            l *= alpha;
+            m_used = m_tile;
+          }
+          // O row *= alpha.  The previous O += P V of this lane has completed (the S_t commit that
+          // signalled this step fires only after every earlier MMA of its issuer), and the next one
+          // waits for this thread's P.
+          rescale_o_row<D>(tO, alpha);
+#pragma unroll
+          for (int c = 0; c < 2; ++c) tmem_ld32(tS + c * 32, sr[c]);
+          tmem_wait_ld();
+          if (n_valid < kTile) {
+#pragma unroll
+            for (int c = 0; c < 2; ++c)
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (c * 32 + e >= n_valid) sr[c][e] = __float_as_uint(-INFINITY);
+          }
+          rowsum = exp_pass(m_used == -INFINITY ? 0.f : -m_used, std::false_type{});
+        }
       }
 #undef SV
-      const f2 acc01 = fadd2(acc[0], acc[1]);
-      const f2 acc23 = fadd2(acc[2], acc[3]);
-      const f2 acc4 = fadd2(acc01, acc23);
-      const float rowsum = acc4.x + acc4.y;
       l += rowsum;
       tmem_wait_st();
       tc_fence_before();

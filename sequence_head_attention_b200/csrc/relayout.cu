@@ -8,8 +8,10 @@
 //   head -> seq:  out_r[b, s', h, :] = in_{h / (H/P)}[b, r S/P + s', h % (H/P), :]
 // When the P ranks are separate processes, the all-to-all itself is a collective (NCCL) between contiguous
 // per-destination blocks, and each rank's local halves are copies of its own shard:
-//   split heads:  out_r[b, s, h', :] = in[b, s, r H/P + h', :]       (before the exchange)
-//   merge heads:  out[b, s, r H/P + h', :] = in_r[b, s, h', :]       (after the way back)
+//   split heads:  out_r[b, s, h', :] = in[b, s, r H/P + h0 + h', :]  (before the exchange)
+//   merge heads:  out[b, s, r H/P + h0 + h', :] = in_r[b, s, h', :]  (after the way back)
+// for h' < n of a sub-range [h0, h0 + n) of every rank's head group (the whole group, or one stage of a
+// chunked exchange).
 // All four move contiguous runs of (H/P) * D elements: one warp copies one run with 16-byte vector loads
 // and stores, up to 4 KB per lane group in flight, so both sides are fully coalesced.  Bit-exact.
 #include <cstdint>
@@ -28,7 +30,8 @@ enum RelayoutMode { kHeadToSeq = 0, kSeqToHead = 1, kSplitHeads = 2, kMergeHeads
 
 template <int kMode>
 __global__ void __launch_bounds__(256) relayout_kernel(const __grid_constant__ RankPtrs rp, int P, int B,
-                                                       int S, int H, long long run_bytes) {
+                                                       int S, int H, long long run_bytes, long long row_bytes,
+                                                       long long group_bytes, long long sub_off) {
   const int Sl = S / P;
   const long long n_runs = (long long)P * B * S;
   const int lane = threadIdx.x & 31;
@@ -38,17 +41,18 @@ __global__ void __launch_bounds__(256) relayout_kernel(const __grid_constant__ R
     const uint8_t* src;
     uint8_t* dst;
     if (kMode == kSplitHeads) {
-      // run = (r, b, s): destination out_r[b, s, :, :] (S here is the rank's own sequence length)
+      // run = (r, b, s): destination out_r[b, s, :, :] (S here is the rank's own sequence length); the source
+      // is the sub-range of rank r's head group in the row of (b, s)
       const long long bs = run % ((long long)B * S);
       const int r = (int)(run / ((long long)B * S));
-      src = rp.in[0] + (bs * P + r) * run_bytes;
+      src = rp.in[0] + bs * row_bytes + r * group_bytes + sub_off;
       dst = rp.out[r] + bs * run_bytes;
     } else if (kMode == kMergeHeads) {
-      // run = (b, s, r): destination out[b, s, r H/P : (r+1) H/P, :], contiguous in r
+      // run = (b, s, r): destination the sub-range of rank r's head group in out[b, s]
       const int r = (int)(run % P);
       const long long bs = run / P;
       src = rp.in[r] + bs * run_bytes;
-      dst = rp.out[0] + (bs * P + r) * run_bytes;
+      dst = rp.out[0] + bs * row_bytes + r * group_bytes + sub_off;
     } else if (kMode == kSeqToHead) {
       // run = (r, b, s): destination out_r[b, s, :, :], contiguous in s
       const int s = (int)(run % S);
@@ -94,10 +98,13 @@ __global__ void __launch_bounds__(256) relayout_kernel(const __grid_constant__ R
 }  // namespace
 
 static sp_status launch_runs(const RankPtrs& rp, int mode, int P, int B, int S, int H, int D, int elem_bytes,
-                             cudaStream_t stream) {
+                             cudaStream_t stream, int h0 = 0, int n_heads = -1) {
   // A run is the H/P heads of one (rank, b, s): H/P * D elements.  In the seq-sharded layout a row of
-  // H heads holds P consecutive runs, which is what the kernel's "* P + r" indexing uses.
-  const long long run_bytes = (long long)(H / P) * D * elem_bytes;
+  // H heads holds P consecutive runs, which is what the kernel's "* P + r" indexing uses.  The head-group
+  // copies move a sub-range [h0, h0 + n_heads) of each group.
+  const long long row_bytes = (long long)H * D * elem_bytes, group_bytes = row_bytes / P;
+  const long long run_bytes = n_heads < 0 ? group_bytes : (long long)n_heads * D * elem_bytes;
+  const long long sub_off = (long long)h0 * D * elem_bytes;
   const long long n_runs = (long long)P * B * S;
   if (n_runs == 0) return SP_OK;
   int dev = 0;
@@ -106,10 +113,14 @@ static sp_status launch_runs(const RankPtrs& rp, int mode, int P, int B, int S, 
   const long long cap = (long long)num_sms(dev) * 8;
   if (blocks > cap) blocks = cap;
   switch (mode) {
-    case kSeqToHead: relayout_kernel<kSeqToHead><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes); break;
-    case kHeadToSeq: relayout_kernel<kHeadToSeq><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes); break;
-    case kSplitHeads: relayout_kernel<kSplitHeads><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes); break;
-    default: relayout_kernel<kMergeHeads><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes); break;
+    case kSeqToHead: relayout_kernel<kSeqToHead><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes, row_bytes,
+                                                                   group_bytes, sub_off); break;
+    case kHeadToSeq: relayout_kernel<kHeadToSeq><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes, row_bytes,
+                                                                   group_bytes, sub_off); break;
+    case kSplitHeads: relayout_kernel<kSplitHeads><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes, row_bytes,
+                                                                   group_bytes, sub_off); break;
+    default: relayout_kernel<kMergeHeads><<<(unsigned)blocks, 256, 0, stream>>>(rp, P, B, S, H, run_bytes, row_bytes,
+                                                                   group_bytes, sub_off); break;
   }
   return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
 }
@@ -125,12 +136,12 @@ sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, i
 }
 
 sp_status launch_head_groups(const void* const* in, void* const* out, bool split, int P, int B, int S, int H, int D,
-                             int elem_bytes, cudaStream_t stream) {
+                             int h0, int n_heads, int elem_bytes, cudaStream_t stream) {
   RankPtrs rp = {};
   const int n_in = split ? 1 : P, n_out = split ? P : 1;
   for (int r = 0; r < n_in; ++r) rp.in[r] = static_cast<const uint8_t*>(in[r]);
   for (int r = 0; r < n_out; ++r) rp.out[r] = static_cast<uint8_t*>(out[r]);
-  return launch_runs(rp, split ? kSplitHeads : kMergeHeads, P, B, S, H, D, elem_bytes, stream);
+  return launch_runs(rp, split ? kSplitHeads : kMergeHeads, P, B, S, H, D, elem_bytes, stream, h0, n_heads);
 }
 
 }  // namespace spattn

@@ -105,9 +105,9 @@ sp_status launch_merge(const float* const* o_parts, const float* const* lse_part
 sp_status launch_relayout(const void* const* in_ranks, void* const* out_ranks, int P, int B, int S,
                           int H, int D, int elem_bytes, bool seq_to_head, cudaStream_t stream);
 // The local halves of a multi-process Ulysses exchange: split (in[0] -> out[0..P-1]) or merge
-// (in[0..P-1] -> out[0]) of the P head groups of a [B, S, H, D] sequence shard.
+// (in[0..P-1] -> out[0]) of heads [h0, h0 + n_heads) of each of the P head groups of a [B, S, H, D] shard.
 sp_status launch_head_groups(const void* const* in, void* const* out, bool split, int P, int B, int S, int H, int D,
-                             int elem_bytes, cudaStream_t stream);
+                             int h0, int n_heads, int elem_bytes, cudaStream_t stream);
 sp_status launch_tile_list(const uint8_t* mask, int H, int T, int32_t* row_ptr, int32_t* col_idx,
                            int32_t* counts, cudaStream_t stream);
 sp_status launch_debug_wait(unsigned long long timeout_ns, cudaStream_t stream);

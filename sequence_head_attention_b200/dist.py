@@ -5,16 +5,19 @@ Both schemes start from the same placement: rank r holds positions [r S/P, (r+1)
 heads, as [B, S/P, H, D] tensors in its own GPU's memory, and ends with the same rows of O.
 
 UlyssesAttention   ("HCMS: Head-Chunked Multi-Stream Pipeline ...", abstract: all-to-all based sequence
-                   parallelism; "db-SP ...", abstract: parallelism along the head dimension as in Ulysses)
-    1. sp_split_heads cuts each of Q, K, V into P head groups, written straight into the send buffer
-       [P, 3, B, S/P, H/P, D] (block r goes to rank r);
-    2. one all-to-all: block g of the receive buffer holds rank g's positions of this rank's heads;
-    3. sp_attn_fwd_seq_sharded attends this rank's H/P heads over the whole sequence, reading the P received
-       blocks as its sequence shards and writing O into the P blocks of the O send buffer (the head
-       chunks of the whole model are cut at the rank boundaries, as on one GPU);
-    4. a second all-to-all returns O's blocks to the ranks that own those positions;
-    5. sp_merge_heads joins the P head groups into this rank's O shard [B, S/P, H, D].
-    The lse stays head-sharded: rank r's [B, H/P, S] for its heads.
+                   parallelism, heads processed in chunks so that communication overlaps computation;
+                   "db-SP ...", abstract: parallelism along the head dimension as in Ulysses)
+    Each rank's H/P heads are processed in `stages` head chunks (1: one exchange of everything).  Per stage:
+    1. sp_split_heads cuts each of Q, K, V into P head groups (the stage's heads of each rank's group),
+       written straight into the stage's send buffer [P, 3, B, S/P, n, D] (block r goes to rank r);
+    2. an all-to-all: block g of the receive buffer holds rank g's positions of this rank's stage heads;
+    3. sp_attn_fwd_seq_sharded attends those heads over the whole sequence, reading the P received blocks as
+       its sequence shards and writing O into the P blocks of the stage's O send buffer;
+    4. an all-to-all returns O's blocks to the ranks that own those positions;
+    5. sp_merge_heads places the stage's heads of the P groups into this rank's O shard [B, S/P, H, D].
+    The collectives are asynchronous: the all-to-all of stage c + 1 is posted before the attention of stage
+    c and awaited after it, and each stage's O goes back while the next stage computes, so with NCCL the
+    exchanges run beside the attention kernels.  The lse stays head-sharded: rank r's [B, H/P, S].
 
 RingAttention      ("CHARM+: How Cross-Hardware Attention Breaks Through Distributed Communication
                    Bottlenecks", Ring-Attention paragraph: Q stays local while the KV blocks travel round a
@@ -65,12 +68,12 @@ class LibraryKernels:
     acc_dtype = torch.float32
 
     @staticmethod
-    def split_heads(x, outs):
-        spattn.sp_split_heads(x, outs)
+    def split_heads(x, outs, heads):
+        spattn.sp_split_heads(x, outs, heads=heads)
 
     @staticmethod
-    def merge_heads(ins, out):
-        spattn.sp_merge_heads(ins, out)
+    def merge_heads(ins, out, heads):
+        spattn.sp_merge_heads(ins, out, heads=heads)
 
     @staticmethod
     def attention_sharded(q_shards, k_shards, v_shards, o_shards, lse, head_chunks, causal):
@@ -90,9 +93,19 @@ class LibraryKernels:
         spattn.sp_convert_f32_to_bf16(o_acc, o)
 
 
+def stage_bounds(n, stages):
+    """Contiguous near-equal head chunks of n heads in `stages` stages (the first ones one larger)."""
+    stages = max(1, min(int(stages), n))
+    q, r = divmod(n, stages)
+    cuts = [0]
+    for c in range(stages):
+        cuts.append(cuts[-1] + q + (1 if c < r else 0))
+    return list(zip(cuts[:-1], cuts[1:]))
+
+
 class UlyssesAttention:
     def __init__(self, B, S, H, D, head_chunks=None, causal=False, group=None, device=None, dtype=torch.bfloat16,
-                 kernels=LibraryKernels):
+                 kernels=LibraryKernels, stages=1):
         self.group = group
         self.P = dist.get_world_size(group)
         self.rank = dist.get_rank(group)
@@ -102,34 +115,69 @@ class UlyssesAttention:
         self.B, self.S, self.H, self.D, self.Sl, self.Hl = B, S, H, D, S // P, H // P
         self.causal = causal
         self.kernels = kernels
-        self.chunks = rank_chunks(head_chunks or (H,), H, P)[self.rank]
-        blk = (B, self.Sl, self.Hl, D)
-        self.send = torch.empty((P, 3) + blk, dtype=dtype, device=device)
-        self.recv = torch.empty_like(self.send)
-        self.o_send = torch.empty((P,) + blk, dtype=dtype, device=device)
-        self.o_recv = torch.empty_like(self.o_send)
-        self.lse = torch.empty((B, self.Hl, S), dtype=kernels.acc_dtype, device=device)
+        self.stages = stage_bounds(self.Hl, stages)
+        # the model's head chunks, cut at the rank boundaries and then at the stage boundaries (they only
+        # order the work within a launch: each stage's launch takes its part of this rank's chunk list)
+        rank_chunk = rank_chunks(head_chunks or (H,), H, P)[self.rank]
+        self.chunks = []
+        for h0, h1 in self.stages:
+            part, a = [], 0
+            for c in rank_chunk:
+                lo, hi = max(a, h0), min(a + c, h1)
+                if hi > lo:
+                    part.append(hi - lo)
+                a += c
+            self.chunks.append(part)
+        self.send, self.recv, self.o_send, self.o_recv, self.lse = [], [], [], [], []
+        for h0, h1 in self.stages:
+            blk = (B, self.Sl, h1 - h0, D)
+            self.send.append(torch.empty((P, 3) + blk, dtype=dtype, device=device))
+            self.recv.append(torch.empty((P, 3) + blk, dtype=dtype, device=device))
+            self.o_send.append(torch.empty((P,) + blk, dtype=dtype, device=device))
+            self.o_recv.append(torch.empty((P,) + blk, dtype=dtype, device=device))
+            self.lse.append(torch.empty((B, h1 - h0, S), dtype=kernels.acc_dtype, device=device))
 
     def forward(self, q, k, v, out=None, phase=None):
-        """q, k, v: this rank's [B, S/P, H, D] shards.  Returns its [B, S/P, H, D] shard of O.
-        phase(name, fn), if given, runs each part (to bracket it with timing events)."""
-        P = self.P
+        """q, k, v: this rank's [B, S/P, H, D] shards.  Returns its [B, S/P, H, D] shard of O; the lse of this
+        rank's heads is left in self.lse (one [B, n, S] tensor per stage).  phase(name, fn), if given, runs
+        each part (to bracket it with timing events)."""
+        P, n = self.P, len(self.stages)
         run = phase or (lambda name, fn: fn())
-        run("split", lambda: [self.kernels.split_heads(x, [self.send[r, i] for r in range(P)])
-                              for i, x in enumerate((q, k, v))])
-        run("exchange", lambda: dist.all_to_all_single(self.recv, self.send, group=self.group))
-        run("attn", lambda: self.kernels.attention_sharded(
-            [self.recv[g, 0] for g in range(P)], [self.recv[g, 1] for g in range(P)],
-            [self.recv[g, 2] for g in range(P)], [self.o_send[g] for g in range(P)], self.lse, self.chunks,
-            self.causal))
-        run("exchange", lambda: dist.all_to_all_single(self.o_recv, self.o_send, group=self.group))
+
+        def a2a(dst, src):
+            return dist.all_to_all_single(dst, src, group=self.group, async_op=True)
+
+        def split():
+            for c, (h0, h1) in enumerate(self.stages):
+                for i, x in enumerate((q, k, v)):
+                    self.kernels.split_heads(x, [self.send[c][r, i] for r in range(P)], (h0, h1 - h0))
+
+        run("split", split)
+        pending = {0: a2a(self.recv[0], self.send[0])}
+        back = []
+        for c in range(n):
+            if c + 1 < n:
+                pending[c + 1] = a2a(self.recv[c + 1], self.send[c + 1])  # the next stage's heads travel now
+            run("exchange", pending.pop(c).wait)
+            rc, oc = self.recv[c], self.o_send[c]
+            run("attn", lambda rc=rc, oc=oc, c=c: self.kernels.attention_sharded(
+                [rc[g, 0] for g in range(P)], [rc[g, 1] for g in range(P)], [rc[g, 2] for g in range(P)],
+                [oc[g] for g in range(P)], self.lse[c], self.chunks[c], self.causal))
+            back.append(a2a(self.o_recv[c], self.o_send[c]))  # this stage's O goes back while the next computes
         o = out if out is not None else torch.empty_like(q)
-        run("merge", lambda: self.kernels.merge_heads([self.o_recv[r] for r in range(P)], o))
+        for c, (h0, h1) in enumerate(self.stages):
+            run("exchange", back[c].wait)
+            run("merge", lambda c=c, h0=h0, h1=h1: self.kernels.merge_heads(
+                [self.o_recv[c][r] for r in range(P)], o, (h0, h1 - h0)))
         return o
+
+    def lse_heads(self):
+        """This rank's lse [B, H/P, S] (the stages' lse joined along the heads)."""
+        return torch.cat(self.lse, dim=1)
 
     def bytes_exchanged(self):
         """Bytes this rank sends to other ranks per forward (Q, K, V out, O back; its own block stays)."""
-        per_block = self.B * self.Sl * self.Hl * self.D * self.send.element_size()
+        per_block = self.B * self.Sl * self.Hl * self.D * self.send[0].element_size()
         return 4 * (self.P - 1) * per_block
 
 

@@ -54,8 +54,8 @@ def lib() -> ctypes.CDLL:
                 "sp_seq_to_head_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_head_to_seq_relayout": (I, [P, P, I, I, I, I, I, I, P]),
                 "sp_attn_fwd_seq_sharded": (I, [P, P, P, P, P, I, I, I, I, I, I, I, P, I, I, P]),
-                "sp_split_heads": (I, [P, P, I, I, I, I, I, I, P]),
-                "sp_merge_heads": (I, [P, P, I, I, I, I, I, I, P]),
+                "sp_split_heads": (I, [P, P, I, I, I, I, I, I, I, I, P]),
+                "sp_merge_heads": (I, [P, P, I, I, I, I, I, I, I, I, P]),
                 "sp_attn_fwd_items": (I, [P, P, P, P, P, I, I, I, I, P, I, I, P, P, Z, P]),
                 "sp_attn_bwd_workspace_bytes": (Z, [I, I, I, I]),
                 "sp_attn_bwd": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, P, Z, P]),
@@ -281,29 +281,35 @@ def sp_head_to_seq_relayout(in_ranks, out_ranks, S=None, H=None, stream=None):
     return out_ranks
 
 
-def sp_split_heads(x, out_ranks, stream=None):
-    """x [B, S, H, D] (this rank's sequence shard) -> P head groups out_ranks[r] [B, S, H/P, D] (bit-exact)."""
+def sp_split_heads(x, out_ranks, heads=None, stream=None):
+    """x [B, S, H, D] (this rank's sequence shard) -> P head groups out_ranks[r] [B, S, n, D] holding heads
+    [r H/P + h0, r H/P + h0 + n) with heads=(h0, n) (default: each whole group), bit-exact."""
     P = len(out_ranks)
     B, S, H, D = x.shape
+    h0, n = (0, H // P) if heads is None else (int(heads[0]), int(heads[1]))
     _need(x.is_cuda and x.is_contiguous(), "x must be a contiguous CUDA tensor")
     for t in out_ranks:
-        _need(t.is_cuda and t.is_contiguous() and t.dtype == x.dtype and tuple(t.shape) == (B, S, H // P, D)
-              and t.device == x.device, "out_ranks must be contiguous [B, S, H/P, D] of x's dtype and device")
+        _need(t.is_cuda and t.is_contiguous() and t.dtype == x.dtype and tuple(t.shape) == (B, S, n, D)
+              and t.device == x.device, "out_ranks must be contiguous [B, S, n, D] of x's dtype and device")
     op, _k = _ptr_array(out_ranks)
-    _check("sp_split_heads", lib().sp_split_heads(_ptr(x), op, P, B, S, H, D, x.element_size(), _stream(stream)))
+    _check("sp_split_heads", lib().sp_split_heads(_ptr(x), op, P, B, S, H, D, h0, n, x.element_size(),
+                                                  _stream(stream)))
     return out_ranks
 
 
-def sp_merge_heads(in_ranks, out, stream=None):
-    """P head groups in_ranks[r] [B, S, H/P, D] -> out [B, S, H, D] (bit-exact)."""
+def sp_merge_heads(in_ranks, out, heads=None, stream=None):
+    """P head groups in_ranks[r] [B, S, n, D] -> heads [r H/P + h0, r H/P + h0 + n) of out [B, S, H, D] with
+    heads=(h0, n) (default: each whole group), bit-exact; out's other heads are left untouched."""
     P = len(in_ranks)
     B, S, H, D = out.shape
+    h0, n = (0, H // P) if heads is None else (int(heads[0]), int(heads[1]))
     _need(out.is_cuda and out.is_contiguous(), "out must be a contiguous CUDA tensor")
     for t in in_ranks:
-        _need(t.is_cuda and t.is_contiguous() and t.dtype == out.dtype and tuple(t.shape) == (B, S, H // P, D)
-              and t.device == out.device, "in_ranks must be contiguous [B, S, H/P, D] of out's dtype and device")
+        _need(t.is_cuda and t.is_contiguous() and t.dtype == out.dtype and tuple(t.shape) == (B, S, n, D)
+              and t.device == out.device, "in_ranks must be contiguous [B, S, n, D] of out's dtype and device")
     ip, _k = _ptr_array(in_ranks)
-    _check("sp_merge_heads", lib().sp_merge_heads(ip, _ptr(out), P, B, S, H, D, out.element_size(), _stream(stream)))
+    _check("sp_merge_heads", lib().sp_merge_heads(ip, _ptr(out), P, B, S, H, D, h0, n, out.element_size(),
+                                                  _stream(stream)))
     return out
 
 

@@ -144,12 +144,14 @@ def test_split_and_merge_heads_reject_on_host(L):
     o = ctypes.cast(outs, ctypes.c_void_p)
     x = 5 << 24
     f, g = L.sp_split_heads, L.sp_merge_heads
-    assert f(x, o, 4, 1, 16, 6, 64, 2, None) == spattn.SP_ERR_INVALID_ARG     # H % P
-    assert f(x, o, 4, 1, 16, 8, 4, 2, None) == spattn.SP_ERR_INVALID_ARG     # D * elem not a multiple of 16
-    assert f(x, o, 4, 1, 16, 8, 64, 3, None) == spattn.SP_ERR_INVALID_ARG    # elem_bytes
-    assert f(x + 8, o, 4, 1, 16, 8, 64, 2, None) == spattn.SP_ERR_INVALID_ARG  # misaligned
-    assert f(1 << 24, o, 4, 1, 16, 8, 64, 2, None) == spattn.SP_ERR_INVALID_ARG  # input overlaps output 0
+    assert f(x, o, 4, 1, 16, 6, 64, 0, 1, 2, None) == spattn.SP_ERR_INVALID_ARG     # H % P
+    assert f(x, o, 4, 1, 16, 8, 4, 0, 2, 2, None) == spattn.SP_ERR_INVALID_ARG      # D * elem not a multiple of 16
+    assert f(x, o, 4, 1, 16, 8, 64, 0, 2, 3, None) == spattn.SP_ERR_INVALID_ARG     # elem_bytes
+    assert f(x + 8, o, 4, 1, 16, 8, 64, 0, 2, 2, None) == spattn.SP_ERR_INVALID_ARG  # misaligned
+    assert f(x, o, 4, 1, 16, 8, 64, 1, 2, 2, None) == spattn.SP_ERR_INVALID_ARG     # heads past the group (2)
+    assert f(x, o, 4, 1, 16, 8, 64, 0, 0, 2, None) == spattn.SP_ERR_INVALID_ARG     # no head
+    assert f(1 << 24, o, 4, 1, 16, 8, 64, 0, 2, 2, None) == spattn.SP_ERR_INVALID_ARG  # input overlaps output 0
     same = (ctypes.c_void_p * 4)(1 << 24, 1 << 24, 3 << 24, 4 << 24)
-    assert f(x, ctypes.cast(same, ctypes.c_void_p), 4, 1, 16, 8, 64, 2, None) == spattn.SP_ERR_INVALID_ARG
-    assert g(o, x, 0, 1, 16, 8, 64, 2, None) == spattn.SP_ERR_INVALID_ARG     # P
-    assert g(o, 2 << 24, 4, 1, 16, 8, 64, 2, None) == spattn.SP_ERR_INVALID_ARG  # output overlaps input 1
+    assert f(x, ctypes.cast(same, ctypes.c_void_p), 4, 1, 16, 8, 64, 0, 2, 2, None) == spattn.SP_ERR_INVALID_ARG
+    assert g(o, x, 0, 1, 16, 8, 64, 0, 2, 2, None) == spattn.SP_ERR_INVALID_ARG     # P
+    assert g(o, 2 << 24, 4, 1, 16, 8, 64, 0, 2, 2, None) == spattn.SP_ERR_INVALID_ARG  # output overlaps input 1

@@ -27,15 +27,23 @@ class OracleKernels:
     acc_dtype = torch.float64
 
     @staticmethod
-    def split_heads(x, outs):
+    def split_heads(x, outs, heads):
         import oracle
+        h0, n = heads
         for o, part in zip(outs, oracle.split_heads(x.numpy(), len(outs))):
-            o.copy_(torch.from_numpy(part))
+            o.copy_(torch.from_numpy(part[:, :, h0:h0 + n]))
 
     @staticmethod
-    def merge_heads(ins, out):
+    def merge_heads(ins, out, heads):
+        # the stage's heads of each group into out (the oracle's merge of whole groups, with the other heads
+        # of every group taken from out as it stands)
         import oracle
-        out.copy_(torch.from_numpy(oracle.merge_heads([t.numpy() for t in ins])))
+        h0, n = heads
+        P = len(ins)
+        groups = oracle.split_heads(out.numpy(), P)
+        for r in range(P):
+            groups[r][:, :, h0:h0 + n] = ins[r].numpy()
+        out.copy_(torch.from_numpy(oracle.merge_heads(groups)))
 
     @staticmethod
     def attention_sharded(q_shards, k_shards, v_shards, o_shards, lse, head_chunks, causal):
@@ -73,7 +81,7 @@ def _inputs(B, S, H, D, seed):
     return q.double(), k.double(), v.double()
 
 
-def _worker(rank, world, port, scheme, causal, out):
+def _worker(rank, world, port, scheme, causal, out, stages=1):
     os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "MASTER_ADDR": "127.0.0.1",
                        "MASTER_PORT": str(port)})
     sys.path.insert(0, ROOT)
@@ -92,16 +100,18 @@ def _worker(rank, world, port, scheme, causal, out):
         ref_o, ref_l = oracle.attention(q.numpy(), k.numpy(), v.numpy(), causal=causal, nthreads=1)
         if scheme == "ulysses":
             sp = sp_dist.UlyssesAttention(B, S, H, D, head_chunks=[1, H - 1], causal=causal, dtype=torch.float64,
-                                          kernels=OracleKernels)
+                                          kernels=OracleKernels, stages=stages)
             o = sp.forward(*mine)
-            # the exchange delivered exactly the seq -> head relayout of every tensor (bit for bit)
+            # the exchanges delivered exactly the seq -> head relayout of every tensor (bit for bit), stage by
+            # stage
             for i, t in enumerate((q, k, v)):
                 shards = [t[:, g * Sl:(g + 1) * Sl].numpy() for g in range(world)]
                 want = oracle.seq_to_head(shards, H)[rank]
-                got = torch.cat([sp.recv[g, i] for g in range(world)], dim=1).numpy()
+                got = torch.cat([torch.cat([sp.recv[c][g, i] for g in range(world)], dim=1)
+                                 for c in range(len(sp.stages))], dim=2).numpy()
                 assert np.array_equal(got, want)
             Hl = H // world
-            lse_err = float(np.max(np.abs(sp.lse.numpy() - ref_l[:, rank * Hl:(rank + 1) * Hl])))
+            lse_err = float(np.max(np.abs(sp.lse_heads().numpy() - ref_l[:, rank * Hl:(rank + 1) * Hl])))
             rounds = None
         else:
             sp = sp_dist.RingAttention(B, S, H, D, causal=causal, dtype=torch.float64, kernels=OracleKernels)
@@ -114,14 +124,17 @@ def _worker(rank, world, port, scheme, causal, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 4])
-@pytest.mark.parametrize("scheme", ["ulysses", "ring"])
-@pytest.mark.parametrize("causal", [False, True])
-def test_sequence_parallel_schemes_on_gloo_ranks(world, scheme, causal):
+@pytest.mark.parametrize("world,scheme,causal,stages", [
+    (2, "ulysses", False, 1), (4, "ulysses", True, 1), (2, "ulysses", True, 3), (4, "ulysses", False, 2),
+    (2, "ring", False, 1), (2, "ring", True, 1), (4, "ring", False, 1), (4, "ring", True, 1),
+])
+def test_sequence_parallel_schemes_on_gloo_ranks(world, scheme, causal, stages):
+    """Ulysses in one exchange and in head-chunk stages (HCMS: the next stage's all-to-all posted before the
+    current stage's attention), and the ring, on 2 and 4 ranks."""
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, scheme, causal, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, scheme, causal, q, stages)) for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:

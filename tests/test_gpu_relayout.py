@@ -94,3 +94,15 @@ def test_split_and_merge_heads_bit_exact(P, B, S, H, D, dtype):
         assert torch.all(outs_buf[r][:guard] == 7) and torch.all(outs_buf[r][-guard:] == 7)
     assert np.array_equal(_bits(back), oracle.merge_heads(ref))
     assert np.array_equal(_bits(back), _bits(x))
+    # stages of a chunked exchange: heads [h0, h0 + n) of every group, against the oracle's groups sliced
+    Hl = H // P
+    cuts = [0, (Hl + 1) // 2, Hl] if Hl > 1 else [0, 1]
+    back2 = torch.zeros_like(xd)
+    for h0, h1 in zip(cuts[:-1], cuts[1:]):
+        part = [torch.empty((B, S, h1 - h0, D), dtype=dtype, device="cuda") for _ in range(P)]
+        spattn.sp_split_heads(xd, part, heads=(h0, h1 - h0))
+        spattn.sp_merge_heads(part, back2, heads=(h0, h1 - h0))
+        torch.cuda.synchronize()
+        for r in range(P):
+            assert np.array_equal(_bits(part[r]), ref[r][:, :, h0:h1])
+    assert np.array_equal(_bits(back2), _bits(x))
