@@ -479,7 +479,9 @@ def measure_main(wname, args, peaks, dev, stream, world, seed, headline):
     fused = wname == "video_dit" and args.ulysses == "fused"
     # Launch overlap where the step's attention launches follow one another and no kernel writes the Q, K, V
     # of the launch after it: the per-rank launches on the shards, the ring's blocks, the masked launches.
-    overlap = not args.no_overlap and (fused or wname != "video_dit")
+    # The per-rank launches also write disjoint heads of the shards (and lse rows), so they overlap their
+    # outputs too (mode 2); a ring block reads the running result the block before wrote (mode 1).
+    overlap = 0 if args.no_overlap or (wname == "video_dit" and not fused) else (2 if fused else 1)
     spattn.sp_set_launch_overlap(overlap)
     step = make_step(wname, w, q, k, v, mask, dev, fused, with_partials=wname == "ring_causal")
     for _ in range(args.warmup):
@@ -561,7 +563,7 @@ def latency_report(wname, dev, stream, peaks, reps=200):
     import torch
     from sequence_head_attention_b200 import spattn, synth
     w = synth.WORKLOADS[wname]
-    spattn.sp_set_launch_overlap(False)  # plain calls, each launch after the previous kernel
+    spattn.sp_set_launch_overlap(0)  # plain calls, each launch after the previous kernel
     q, k, v = (t.to(dev) for t in synth.qkv(w.B, w.S, w.H, w.D, seed=0, scale=w.scale)[:3])
     o = torch.empty_like(q)
     lse = torch.empty((w.B, w.H, w.S), dtype=torch.float32, device=dev)

@@ -352,17 +352,22 @@ SP_API sp_status sp_check_device_error(sp_stream stream);
 SP_API sp_status sp_check_device_error_bits(sp_stream stream, unsigned int* bits);
 
 /*
- * Launch overlap (default off).  With it on, every attention launch (sp_attn_fwd and the other attention
+ * Launch overlap (default 0, off).  With it on, every attention launch (sp_attn_fwd and the other attention
  * entry points) may start while the kernel enqueued just before it on the same stream is still finishing:
  * its CTAs take the SMs that kernel frees (programmatic dependent launch), which fills the tail of a
- * sequence of attention launches such as one launch per Ulysses rank or per ring round.  An overlapped
- * launch reads only q, k and v early: it writes o and lse (and sp_attn_fwd_partial_merge reads its running
- * result) only after the kernel before it has completed, and a masked or item-list launch waits for it
- * before reading anything (that kernel may have built its tile list).  The caller promises that q, k and
- * v are not written by the kernel enqueued just before the launch.  Kernels enqueued after an attention
- * launch wait for it as usual.  Applies to later launches; process-wide.
+ * sequence of attention launches such as one launch per Ulysses rank or per ring round.
+ *   mode 1: an overlapped launch reads only q, k and v early; it writes o and lse (and
+ *           sp_attn_fwd_partial_merge reads its running result) only after the kernel before it has
+ *           completed.  The caller promises that q, k and v are not written by that kernel.
+ *   mode 2: as mode 1, and the caller also promises that the kernel just before neither reads nor writes
+ *           the parts of o and lse this launch writes (e.g. launches for disjoint heads of one output), so
+ *           the launch writes them without waiting.  sp_attn_fwd_partial_merge still waits before reading
+ *           its running result.
+ * In both modes a masked or item-list launch waits for the kernel before it (which may have built its tile
+ * list) before reading anything.  Kernels enqueued after an attention launch wait for it as usual.  Applies
+ * to later launches; process-wide.
  */
-SP_API void sp_set_launch_overlap(int enable);
+SP_API void sp_set_launch_overlap(int mode);
 
 /* Time limit of every device-side wait, in nanoseconds (default 2e9).  Applies to later launches. */
 SP_API void sp_set_wait_timeout_ns(unsigned long long ns);

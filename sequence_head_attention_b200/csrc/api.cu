@@ -24,7 +24,7 @@ int g_num_sms[kMaxDevices] = {};
 unsigned int* g_err_addr[kMaxDevices] = {};
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 unsigned long long g_timeout_ns = 2000000000ull;
-bool g_overlap = false;
+int g_overlap = 0;
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -119,7 +119,7 @@ int num_sms(int device) {
 
 unsigned long long wait_timeout_ns() { return g_timeout_ns; }
 
-bool launch_overlap() { return g_overlap; }
+int launch_overlap() { return g_overlap; }
 
 unsigned int* device_error_word() {
   int dev = 0;
@@ -199,9 +199,9 @@ const char* sp_status_string(sp_status s) {
 
 const char* sp_version(void) { return "spattn 0.1 (sm_100a)"; }
 
-void sp_set_launch_overlap(int enable) {
+void sp_set_launch_overlap(int mode) {
   std::lock_guard<std::mutex> lk(g_mu);
-  g_overlap = enable != 0;
+  g_overlap = mode <= 0 ? 0 : (mode == 1 ? 1 : 2);
 }
 
 void sp_set_wait_timeout_ns(unsigned long long ns) {

@@ -1128,8 +1128,9 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
       ++total_pv;
     }
     if (!ok) break;
-    // Overlapped launch: nothing is written (or, merging, read) before the kernel before it has completed.
-    if (p.pdl) pdl_wait();
+    // Overlapped launch: nothing is written (or, merging, read) before the kernel before it has completed,
+    // unless the caller promised that kernel touches none of this launch's outputs.
+    if (p.pdl_wait_epi) pdl_wait();
     // Epilogue: O / l and lse for the rows of this lane.
     if (kSplit && lane_valid) {
       ok = split_epilogue<D>(p, tm, sbase, bars, trow, it, q_row, row, warp, lane, lane_t, q_row < it.q_end, l, m_used,
@@ -1316,8 +1317,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_holder;
   if (p.pdl) {
     // Set up: the next launch may start on the SMs this grid frees.  A launch whose tile or item list the
-    // kernel before it wrote waits for that kernel here; every launch waits for it before its epilogue
-    // writes (run_softmax), so only Q, K and V are read early: they are the caller's promise.
+    // kernel before it wrote waits for that kernel here; otherwise it waits before its first epilogue
+    // (run_softmax) or, when the caller promised that the kernel before touches none of its outputs, not
+    // at all (a merging launch always waits before reading its running result).
     if (threadIdx.x == 0) pdl_launch_dependents();
     if (p.pdl_wait_start) pdl_wait();
   }
@@ -1479,8 +1481,10 @@ sp_status launch_attn_sharded(const AttnParams& p_in, cudaStream_t stream) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return SP_ERR_CUDA;
   const int sms = num_sms(dev);
-  p.pdl = launch_overlap() ? 1 : 0;
-  p.pdl_wait_start = (p.row_ptr || p.item_list) ? 1 : 0;  // lists built by the kernel just before
+  const int overlap = launch_overlap();
+  p.pdl = overlap > 0 ? 1 : 0;
+  p.pdl_wait_start = (p.pdl && (p.row_ptr || p.item_list)) ? 1 : 0;  // lists built by the kernel just before
+  p.pdl_wait_epi = (p.pdl && (overlap == 1 || p.o_merge)) ? 1 : 0;    // a running result is always waited for
   const bool pair = p.D == 128 && !p.row_ptr && !p.item_list && sms >= 2 && pair_enabled();
   TMaps tm{};  // the kernel argument (copied at launch)
   for (int r = 0; r < p.n_shards; ++r)

@@ -34,6 +34,7 @@ struct AttnParams {
   int pdl;          // 1: launched to overlap the kernel before it on the stream (programmatic dependent
                     // launch); reads of what that kernel writes wait for it (pdl_wait below)
   int pdl_wait_start;  // 1: wait for the previous kernel before reading anything (its output is an input here)
+  int pdl_wait_epi;    // 1: wait for the previous kernel before the first epilogue (writes, or merging reads)
   const int* item_list; // device list of work-item ids (nullptr: items 0 .. n_items-1); ids index the
                         // one-chunk layout (b * H + h) * n_qpairs + qp, and ids outside it are skipped
   int item_space;       // number of valid ids (B * H * n_qpairs) when item_list is set
@@ -88,7 +89,7 @@ bool encode_bshd_tmap(CUtensorMap* map, const void* base, int B, int S, int H, i
 // (64 bf16 or 32 fp32 values) by 32 positions, 128-byte swizzle.
 bool encode_o_tmap(CUtensorMap* map, void* base, int B, int S, int H, int D, bool f32);
 unsigned long long wait_timeout_ns();
-bool launch_overlap();  // sp_set_launch_overlap
+int launch_overlap();  // sp_set_launch_overlap: 0 off, 1 inputs, 2 inputs and outputs
 unsigned int* device_error_word();  // address of the current device's error word, or nullptr
 
 // Launchers (host validation is done by the C entry points before these are called).

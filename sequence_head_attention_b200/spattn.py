@@ -509,10 +509,11 @@ def sp_set_wait_timeout_ns(ns: int) -> None:
     lib().sp_set_wait_timeout_ns(int(ns))
 
 
-def sp_set_launch_overlap(enable: bool) -> None:
-    """Let each attention launch start while the kernel before it on the stream finishes (see the header
-    for what the caller promises)."""
-    lib().sp_set_launch_overlap(int(bool(enable)))
+def sp_set_launch_overlap(mode) -> None:
+    """Let each attention launch start while the kernel before it on the stream finishes: 0 (or False) off,
+    1 (or True) early reads of q, k, v only, 2 also outputs written without waiting (see the header for
+    what the caller promises in each mode)."""
+    lib().sp_set_launch_overlap(int(mode))
 
 
 def sp_debug_wait_timeout(timeout_ns: int, stream=None) -> None:

@@ -15,13 +15,13 @@ pytestmark = pytest.mark.gpu
 
 @pytest.fixture
 def overlap():
-    spattn.sp_set_launch_overlap(True)
+    spattn.sp_set_launch_overlap(1)
     yield
-    spattn.sp_set_launch_overlap(False)
+    spattn.sp_set_launch_overlap(0)
 
 
-def _run(fn, overlap_on):
-    spattn.sp_set_launch_overlap(overlap_on)
+def _run(fn, mode):
+    spattn.sp_set_launch_overlap(mode)
     out = fn()
     torch.cuda.synchronize()
     st, bits = spattn.sp_check_device_error_bits()
@@ -39,10 +39,11 @@ def test_rank_launches_on_shards(overlap):
             step.run()
         return step.o_seq + [step.lse_all]
 
-    ref = _run(go, False)
-    got = _run(go, True)
-    for a, b in zip(got, ref):
-        assert torch.equal(a, b)
+    ref = _run(go, 0)
+    for mode in (1, 2):  # mode 2: the ranks write disjoint heads, so outputs are written without waiting
+        got = _run(go, mode)
+        for a, b in zip(got, ref):
+            assert torch.equal(a, b)
 
 
 def test_ring_merging_launches(overlap):
@@ -55,8 +56,8 @@ def test_ring_merging_launches(overlap):
             step.run()
         return [step.o, step.lse]
 
-    ref = _run(go, False)
-    got = _run(go, True)
+    ref = _run(go, 0)
+    got = _run(go, 1)
     for a, b in zip(got, ref):
         assert torch.equal(a, b)
 
@@ -71,7 +72,7 @@ def test_masked_launches(overlap):
             step.run()
         return [step.o, step.lse]
 
-    ref = _run(go, False)
-    got = _run(go, True)
+    ref = _run(go, 0)
+    got = _run(go, 1)
     for a, b in zip(got, ref):
         assert torch.equal(a, b)
