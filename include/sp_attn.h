@@ -81,7 +81,9 @@ typedef void* sp_stream;
  * Bytes of device workspace sp_attn_fwd / sp_attn_fwd_partial need for these sizes.
  * n_kv_blocks > 1 needs n_kv_blocks fp32 partials (O [B,S,H,D] and LSE [B,H,S] each); has_mask != 0
  * needs the compacted tile list (H * ceil(S/128) + 1 row offsets and up to H * ceil(S/128)^2 tile
- * indices, int32).  Returns 0 when neither applies, and 0 for invalid sizes.
+ * indices, int32) and the launch's work order (B * H * ceil(ceil(S/128) / 2) item ids, int32: a masked
+ * launch claims its work items most kept tiles first).  Each section is rounded up to 256 bytes.
+ * Returns 0 when neither applies, and 0 for invalid sizes.
  */
 SP_API size_t sp_attn_fwd_workspace_bytes(int B, int S, int H, int D, int n_kv_blocks, int has_mask);
 

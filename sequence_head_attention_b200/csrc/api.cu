@@ -31,10 +31,10 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t parts_o = 0, parts_lse = 0, row_ptr = 0, col_idx = 0, counts = 0, total = 0;
+  size_t parts_o = 0, parts_lse = 0, row_ptr = 0, col_idx = 0, counts = 0, order = 0, total = 0;
 };
 
-// Workspace: [n_kv_blocks fp32 O partials][n_kv_blocks fp32 LSE partials][row_ptr][col_idx][counts]
+// Workspace: [n_kv_blocks fp32 O partials][n_kv_blocks fp32 LSE partials][row_ptr][col_idx][counts][order]
 WsLayout ws_layout(int B, int S, int H, int D, int n_kv_blocks, int has_mask) {
   WsLayout w;
   size_t off = 0;
@@ -52,6 +52,8 @@ WsLayout ws_layout(int B, int S, int H, int D, int n_kv_blocks, int has_mask) {
     off += align_up(H * T * T * sizeof(int32_t), 256);
     w.counts = off;
     off += align_up(H * T * sizeof(int32_t), 256);
+    w.order = off;  // the launch's work order: B * H * ceil(T / 2) item ids
+    off += align_up((size_t)B * H * ((T + 1) / 2) * sizeof(int32_t), 256);
   }
   w.total = off;
   return w;
@@ -373,6 +375,14 @@ sp_status sp_attn_fwd(const void* q, const void* k, const void* v, void* o, floa
     p.o = o;
     p.o_f32 = 0;
     p.lse = lse;
+    if (block_mask && n_chunks == 1) {
+      // claim the items most-kept-tiles first, so that the launch ends with short items
+      int32_t* order = reinterpret_cast<int32_t*>(ws + wl.order);
+      if (launch_item_order(p.row_ptr, B, H, p.mask_T, p.n_qpairs, order, st)) {
+        p.item_list = order;
+        p.item_space = p.n_items;
+      }
+    }
     return launch_attn(p, q, k, v, st);
   }
   // KV blocks: ceil(S / n) keys each (a multiple of 128 with a mask), partials into the workspace, then

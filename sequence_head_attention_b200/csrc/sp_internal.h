@@ -111,6 +111,9 @@ sp_status launch_head_groups(const void* const* in, void* const* out, bool split
                              int h0, int n_heads, int elem_bytes, cudaStream_t stream);
 sp_status launch_tile_list(const uint8_t* mask, int H, int T, int32_t* row_ptr, int32_t* col_idx,
                            int32_t* counts, cudaStream_t stream);
+// Item ids of a block-sparse launch (one head chunk, pairs of query tiles) ordered by kept tiles, most first,
+// into order[B * H * NP]; false (nothing launched) when the costs span more bins than the sort handles.
+bool launch_item_order(const int32_t* row_ptr, int B, int H, int T, int NP, int32_t* order, cudaStream_t stream);
 sp_status launch_debug_wait(unsigned long long timeout_ns, cudaStream_t stream);
 sp_status launch_debug_exp2_poly(const float* x, float* y, int n, cudaStream_t stream);
 

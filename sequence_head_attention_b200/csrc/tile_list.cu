@@ -81,6 +81,63 @@ __global__ void __launch_bounds__(256) tile_fill_kernel(const uint8_t* mask, int
   }
 }
 
+// Work order of a block-sparse launch: the item ids (b * H + h) * NP + qp (a pair of query tiles 2 qp and
+// 2 qp + 1 of head h) sorted by their kept tiles, most first, so that the dynamically claimed items of the
+// launch end with the short ones (longest-processing-time order; per-head densities vary several-fold).
+// A counting sort in one block: histogram of the costs (0 .. 2T) in shared memory, exclusive offsets from
+// the largest cost down, then each item placed with a shared-memory atomic (items of equal cost land in any
+// order; each item's arithmetic does not depend on it).
+constexpr int kMaxOrderBins = 4096;
+__global__ void __launch_bounds__(1024) item_order_kernel(const int32_t* row_ptr, int B, int H, int T, int NP,
+                                                          int32_t* order) {
+  __shared__ int32_t bins[kMaxOrderBins];
+  __shared__ int32_t warp_tot[32];
+  const int n_bins = 2 * T + 1, n_items = B * H * NP, tid = threadIdx.x;
+  auto cost = [&](int w) {
+    const int h = (w / NP) % H, qp = w % NP;
+    const int r0 = h * T + 2 * qp;
+    int c = row_ptr[r0 + 1] - row_ptr[r0];
+    if (2 * qp + 1 < T) c += row_ptr[r0 + 2] - row_ptr[r0 + 1];
+    return c;
+  };
+  for (int i = tid; i < n_bins; i += 1024) bins[i] = 0;
+  __syncthreads();
+  for (int w = tid; w < n_items; w += 1024) atomicAdd(&bins[cost(w)], 1);
+  __syncthreads();
+  // exclusive scan from the largest cost down: bins[c] <- number of items of cost > c
+  const int per = (n_bins + 1023) / 1024;
+  const int lo = n_bins - 1 - tid * per;  // this thread's bins: lo, lo - 1, ... (descending cost)
+  int local = 0;
+  for (int k = 0; k < per && lo - k >= 0; ++k) local += bins[lo - k];
+  const int lane = tid & 31, warp = tid >> 5;
+  int x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_tot[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int t = warp_tot[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, t, o);
+      if (lane >= o) t += y;
+    }
+    warp_tot[lane] = t;
+  }
+  __syncthreads();
+  int run = x - local + (warp > 0 ? warp_tot[warp - 1] : 0);
+  for (int k = 0; k < per && lo - k >= 0; ++k) {
+    const int c = bins[lo - k];
+    bins[lo - k] = run;
+    run += c;
+  }
+  __syncthreads();
+  for (int w = tid; w < n_items; w += 1024) order[atomicAdd(&bins[cost(w)], 1)] = w;
+}
+
 __global__ void debug_wait_kernel(unsigned long long timeout_ns, unsigned int* err) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
@@ -119,6 +176,12 @@ sp_status launch_tile_list(const uint8_t* mask, int H, int T, int32_t* row_ptr, 
   tile_scan_kernel<<<1, 1024, 0, stream>>>(counts, rows, row_ptr);
   tile_fill_kernel<<<blocks, 256, 0, stream>>>(mask, rows, T, row_ptr, col_idx);
   return cudaGetLastError() == cudaSuccess ? SP_OK : SP_ERR_CUDA;
+}
+
+bool launch_item_order(const int32_t* row_ptr, int B, int H, int T, int NP, int32_t* order, cudaStream_t stream) {
+  if (2LL * T + 1 > kMaxOrderBins || (long long)B * H * NP > 0x7fffffffLL) return false;  // no order: natural one
+  item_order_kernel<<<1, 1024, 0, stream>>>(row_ptr, B, H, T, NP, order);
+  return cudaGetLastError() == cudaSuccess;
 }
 
 sp_status launch_debug_wait(unsigned long long timeout_ns, cudaStream_t stream) {

@@ -38,7 +38,8 @@ def test_workspace_bytes_arithmetic(L):
     # two fp32 partials of O [1,256,4,64] and LSE [1,4,256], each rounded up to 256 bytes
     assert spattn.sp_attn_fwd_workspace_bytes(1, 256, 4, 64, 2, False) == 2 * 256 * 4 * 64 * 4 + 2 * 4 * 256 * 4
     T = 2
-    mask_bytes = 256 * (-(-(4 * T + 1) * 4 // 256)) + 256 * (-(-(4 * T * T) * 4 // 256)) + 256 * (-(-(4 * T) * 4 // 256))
+    mask_bytes = (256 * (-(-(4 * T + 1) * 4 // 256)) + 256 * (-(-(4 * T * T) * 4 // 256)) + 256 * (-(-(4 * T) * 4 // 256))
+                  + 256 * (-(-(1 * 4 * ((T + 1) // 2)) * 4 // 256)))  # row_ptr, col_idx, counts, work order
     assert spattn.sp_attn_fwd_workspace_bytes(1, 256, 4, 64, 1, True) == mask_bytes
     assert spattn.sp_attn_fwd_workspace_bytes(1, 256, 4, 96, 1, False) == 0  # D must be 64 or 128
 

@@ -67,3 +67,24 @@ def test_empty_item_list_is_a_no_op():
     spattn.sp_attn_fwd_items(q, q, q, o, None, torch.zeros(0, dtype=torch.int32, device="cuda"))
     torch.cuda.synchronize()
     assert torch.all(o == 2.0)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_masked_launch_in_cost_order_equals_natural_order(causal):
+    """sp_attn_fwd with a mask claims its items most kept tiles first; the result is bitwise that of the
+    same items claimed in their natural order (each item's arithmetic does not depend on the order)."""
+    B, S, H, D = 2, 3000, 5, 128
+    q, k, v = (t.cuda() for t in synth.qkv(B, S, H, D, seed=77, scale=0.5))
+    mask = synth.block_mask(H, S, seed=77).cuda()
+    T = (S + 127) // 128
+    NP = (T + 1) // 2
+    o1 = torch.empty_like(q)
+    l1 = torch.empty((B, H, S), device="cuda")
+    spattn.sp_attn_fwd(q, k, v, o1, l1, causal=causal, block_mask=mask)
+    items = torch.arange(B * H * NP, dtype=torch.int32, device="cuda")
+    o2 = torch.full_like(q, float("nan"))
+    l2 = torch.full((B, H, S), float("nan"), device="cuda")
+    spattn.sp_attn_fwd_items(q, k, v, o2, l2, items, causal=causal, block_mask=mask)
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
