@@ -393,6 +393,7 @@ def backward_report(w, q, k, v, reps, stream, peaks, dev):
     import torch
     from sequence_head_attention_b200 import spattn
     hl = w.H // max(1, w.ranks)
+    spattn.sp_set_launch_overlap(0)
     qh, kh, vh = (t[:, :, :hl].contiguous().to(dev) for t in (q, k, v))
     B, S, _, D = qh.shape
     o = torch.empty_like(qh)

@@ -707,9 +707,9 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
 //   o <- (o wa + (O / l) wb) / (wa + wb),   lse <- (c + log2(wa + wb)) ln 2.
 // A row whose running lse is -inf has no running result: its o is not read into the sum (it may hold
 // anything).  A row that saw no key of this block keeps o and lse as they are.
-// Each thread loads its row of the running o into registers before the last P V is awaited (so the loads
-// overlap it), merges it with the block's O from TMEM, and the warp's 32 rows leave as 32 x 32 fp32 boxes
-// through its staging buffers and TMA stores.  Returns false when a wait gave up (the error is recorded).
+// The warp's 32 rows of the running o move as 32 x 32 fp32 boxes: TMA loads into the warp's staging
+// buffers (issued before the last P V is awaited, so they overlap it), the merge in shared memory, TMA
+// stores from the same buffers.  Returns false when a wait gave up (the error is recorded).
 // ------------------------------------------------------------------------------------------------
 template <int D, bool kPair, bool kSplit>
 __device__ __forceinline__ bool merge_epilogue(const AttnParams& p, const TMaps& tm, uint32_t sbase, const Bars& bars,
@@ -717,23 +717,24 @@ __device__ __forceinline__ bool merge_epilogue(const AttnParams& p, const TMaps&
                                                int lane_t, bool row_ok, float l, float m_used, uint32_t total_pv,
                                                uint32_t& stg_ph, volatile int* abort_flag) {
   using C = Cfg<D, kPair, kSplit>;
-  (void)stg_ph;
+  constexpr int kBoxes = D / 32;  // fp32 boxes of 32 columns per row
+  constexpr int kFirst = C::kStgBufs < kBoxes ? C::kStgBufs : kBoxes;
   const uint64_t tmo = p.timeout_ns;
-  // This thread's row of the running result: its lse, and its D fp32 values of O, loaded into registers
-  // (free at this point: the S row is dead) before the last P V is awaited, so the loads overlap it.  A row
-  // with no running result (lse -inf) or past the end is not loaded.
+  const uint32_t stg0 = sbase + C::kStgOff + (uint32_t)warp * (4096u * C::kStgBufs);
+  const CUtensorMap* omap = &tm.o[0];
+  const int row0 = q_row - row + (warp & 3) * 32;
+  if (lane == 0) {
+#pragma unroll
+    for (int c = 0; c < kFirst; ++c) {
+      mbar_arrive_expect_tx(bars.stg_full(warp, c), 4096u);
+      tma_load_4d(stg0 + 4096u * c, omap, bars.stg_full(warp, c), 32 * c, it.h, row0, it.b);
+    }
+  }
+  __syncwarp();
+  uint32_t pending = (1u << kFirst) - 1u;  // staging buffers with a load in flight
+  // Weights of the running result and of this block's rows (no global read yet depends on the MMAs).
   const size_t l_idx = ((size_t)it.b * p.H + it.h) * p.S + q_row;
   const float la = row_ok ? p.lse[l_idx] * 1.4426950408889634f : -INFINITY;
-  float4 acc[D / 4];
-  if (la != -INFINITY) {
-    const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(p.o) +
-                                                        (((size_t)it.b * p.S + q_row) * p.H + it.h) * D);
-#pragma unroll
-    for (int e = 0; e < D / 4; ++e) acc[e] = __ldcs(src + e);
-  } else {
-#pragma unroll
-    for (int e = 0; e < D / 4; ++e) acc[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
   const bool has = l > 0.f && m_used != -INFINITY;
   float wa = 1.f, wb = 0.f, lnew = la;
   if (has) {
@@ -748,50 +749,58 @@ __device__ __forceinline__ bool merge_epilogue(const AttnParams& p, const TMaps&
   }
   bool ok = mbar_wait(bars.pv_done(lane_t), (total_pv - 1) & 1, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err);
   ok = __all_sync(0xffffffffu, ok);
-  if (!ok) return false;
-  tc_fence_after();
-  // Out through the warp's staging buffers and TMA stores, 32 fp32 columns of its 32 rows per box.
-  const uint32_t stg0 = sbase + C::kStgOff + (uint32_t)warp * (4096u * C::kStgBufs);
-  const CUtensorMap* omap = &tm.o[0];
-  const int row0 = q_row - row + (warp & 3) * 32;
+  if (ok) {
+    tc_fence_after();
+#pragma unroll 1
+    for (int c = 0; c < kBoxes; ++c) {
+      const int b = c % C::kStgBufs;
+      const uint32_t stg = stg0 + 4096u * (uint32_t)b;
+      ok = mbar_wait(bars.stg_full(warp, b), (stg_ph >> b) & 1u, tmo, ERR_TIMEOUT_STG, abort_flag, p.err);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      stg_ph ^= 1u << b;
+      pending &= ~(1u << b);
+      uint32_t v[32];
+      tmem_ld32(tO + c * 32, v);
+      tmem_wait_ld();
 #pragma unroll
-  for (int c = 0; c < D / 32; ++c) {
-    uint32_t v[32];
-    tmem_ld32(tO + c * 32, v);
-    tmem_wait_ld();
-    uint32_t r[32];
+      for (int e = 0; e < 8; ++e) {
+        const uint32_t addr = stg + (uint32_t)lane * 128u + (uint32_t)((e ^ (lane & 7)) << 4);
+        uint32_t a[4];
+        ld_shared_v4(addr, a[0], a[1], a[2], a[3]);
+        uint32_t r[4];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float4 a = acc[c * 8 + e];
-      const float av[4] = {a.x, a.y, a.z, a.w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        // wa == 0: the row had no running result; wb == 0: the row saw no key of this block
-        const float x = wa > 0.f ? av[j] * wa : 0.f;
-        const float y = wb > 0.f ? __uint_as_float(v[4 * e + j]) * wb : 0.f;
-        r[4 * e + j] = __float_as_uint(x + y);
+        for (int j = 0; j < 4; ++j) {
+          const float x = wa > 0.f ? __uint_as_float(a[j]) * wa : 0.f;
+          const float y = wb > 0.f ? __uint_as_float(v[4 * e + j]) * wb : 0.f;
+          r[j] = __float_as_uint(x + y);
+        }
+        st_shared_v4(addr, r[0], r[1], r[2], r[3]);
       }
-    }
-    const uint32_t stg = stg0 + 4096u * (uint32_t)(c % C::kStgBufs);
-    if (c >= C::kStgBufs) {  // the store that last used this buffer must have read it
+      fence_proxy_async_smem();
+      __syncwarp();
       if (lane == 0) {
-        if (C::kStgBufs == 2)
-          bulk_wait_read_but1();
-        else
+        tma_store_4d(omap, stg, 32 * c, it.h, row0, it.b);
+        bulk_commit_group();
+        if (c + C::kStgBufs < kBoxes) {  // refill this buffer with a later box once the store has read it
           bulk_wait_read_all();
+          mbar_arrive_expect_tx(bars.stg_full(warp, b), 4096u);
+          tma_load_4d(stg, omap, bars.stg_full(warp, b), 32 * (c + C::kStgBufs), it.h, row0, it.b);
+        }
       }
+      if (c + C::kStgBufs < kBoxes) pending |= 1u << b;
       __syncwarp();
     }
-#pragma unroll
-    for (int e = 0; e < 8; ++e)
-      st_shared_v4(stg + (uint32_t)lane * 128u + (uint32_t)(((e ^ (lane & 7)) << 4)), r[4 * e], r[4 * e + 1],
-                   r[4 * e + 2], r[4 * e + 3]);
-    fence_proxy_async_smem();
-    __syncwarp();
-    if (lane == 0) {
-      tma_store_4d(omap, stg, 32 * c, it.h, row0, it.b);
-      bulk_commit_group();
-    }
+  }
+  if (!ok) {
+    // Leave no load in flight into shared memory: wait (bounded) for every outstanding one.
+#pragma unroll 1
+    for (int b = 0; b < C::kStgBufs; ++b)
+      if (pending & (1u << b)) {
+        warp_mbar_wait(bars.stg_full(warp, b), (stg_ph >> b) & 1u, tmo, ERR_TIMEOUT_STG, nullptr, p.err);
+        stg_ph ^= 1u << b;
+      }
+    return false;
   }
   if (lane == 0) bulk_wait_read_all();  // the buffers are free for the next item
   __syncwarp();

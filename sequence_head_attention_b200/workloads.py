@@ -20,24 +20,8 @@ from __future__ import annotations
 import torch
 
 from . import spattn
+from .dist import rank_chunks  # noqa: F401  (the head chunks of each simulated rank)
 from .synth import TILE, Workload, split_seq
-
-
-def rank_chunks(chunks, H, P):
-    """Split a global head-chunk list at the rank boundaries (multiples of H/P).  Each rank gets the
-    chunks inside its head range; a chunk that straddles a boundary is cut there."""
-    Hl = H // P
-    out = [[] for _ in range(P)]
-    h0 = 0
-    for c in chunks:
-        a, e = h0, h0 + c
-        while a < e:
-            r = a // Hl
-            cut = min(e, (r + 1) * Hl)
-            out[r].append(cut - a)
-            a = cut
-        h0 = e
-    return out
 
 
 class UlyssesStep:
