@@ -62,10 +62,16 @@ constexpr int kSchedSlots = 64;  // launch-rotated work counters
 __device__ unsigned int g_attn_sched[2 * kSchedSlots];
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: O and l are rescaled when m grows by > 2^8
 constexpr uint32_t kPCol = 64;  // P_t (bf16 pairs) lives over the last 64 of S_t's 128 columns
-#ifndef SP_EXP2_POLY_PAIRS
-#define SP_EXP2_POLY_PAIRS 0  // of every 8 pairs of exponentials, this many run on the FMA pipe
+// Of every 8 pairs of exponentials, this many run on the FMA pipe (the rest on the MUFU unit).  Measured on
+// a B200: one in eight speeds split-key launches (one query tile per CTA) by 2-3%, and slows the launches with
+// two query tiles per CTA (6% for CTA pairs), whose softmax warps have no registers to spare.
+#ifdef SP_EXP2_POLY_PAIRS
+template <bool kSplit>
+constexpr int poly_pairs() { return SP_EXP2_POLY_PAIRS; }
+#else
+template <bool kSplit>
+constexpr int poly_pairs() { return kSplit ? 1 : 0; }
 #endif
-constexpr int kPolyPairs = SP_EXP2_POLY_PAIRS;
 
 // kSplit: both lanes work on ONE query tile and take alternate kept key tiles of its list (lane 0 the even
 // ones, lane 1 the odd ones), each with its own running maximum, sum and O; the epilogue merges the two.
@@ -1011,12 +1017,13 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
             if (c * 32 + e >= n_valid) sr[c][e] = __float_as_uint(-INFINITY);
       }
       const f2 sc2 = {scale_log2, scale_log2};
-      // 2^(s * scale - m) for the two columns of pair e of the row (of every 8 pairs, kPolyPairs go through
-      // the FMA-pipe polynomial and the rest through ex2.approx).
+      // 2^(s * scale - m) for the two columns of pair e of the row (of every 8 pairs, kPoly go through the
+      // FMA-pipe polynomial and the rest through ex2.approx).
+      constexpr int kPoly = poly_pairs<kSplit>();
       auto exp_pair = [&](int i, int e, f2 nm2) -> f2 {
         const f2 x = ffma2(f2{SV(i), SV(i + 1)}, sc2, nm2);
         f2 pr;
-        if (((e >> 1) & 7) >= 8 - kPolyPairs) {
+        if (((e >> 1) & 7) >= 8 - kPoly) {
           pr = exp2_poly2(x);
         } else {
           pr.x = ex2_approx(x.x);
