@@ -82,7 +82,8 @@ typedef void* sp_stream;
  * n_kv_blocks > 1 needs n_kv_blocks fp32 partials (O [B,S,H,D] and LSE [B,H,S] each); has_mask != 0
  * needs the compacted tile list (H * ceil(S/128) + 1 row offsets and up to H * ceil(S/128)^2 tile
  * indices, int32) and the launch's work order (B * H * ceil(ceil(S/128) / 2) item ids, int32: a masked
- * launch claims its work items most kept tiles first).  Each section is rounded up to 256 bytes.
+ * launch claims its work items head by head, the heads with the most kept tiles first, and within a head
+ * the items with the most kept tiles first).  Each section is rounded up to 256 bytes.
  * Returns 0 when neither applies, and 0 for invalid sizes.
  */
 SP_API size_t sp_attn_fwd_workspace_bytes(int B, int S, int H, int D, int n_kv_blocks, int has_mask);

@@ -82,30 +82,50 @@ __global__ void __launch_bounds__(256) tile_fill_kernel(const uint8_t* mask, int
 }
 
 // Work order of a block-sparse launch: the item ids (b * H + h) * NP + qp (a pair of query tiles 2 qp and
-// 2 qp + 1 of head h) sorted by their kept tiles, most first, so that the dynamically claimed items of the
-// launch end with the short ones (longest-processing-time order; per-head densities vary several-fold).
-// A counting sort in one block: histogram of the costs (0 .. 2T) in shared memory, exclusive offsets from
-// the largest cost down, then each item placed with a shared-memory atomic (items of equal cost land in any
-// order; each item's arithmetic does not depend on it).
+// 2 qp + 1 of head h), head by head, the heads with the most kept tiles first, and within each (b, h) the
+// items with the most kept tiles first.  Head by head, the CTAs running at the same time work on one or two
+// heads and share their K and V in L2 (sorting every item by its cost, across heads, put all heads in flight
+// at once and multiplied the launch's DRAM reads seven-fold); densest heads first and longest items first
+// within a head, the dynamically claimed last items of the launch are the sparsest head's short ones
+// (longest-processing-time order; per-head densities vary several-fold).  One block per (b, h): its rank
+// among the heads by total kept tiles (ties by id), then a counting sort of its NP items, histogram of the
+// costs (0 .. 2T) in shared memory, exclusive offsets from the largest cost down, each item placed with a
+// shared-memory atomic (items of equal cost land in any order; each item's arithmetic does not depend on it).
 constexpr int kMaxOrderBins = 4096;
-__global__ void __launch_bounds__(1024) item_order_kernel(const int32_t* row_ptr, int B, int H, int T, int NP,
-                                                          int32_t* order) {
+constexpr int kOrderThreads = 256;
+__global__ void __launch_bounds__(kOrderThreads) item_order_kernel(const int32_t* row_ptr, int H, int T, int NP,
+                                                                   int32_t* order) {
   __shared__ int32_t bins[kMaxOrderBins];
-  __shared__ int32_t warp_tot[32];
-  const int n_bins = 2 * T + 1, n_items = B * H * NP, tid = threadIdx.x;
-  auto cost = [&](int w) {
-    const int h = (w / NP) % H, qp = w % NP;
+  __shared__ int32_t warp_tot[kOrderThreads / 32];
+  __shared__ int32_t rank_part[kOrderThreads / 32];
+  const int seg = blockIdx.x, h = seg % H, n_seg = gridDim.x;  // (b, h)
+  const int n_bins = 2 * T + 1, tid = threadIdx.x;
+  // the segment's place among the heads: segments with more kept tiles, or as many and a lower id, go first
+  auto head_total = [&](int hh) { return row_ptr[hh * T + T] - row_ptr[hh * T]; };
+  const int mine = head_total(h);
+  int before = 0;
+  for (int s2 = tid; s2 < n_seg; s2 += kOrderThreads) {
+    const int t2 = head_total(s2 % H);
+    before += (t2 > mine || (t2 == mine && s2 < seg)) ? 1 : 0;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) before += __shfl_xor_sync(0xffffffffu, before, o);
+  if ((tid & 31) == 0) rank_part[tid >> 5] = before;
+  auto cost = [&](int qp) {
     const int r0 = h * T + 2 * qp;
     int c = row_ptr[r0 + 1] - row_ptr[r0];
     if (2 * qp + 1 < T) c += row_ptr[r0 + 2] - row_ptr[r0 + 1];
     return c;
   };
-  for (int i = tid; i < n_bins; i += 1024) bins[i] = 0;
+  for (int i = tid; i < n_bins; i += kOrderThreads) bins[i] = 0;
   __syncthreads();
-  for (int w = tid; w < n_items; w += 1024) atomicAdd(&bins[cost(w)], 1);
+  int rank = 0;
+#pragma unroll
+  for (int w = 0; w < kOrderThreads / 32; ++w) rank += rank_part[w];
+  for (int qp = tid; qp < NP; qp += kOrderThreads) atomicAdd(&bins[cost(qp)], 1);
   __syncthreads();
-  // exclusive scan from the largest cost down: bins[c] <- number of items of cost > c
-  const int per = (n_bins + 1023) / 1024;
+  // exclusive scan from the largest cost down: bins[c] <- number of the segment's items of cost > c
+  const int per = (n_bins + kOrderThreads - 1) / kOrderThreads;
   const int lo = n_bins - 1 - tid * per;  // this thread's bins: lo, lo - 1, ... (descending cost)
   int local = 0;
   for (int k = 0; k < per && lo - k >= 0; ++k) local += bins[lo - k];
@@ -119,13 +139,13 @@ __global__ void __launch_bounds__(1024) item_order_kernel(const int32_t* row_ptr
   if (lane == 31) warp_tot[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int t = warp_tot[lane];
+    int t = lane < kOrderThreads / 32 ? warp_tot[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, t, o);
       if (lane >= o) t += y;
     }
-    warp_tot[lane] = t;
+    if (lane < kOrderThreads / 32) warp_tot[lane] = t;
   }
   __syncthreads();
   int run = x - local + (warp > 0 ? warp_tot[warp - 1] : 0);
@@ -135,7 +155,8 @@ __global__ void __launch_bounds__(1024) item_order_kernel(const int32_t* row_ptr
     run += c;
   }
   __syncthreads();
-  for (int w = tid; w < n_items; w += 1024) order[atomicAdd(&bins[cost(w)], 1)] = w;
+  int32_t* out = order + (size_t)rank * NP;
+  for (int qp = tid; qp < NP; qp += kOrderThreads) out[atomicAdd(&bins[cost(qp)], 1)] = seg * NP + qp;
 }
 
 __global__ void debug_wait_kernel(unsigned long long timeout_ns, unsigned int* err) {
@@ -179,8 +200,10 @@ sp_status launch_tile_list(const uint8_t* mask, int H, int T, int32_t* row_ptr, 
 }
 
 bool launch_item_order(const int32_t* row_ptr, int B, int H, int T, int NP, int32_t* order, cudaStream_t stream) {
-  if (2LL * T + 1 > kMaxOrderBins || (long long)B * H * NP > 0x7fffffffLL) return false;  // no order: natural one
-  item_order_kernel<<<1, 1024, 0, stream>>>(row_ptr, B, H, T, NP, order);
+  if (2LL * T + 1 > kMaxOrderBins || (long long)B * H * NP > 0x7fffffffLL || (long long)B * H > 0x7fffffffLL)
+    return false;  // no order: the natural one
+  if ((long long)B * H * NP == 0) return true;
+  item_order_kernel<<<B * H, kOrderThreads, 0, stream>>>(row_ptr, H, T, NP, order);
   return cudaGetLastError() == cudaSuccess;
 }
 

@@ -71,7 +71,7 @@ def test_empty_item_list_is_a_no_op():
 
 @pytest.mark.parametrize("causal", [False, True])
 def test_masked_launch_in_cost_order_equals_natural_order(causal):
-    """sp_attn_fwd with a mask claims its items most kept tiles first; the result is bitwise that of the
+    """sp_attn_fwd with a mask claims its items in its cost order; the result is bitwise that of the
     same items claimed in their natural order (each item's arithmetic does not depend on the order)."""
     B, S, H, D = 2, 3000, 5, 128
     q, k, v = (t.cuda() for t in synth.qkv(B, S, H, D, seed=77, scale=0.5))
@@ -88,3 +88,37 @@ def test_masked_launch_in_cost_order_equals_natural_order(causal):
     torch.cuda.synchronize()
     assert spattn.sp_check_device_error() == spattn.SP_OK
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_masked_launch_work_order_heads_densest_first_items_longest_first():
+    """The work order a masked sp_attn_fwd writes into its workspace (the last section: B * H * ceil(T / 2)
+    item ids) is a permutation of the items that keeps each (b, h)'s items together, takes the (b, h) in
+    order of their head's kept tiles, most first (ties: lower b * H + h first), and within a (b, h) runs from
+    the item with the most kept tiles to the fewest (cost of item (b, h, qp) = kept tiles of query-tile rows
+    2 qp and 2 qp + 1 of head h's mask)."""
+    B, S, H, D = 2, 3000, 5, 128
+    T = (S + 127) // 128
+    NP = (T + 1) // 2
+    q, k, v = (t.cuda() for t in synth.qkv(B, S, H, D, seed=78, scale=0.5))
+    mask = synth.block_mask(H, S, seed=78)
+    ws_bytes = spattn.sp_attn_fwd_workspace_bytes(B, S, H, D, 1, True)
+    ws = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, S), device="cuda")
+    spattn.sp_attn_fwd(q, k, v, o, lse, block_mask=mask.cuda(), workspace=ws)
+    torch.cuda.synchronize()
+    assert spattn.sp_check_device_error() == spattn.SP_OK
+    n = B * H * NP
+    off = ws_bytes - (n * 4 + 255) // 256 * 256
+    order = ws[off:off + 4 * n].cpu().view(torch.int32).numpy()
+    assert sorted(order.tolist()) == list(range(n))
+    rows = (mask != 0).sum(dim=2).numpy()  # kept tiles per (head, query-tile row)
+    total = rows.sum(axis=1)
+    segs = sorted(range(B * H), key=lambda sg: (-int(total[sg % H]), sg))
+    assert len(set(total.tolist())) > 1  # the heads' order is not the natural one by accident
+    for r, seg in enumerate(segs):
+        ids = order[r * NP:(r + 1) * NP]
+        assert set((ids // NP).tolist()) == {seg}
+        h = seg % H
+        cost = [int(rows[h, 2 * qp]) + (int(rows[h, 2 * qp + 1]) if 2 * qp + 1 < T else 0) for qp in ids % NP]
+        assert all(a >= b for a, b in zip(cost, cost[1:])), cost
