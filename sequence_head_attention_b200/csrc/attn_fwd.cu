@@ -90,18 +90,18 @@ struct Cfg {
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = kQTiles * kTileBytes;
   static constexpr int kBarOff = kKVOff + kStages * kKVBytes;
-  // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2], drain, 8-byte
-  // slots for the o_done[2] counters, and stg_full[8][2] (a merging epilogue's loads of the running O into
-  // each softmax warp's staging buffers)
-  static constexpr int kNumBars = 2 + 2 * kStages + 9 + 16;
+  // barriers: q_full, q_empty, kv_full[S], kv_empty[S], s_full[2], p_full[2], pv_done[2], drain, and
+  // stg_full[8][2] (a merging epilogue's loads of the running O into each softmax warp's staging buffers)
+  static constexpr int kNumBars = 2 + 2 * kStages + 7 + 16;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   // misc: TMEM base, abort flag, published-item count, per-warp item-read counts, the item ring (96
-  // bytes); with kSplit also the lanes' exchange: one 8-byte slot per query row (lane 1 posts its row
-  // maximum and sum, lane 0 answers with both lanes' weights) and four hand-off counters, one per TMEM
-  // lane quadrant.
-  static constexpr int kXchOff = kMiscOff + 96;
+  // bytes); the O read-out progress words, 8 per lane (64 bytes); with kSplit also the lanes' exchange:
+  // one 8-byte slot per query row (lane 1 posts its row maximum and sum, lane 0 answers with both lanes'
+  // weights) and four hand-off counters, one per TMEM lane quadrant.
+  static constexpr int kProgOff = kMiscOff + 96;
+  static constexpr int kXchOff = kMiscOff + 160;
   static constexpr int kXcntOff = kXchOff + 128 * 8;
-  static constexpr int kMiscBytes = kSplit ? 96 + 128 * 8 + 16 : 96;
+  static constexpr int kMiscBytes = kSplit ? 160 + 128 * 8 + 16 : 160;
   // then, 1024-aligned, staging for the O stores: per softmax warp two 4 KB buffers (32 rows x 128 bytes)
   // where they fit in the 227 KB a CTA may have, else one
   static constexpr int kStgOff = (kMiscOff + kMiscBytes + 1023) / 1024 * 1024;
@@ -111,9 +111,10 @@ struct Cfg {
   static constexpr uint32_t kIdescS = idesc_bf16_f32(kM, 128, false, false);
   static constexpr uint32_t kIdescPV = idesc_bf16_f32(kM, D, false, true);
   static constexpr uint32_t kRowWarps = kPair ? 8u : 4u;  // softmax warps per lane over the (pair of) CTAs
-  // o_done[t] counts, per item, the softmax warps that have read out O_t: lane t's (kRowWarps), or with
-  // kSplit every softmax warp of the CTA, since each reads both lanes' O for its half of the columns
-  static constexpr uint32_t kODoneWarps = kSplit ? 8u : kRowWarps;
+  // The softmax warps whose read-out of O_t an item's first P V into O_t waits for: lane t's (kRowWarps),
+  // or with kSplit every softmax warp of the CTA, since each reads both lanes' O for its half of the columns.
+  // Each has a progress word of its own, the number of items whose epilogue it has finished.
+  static constexpr uint32_t kProgWords = kSplit ? 8u : kRowWarps;
   static constexpr uint32_t kColS = 0;
   static constexpr uint32_t kColO = 256;
 };
@@ -125,7 +126,7 @@ static_assert(Cfg<128, true>::kSmemBytes <= 232448 && Cfg<128, false>::kSmemByte
               "shared memory");
 
 struct Bars {
-  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, pv_done0, o_done0, drain, stg_full0;
+  uint32_t q_full, q_empty, kv_full0, kv_empty0, s_full0, p_full0, pv_done0, drain, stg_full0, prog0;
   // stg_full[w][b]: staging buffer b of softmax warp w holds the running O loaded for a merge
   __device__ uint32_t stg_full(int w, int b) const { return stg_full0 + 8u * (2 * w + b); }
   __device__ uint32_t kv_full(int s) const { return kv_full0 + 8u * s; }
@@ -133,8 +134,10 @@ struct Bars {
   __device__ uint32_t s_full(int t) const { return s_full0 + 8u * t; }
   __device__ uint32_t p_full(int t) const { return p_full0 + 8u * t; }
   __device__ uint32_t pv_done(int t) const { return pv_done0 + 8u * t; }
-  // o_done[t]: a counter, +1 per softmax warp of lane t per finished item (epilogue reads of O done)
-  __device__ uint32_t o_done(int t) const { return o_done0 + 8u * t; }
+  // prog(t, k): progress word k of lane t (rank 0's shared memory for a pair): the items whose epilogue,
+  // and so whose read-out of O_t, softmax warp k has finished.  A word per warp, not one shared count: a
+  // warp with nothing to read out may finish two items before another has finished one.
+  __device__ uint32_t prog(int t, int k) const { return prog0 + 4u * (8u * t + k); }
 };
 
 struct Item {
@@ -580,7 +583,7 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
     if (!ok) break;
     tc_fence_after();
     // O_t may be overwritten by this item's first P V only after the softmax warps of lane t (4, or 8 over
-    // a pair) have read out the previous item's O: o_done[t] counts one per warp and finished item.
+    // a pair) have read out the previous item's O: each one's progress word has reached this item.
     bool need_odone = n_item > 0;
     bool first_pv = true;
     StepIter st;
@@ -596,9 +599,12 @@ __device__ void run_mma(const AttnParams& p, uint8_t* smem, const Bars& bars, co
       bool good = warp_mbar_wait(bars.kv_full(vs), (pend_v_pos / C::kStages) & 1, tmo, ERR_TIMEOUT_KV_FULL,
                                  abort_flag, p.err);
       if (good && need_odone) {
-        const uint32_t target = C::kODoneWarps * (uint32_t)n_item;
-        good = kPair ? warp_counter_wait_cluster(bars.o_done(t), target, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err)
-                     : warp_counter_wait(bars.o_done(t), target, tmo, ERR_TIMEOUT_O_FREE, abort_flag, p.err);
+#pragma unroll 1
+        for (uint32_t k = 0; k < C::kProgWords && good; ++k)
+          good = kPair ? warp_counter_wait_cluster(bars.prog(t, k), (uint32_t)n_item, tmo, ERR_TIMEOUT_O_FREE,
+                                                   abort_flag, p.err)
+                       : warp_counter_wait(bars.prog(t, k), (uint32_t)n_item, tmo, ERR_TIMEOUT_O_FREE, abort_flag,
+                                           p.err);
         need_odone = false;
       }
       if (good) {
@@ -951,6 +957,132 @@ __device__ __forceinline__ void rescale_o_row(uint32_t tO, float alpha) {
   }
 }
 
+// The epilogue of one item for one softmax warp (O / l and lse of its 32 rows, or their merge into a running
+// result), then the warp's progress word.  Returns false when a wait gave up (the error is recorded).
+// (Measured on a B200: out of line, as a called function, every launch was 3-8% slower.)
+template <int D, bool kPair, bool kSplit>
+__device__ __forceinline__ bool item_epilogue(const AttnParams& p, const TMaps& tm, uint32_t sbase, const Bars& bars,
+                                           uint32_t trow, uint32_t tO, int warp, int lane, int row, int lane_t,
+                                           bool remote, uint32_t prog_word, uint32_t& n_fin, uint32_t& stg_ph,
+                                           uint32_t& n_xch,
+                                           volatile int* abort_flag, const Item& it, float l, float m_used,
+                                           int n_kept, uint32_t total_pv) {
+  using C = Cfg<D, kPair, kSplit>;
+  const uint64_t tmo = p.timeout_ns;
+  bool ok = true;
+  const int q_row = (lane_t ? it.q_start[1] : it.q_start[0]) + row;
+  const bool lane_valid = lane_t ? it.valid[1] : it.valid[0];
+  // Overlapped launch: nothing is written (or, merging, read) before the kernel before it has completed,
+  // unless the caller promised that kernel touches none of this launch's outputs.
+  if (p.pdl_wait_epi) pdl_wait();
+  // Epilogue: O / l and lse for the rows of this lane.
+  if (kSplit && lane_valid) {
+    ok = split_epilogue<D>(p, tm, sbase, bars, trow, it, q_row, row, warp, lane, lane_t, q_row < it.q_end, l, m_used,
+                           n_kept, total_pv, n_xch, abort_flag);
+    ++n_xch;
+    if (!ok) return false;
+  } else if (lane_valid) {
+    const bool row_ok = q_row < it.q_end;  // inside S and inside the pair's shard
+    void* obase = p.o;
+    int orow = q_row, orows = p.S;
+    if (p.n_shards > 1) {  // the pair's sequence shard
+      obase = p.o_shard[it.shard];
+      orow = q_row - it.shard * p.shard_rows;
+      orows = p.shard_rows;
+    }
+    const size_t o_idx = (((size_t)it.b * orows + orow) * p.H + it.h) * D;
+    if (p.o_merge) {
+      // Merge into the running result: rows that saw no key of this launch's range keep it unchanged.
+      if (n_kept > 0) {
+        ok = merge_epilogue<D, kPair, kSplit>(p, tm, sbase, bars, tO, it, q_row, row, warp, lane, lane_t, row_ok, l,
+                                      m_used, total_pv, stg_ph, abort_flag);
+        if (!ok) return false;
+      }
+    } else if (n_kept > 0) {
+      ok = mbar_wait(bars.pv_done(lane_t), (total_pv - 1) & 1, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) return false;
+      tc_fence_after();
+      // A row that never saw a visible key is exactly 0 (the FMA-pipe exponentials of its masked
+      // entries are tiny but not zero).
+      const float inv_l = (l > 0.f && m_used != -INFINITY) ? 1.f / l : 0.f;
+      // O / l leaves through a per-warp staging buffer in shared memory, 128 bytes of each of the warp's
+      // 32 rows at a time (32 fp32 or 64 bf16 values, 128-byte swizzle), and a TMA store of that box:
+      // whole 128-byte lines reach L2, and rows past the shard's (or S's) end are not written.
+      const uint32_t stg0 = sbase + C::kStgOff + (uint32_t)warp * (4096u * C::kStgBufs);
+      const CUtensorMap* omap = &tm.o[p.n_shards > 1 ? it.shard : 0];
+      const int row0 = q_row - row + (warp & 3) * 32 - (p.n_shards > 1 ? it.shard * p.shard_rows : 0);
+      const int n_chunks = p.o_f32 ? D / 32 : D / 64;
+#pragma unroll 1
+      for (int c = 0; c < n_chunks; ++c) {
+        uint32_t v[32];
+        if (p.o_f32) {
+          tmem_ld32(tO + c * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv_l);
+        } else {
+          uint32_t o2[32];
+          tmem_ld32(tO + c * 64, v);
+          tmem_ld32(tO + c * 64 + 32, o2);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            v[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv_l, __uint_as_float(v[2 * e + 1]) * inv_l);
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            v[16 + e] = pack_bf16x2(__uint_as_float(o2[2 * e]) * inv_l, __uint_as_float(o2[2 * e + 1]) * inv_l);
+        }
+        const uint32_t stg = stg0 + 4096u * (uint32_t)(c % C::kStgBufs);
+        if (c >= C::kStgBufs) {  // the store that last used this buffer must have read it
+          if (lane == 0) {
+            if (C::kStgBufs == 2)
+              bulk_wait_read_but1();
+            else
+              bulk_wait_read_all();
+          }
+          __syncwarp();
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          st_shared_v4(stg + (uint32_t)lane * 128u + (uint32_t)(((e ^ (lane & 7)) << 4)), v[4 * e], v[4 * e + 1],
+                       v[4 * e + 2], v[4 * e + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_4d(omap, stg, c * (p.o_f32 ? 32 : 64), it.h, row0, it.b);
+          bulk_commit_group();
+        }
+      }
+      if (lane == 0) bulk_wait_read_all();  // the buffers are free for the next item
+      __syncwarp();
+    } else if (row_ok) {
+      if (p.o_f32) {
+        float4* dst = reinterpret_cast<float4*>(static_cast<float*>(obase) + o_idx);
+        for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(obase) + o_idx);
+        for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    if (row_ok && p.lse && !p.o_merge)
+      p.lse[((size_t)it.b * p.H + it.h) * p.S + q_row] =
+          (l > 0.f && m_used != -INFINITY) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
+  }
+  // This warp has read out O (with kSplit, both lanes' O): its progress word moves on to the next item.
+  tc_fence_before();
+  __syncwarp();
+  ++n_fin;
+  if (lane == 0) {
+    if (remote)
+      st_release_cluster(prog_word, n_fin);
+    else
+      st_release_cta(prog_word, n_fin);
+    if (kSplit) st_release_cta(bars.prog(lane_t ^ 1, warp), n_fin);
+  }
+  return true;
+}
+
 // ------------------------------------------------------------------------------------------------
 // Softmax + epilogue: 4 warps per lane, one query row per thread.
 // ------------------------------------------------------------------------------------------------
@@ -958,10 +1090,14 @@ template <int D, bool kPair, bool kSplit>
 __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase, const Bars& bars, const ItemRing& ir,
                             uint32_t tmem, int lane_t, volatile int* abort_flag) {
   using C = Cfg<D, kPair, kSplit>;
-  // A pair's rank 1 hands its P and its O read-outs to rank 0's barriers and counters.
+  // A pair's rank 1 hands its P and its O read-outs to rank 0's barriers and progress words.
   const bool remote = kPair && cluster_rank() != 0;
   const uint32_t p_full_bar = remote ? map_shared(bars.p_full(lane_t), 0) : bars.p_full(lane_t);
-  const uint32_t o_done_ctr = remote ? map_shared(bars.o_done(lane_t), 0) : bars.o_done(lane_t);
+  // this warp's progress word for lane t: pair, 4 per CTA; split, one per warp of the CTA
+  const int prog_k = kPair ? 4 * (int)cluster_rank() + ((threadIdx.x >> 5) & 3)
+                           : (kSplit ? (int)(threadIdx.x >> 5) : (int)((threadIdx.x >> 5) & 3));
+  const uint32_t prog_word = remote ? map_shared(bars.prog(lane_t, prog_k), 0) : bars.prog(lane_t, prog_k);
+  uint32_t n_fin = 0;  // items whose epilogue this warp has finished
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -976,6 +1112,25 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
   uint32_t stg_ph = 0;  // bit b: phase of this warp's staging-buffer-b load barrier (merging epilogues)
   uint32_t n_xch = 0;   // split keys: epilogue hand-offs this warp has taken part in
   bool ok = true;
+  // Split-key launches (block-sparse, items of few kept tiles) run an item's epilogue after this warp's
+  // first kept step of the next item (S to P touch only the S columns, not O): the tensor core then has
+  // that step's P V queued by the time O has been read out, and the step no longer waits behind the
+  // epilogue.  Measured on a B200: block-sparse +4.7%; dense and causal launches -5 to -9% (the state kept
+  // through the step loop costs their softmax registers), so they finish each item at once.
+  constexpr bool kDefer = kSplit;
+  int prev_w = -1;  // kDefer: the item whose epilogue is pending, or -1
+  float prev_l = 0.f, prev_m = -INFINITY;
+  int prev_kept = 0;
+  uint32_t prev_pv = 0;
+  auto epilogue = [&](const Item& it_, float l_, float m_, int kept_, uint32_t pv_) -> bool {
+    return item_epilogue<D, kPair, kSplit>(p, tm, sbase, bars, trow, tO, warp, lane, row, lane_t, remote, prog_word,
+                                           n_fin, stg_ph, n_xch, abort_flag, it_, l_, m_, kept_, pv_);
+  };
+  auto finish = [&]() -> bool {  // the pending epilogue
+    const Item it_ = decode_item<kPair, kSplit>(p, prev_w);
+    prev_w = -1;
+    return epilogue(it_, prev_l, prev_m, prev_kept, prev_pv);
+  };
 
   for (int n_item = 0;; ++n_item) {
     int w;
@@ -987,7 +1142,6 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
     StepIter st;
     st.init(p, it, kSplit);
     const int q_row = (lane_t ? it.q_start[1] : it.q_start[0]) + row;
-    const bool lane_valid = lane_t ? it.valid[1] : it.valid[0];
     const int lim_row = p.causal ? min(p.kv_lim, q_row + 1) : p.kv_lim;
     float m_used = -INFINITY;  // running maximum of the scaled scores, log2 units
     float l = 0.f;             // running sum of exp2(score - m_used)
@@ -1133,114 +1287,31 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
       }
       ++n_kept;
       ++total_pv;
-    }
-    if (!ok) break;
-    // Overlapped launch: nothing is written (or, merging, read) before the kernel before it has completed,
-    // unless the caller promised that kernel touches none of this launch's outputs.
-    if (p.pdl_wait_epi) pdl_wait();
-    // Epilogue: O / l and lse for the rows of this lane.
-    if (kSplit && lane_valid) {
-      ok = split_epilogue<D>(p, tm, sbase, bars, trow, it, q_row, row, warp, lane, lane_t, q_row < it.q_end, l, m_used,
-                             n_kept, total_pv, n_xch, abort_flag);
-      ++n_xch;
-      if (!ok) break;
-    } else if (lane_valid) {
-      const bool row_ok = q_row < it.q_end;  // inside S and inside the pair's shard
-      void* obase = p.o;
-      int orow = q_row, orows = p.S;
-      if (p.n_shards > 1) {  // the pair's sequence shard
-        obase = p.o_shard[it.shard];
-        orow = q_row - it.shard * p.shard_rows;
-        orows = p.shard_rows;
-      }
-      const size_t o_idx = (((size_t)it.b * orows + orow) * p.H + it.h) * D;
-      if (p.o_merge) {
-        // Merge into the running result: rows that saw no key of this launch's range keep it unchanged.
-        if (n_kept > 0) {
-          ok = merge_epilogue<D, kPair, kSplit>(p, tm, sbase, bars, tO, it, q_row, row, warp, lane, lane_t, row_ok, l,
-                                        m_used, total_pv, stg_ph, abort_flag);
+      if constexpr (kDefer) {
+        if (prev_w >= 0) {  // the previous item's epilogue, now that this step's P is handed over
+          ok = finish();
           if (!ok) break;
         }
-      } else if (n_kept > 0) {
-        ok = mbar_wait(bars.pv_done(lane_t), (total_pv - 1) & 1, tmo, ERR_TIMEOUT_PV_DONE, abort_flag, p.err);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        tc_fence_after();
-        // A row that never saw a visible key is exactly 0 (the FMA-pipe exponentials of its masked
-        // entries are tiny but not zero).
-        const float inv_l = (l > 0.f && m_used != -INFINITY) ? 1.f / l : 0.f;
-        // O / l leaves through a per-warp staging buffer in shared memory, 128 bytes of each of the warp's
-        // 32 rows at a time (32 fp32 or 64 bf16 values, 128-byte swizzle), and a TMA store of that box:
-        // whole 128-byte lines reach L2, and rows past the shard's (or S's) end are not written.
-        const uint32_t stg0 = sbase + C::kStgOff + (uint32_t)warp * (4096u * C::kStgBufs);
-        const CUtensorMap* omap = &tm.o[p.n_shards > 1 ? it.shard : 0];
-        const int row0 = q_row - row + (warp & 3) * 32 - (p.n_shards > 1 ? it.shard * p.shard_rows : 0);
-        const int n_chunks = p.o_f32 ? D / 32 : D / 64;
-#pragma unroll 1
-        for (int c = 0; c < n_chunks; ++c) {
-          uint32_t v[32];
-          if (p.o_f32) {
-            tmem_ld32(tO + c * 32, v);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * inv_l);
-          } else {
-            uint32_t o2[32];
-            tmem_ld32(tO + c * 64, v);
-            tmem_ld32(tO + c * 64 + 32, o2);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              v[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv_l, __uint_as_float(v[2 * e + 1]) * inv_l);
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              v[16 + e] = pack_bf16x2(__uint_as_float(o2[2 * e]) * inv_l, __uint_as_float(o2[2 * e + 1]) * inv_l);
-          }
-          const uint32_t stg = stg0 + 4096u * (uint32_t)(c % C::kStgBufs);
-          if (c >= C::kStgBufs) {  // the store that last used this buffer must have read it
-            if (lane == 0) {
-              if (C::kStgBufs == 2)
-                bulk_wait_read_but1();
-              else
-                bulk_wait_read_all();
-            }
-            __syncwarp();
-          }
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-            st_shared_v4(stg + (uint32_t)lane * 128u + (uint32_t)(((e ^ (lane & 7)) << 4)), v[4 * e], v[4 * e + 1],
-                         v[4 * e + 2], v[4 * e + 3]);
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_4d(omap, stg, c * (p.o_f32 ? 32 : 64), it.h, row0, it.b);
-            bulk_commit_group();
-          }
-        }
-        if (lane == 0) bulk_wait_read_all();  // the buffers are free for the next item
-        __syncwarp();
-      } else if (row_ok) {
-        if (p.o_f32) {
-          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(obase) + o_idx);
-          for (int e = 0; e < D / 4; ++e) dst[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(obase) + o_idx);
-          for (int e = 0; e < D / 8; ++e) dst[e] = make_uint4(0u, 0u, 0u, 0u);
-        }
       }
-      if (row_ok && p.lse && !p.o_merge)
-        p.lse[((size_t)it.b * p.H + it.h) * p.S + q_row] =
-            (l > 0.f && m_used != -INFINITY) ? (m_used + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) {
-      if (remote)
-        counter_add_cluster(o_done_ctr, 1u);
-      else
-        smem_counter_add_release(o_done_ctr, 1u);
-      if (kSplit) smem_counter_add_release(bars.o_done(lane_t ^ 1), 1u);  // it also read the other lane's O
+    if (!ok) break;
+    if constexpr (kDefer) {
+      if (prev_w >= 0) {  // the previous item's epilogue is pending and this item kept no step here
+        ok = finish();
+        if (!ok) break;
+      }
+      prev_w = w;
+      prev_l = l;
+      prev_m = m_used;
+      prev_kept = n_kept;
+      prev_pv = total_pv;
+    } else {
+      ok = epilogue(it, l, m_used, n_kept, total_pv);
+      if (!ok) break;
     }
+  }
+  if constexpr (kDefer) {
+    if (ok && prev_w >= 0) finish();
   }
   if (lane == 0) bulk_wait_all();  // every O store of this warp has landed before the CTA exits
   __syncwarp();
@@ -1261,9 +1332,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   bars.s_full0 = bars.kv_empty0 + 8 * C::kStages;
   bars.p_full0 = bars.s_full0 + 16;
   bars.pv_done0 = bars.p_full0 + 16;
-  bars.o_done0 = bars.pv_done0 + 16;
-  bars.drain = bars.o_done0 + 16;
+  bars.drain = bars.pv_done0 + 16;
   bars.stg_full0 = bars.drain + 8;
+  bars.prog0 = smem_u32(smem + C::kProgOff);
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::kMiscOff + 4);
   ItemRing ir;
@@ -1285,8 +1356,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bars.p_full(t), C::kRowWarps);  // one arrival per softmax warp of the lane (pair: both CTAs)
       mbar_init(bars.pv_done(t), 1);
     }
-    for (int k = 0; k < 2; ++k)  // o_done[0..1] counters
-      *reinterpret_cast<volatile uint32_t*>(smem + C::kBarOff + (bars.o_done0 - bar0) + 8 * k) = 0u;
+    for (int k = 0; k < 16; ++k)  // the progress words of both lanes
+      *reinterpret_cast<volatile uint32_t*>(smem + C::kProgOff + 4 * k) = 0u;
     mbar_init(bars.drain, 2);
     for (int k = 0; k < 16; ++k) mbar_init(bars.stg_full0 + 8u * k, 1);
     if (kSplit)  // the lanes' epilogue hand-off counters
