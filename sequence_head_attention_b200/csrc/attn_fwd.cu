@@ -1115,7 +1115,7 @@ __device__ void run_softmax(const AttnParams& p, const TMaps& tm, uint32_t sbase
   // Split-key launches (block-sparse, items of few kept tiles) run an item's epilogue after this warp's
   // first kept step of the next item (S to P touch only the S columns, not O): the tensor core then has
   // that step's P V queued by the time O has been read out, and the step no longer waits behind the
-  // epilogue.  Measured on a B200: block-sparse +4.7%; dense and causal launches -5 to -9% (the state kept
+  // epilogue.  Measured on a B200: block-sparse +5.8%; dense and causal launches -5 to -9% (the state kept
   // through the step loop costs their softmax registers), so they finish each item at once.
   constexpr bool kDefer = kSplit;
   int prev_w = -1;  // kDefer: the item whose epilogue is pending, or -1
